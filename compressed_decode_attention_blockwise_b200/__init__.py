@@ -1,0 +1,23 @@
+"""Block-DCT int8 KV-cache codec and coefficient-domain decode attention for
+NVIDIA B200 (sm_100a).
+
+The compute lives in ``libfc.so`` (C ABI declared in ``include/fc.h``);
+``_lib`` is its ctypes binding and ``archive`` the host bookkeeping of one
+layer's compressed K/V streams (raw tail, capacity-doubling archive).
+"""
+
+from . import _lib
+from ._lib import (FcArchive, FcError, FcTail, fc_append_step,
+                   fc_archive_copy_prefix, fc_combine, fc_compress_blocks,
+                   fc_decode_attention, fc_decode_plan,
+                   fc_decode_workspace_bytes, fc_status_string,
+                   fc_storage_bytes, fc_workspace_status)
+from .archive import CodecKVCache, CodecStream, grown_capacity
+
+__all__ = [
+    "CodecKVCache", "CodecStream", "grown_capacity", "FcArchive", "FcTail",
+    "FcError", "fc_compress_blocks", "fc_append_step",
+    "fc_archive_copy_prefix", "fc_decode_plan", "fc_decode_workspace_bytes",
+    "fc_decode_attention", "fc_combine", "fc_workspace_status",
+    "fc_storage_bytes", "fc_status_string",
+]

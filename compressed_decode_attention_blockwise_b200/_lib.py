@@ -1,0 +1,243 @@
+"""Thin ctypes binding of libfc (``include/fc.h``).
+
+Argument marshalling only: tensors become device pointers, element strides
+and the current CUDA stream; every computation runs in libfc's kernels. A
+missing library is an error, never a fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfc.so")
+
+FC_OK = 0
+FC_ERR_INVALID = 1
+FC_ERR_UNSUPPORTED = 2
+FC_ERR_CAPACITY = 3
+FC_ERR_CUDA = 4
+FC_ERR_DEVICE = 5
+
+FC_DTYPE_F32 = 0
+FC_DTYPE_BF16 = 1
+FC_DTYPE_I8 = 2
+
+_DTYPE_CODE = {torch.float32: FC_DTYPE_F32, torch.bfloat16: FC_DTYPE_BF16,
+               torch.int8: FC_DTYPE_I8}
+
+# Every symbol include/fc.h declares.
+EXPORTS = (
+    "fc_compress_blocks", "fc_append_step", "fc_archive_copy_prefix",
+    "fc_decode_plan", "fc_decode_workspace_bytes", "fc_decode_attention",
+    "fc_combine", "fc_workspace_status", "fc_storage_bytes",
+    "fc_status_string",
+)
+
+
+class FcError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s failed: %s (status %d)"
+                         % (where, fc_status_string(status), status))
+
+
+class FcArchive(ctypes.Structure):
+    _fields_ = [
+        ("coeffs", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+        ("coeff_dtype", ctypes.c_int32), ("R", ctypes.c_int32),
+        ("S", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("B", ctypes.c_int64), ("H", ctypes.c_int64), ("D", ctypes.c_int64),
+        ("capacity", ctypes.c_int64), ("n_blocks", ctypes.c_int64),
+        ("coeff_stride_b", ctypes.c_int64), ("coeff_stride_h", ctypes.c_int64),
+        ("scale_stride_b", ctypes.c_int64), ("scale_stride_h", ctypes.c_int64),
+    ]
+
+
+class FcTail(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p), ("dtype", ctypes.c_int32),
+        ("len", ctypes.c_int32), ("stride_b", ctypes.c_int64),
+        ("stride_h", ctypes.c_int64),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libfc.so from the package directory (raises if it is missing)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            "libfc.so is missing at %s: build it with `python -m "
+            "compressed_decode_attention_blockwise_b200.build`" % LIB_PATH)
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    I32 = ctypes.c_int32
+    I64 = ctypes.c_int64
+    PI64 = ctypes.POINTER(ctypes.c_int64)
+    PA = ctypes.POINTER(FcArchive)
+    PT = ctypes.POINTER(FcTail)
+    sig = {
+        "fc_compress_blocks": (ctypes.c_int, [P, I32, PI64, I64, PA, PT, P]),
+        "fc_append_step": (ctypes.c_int, [P, P, I32, PI64, PI64, PA, PA, PT,
+                                          PT, P]),
+        "fc_archive_copy_prefix": (ctypes.c_int, [PA, PA, P]),
+        "fc_decode_plan": (ctypes.c_int, [PA, PT, I64,
+                                          ctypes.POINTER(ctypes.c_int32)]),
+        "fc_decode_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I32]),
+        "fc_decode_attention": (ctypes.c_int, [P, I32, PI64, I64, PA, PA, PT,
+                                               PT, ctypes.c_float, I32, I32,
+                                               P, ctypes.c_size_t, P, I32,
+                                               PI64, P]),
+        "fc_combine": (ctypes.c_int, [P, ctypes.c_size_t, I64, I64, I64, I32,
+                                      P, I32, PI64, P]),
+        "fc_workspace_status": (ctypes.c_int, [P, ctypes.c_size_t,
+                                               ctypes.POINTER(ctypes.c_uint32),
+                                               P]),
+        "fc_storage_bytes": (ctypes.c_int64, [PA, PT]),
+        "fc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def fc_status_string(status: int) -> str:
+    return load().fc_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != FC_OK:
+        raise FcError(status, where)
+
+
+def dtype_code(dt: torch.dtype) -> int:
+    try:
+        return _DTYPE_CODE[dt]
+    except KeyError:
+        raise ValueError("unsupported dtype %s" % dt) from None
+
+
+def _strides4(t: torch.Tensor):
+    if t.dim() != 4:
+        raise ValueError("expected a 4-d tensor, got shape %s"
+                         % (tuple(t.shape),))
+    return (ctypes.c_int64 * 4)(*t.stride())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, *tensors):
+    """cudaStream_t handle: the given stream or torch's current one."""
+    if stream is not None:
+        return ctypes.c_void_p(int(getattr(stream, "cuda_stream", stream)))
+    for t in tensors:
+        if t is not None and t.is_cuda:
+            return ctypes.c_void_p(torch.cuda.current_stream(t.device)
+                                   .cuda_stream)
+    return ctypes.c_void_p(0)
+
+
+def _ref(x):
+    return None if x is None else ctypes.byref(x)
+
+
+# ------------------------------------------------------------------ calls
+
+def fc_compress_blocks(x: torch.Tensor, arc: FcArchive,
+                       tail: Optional[FcTail] = None, stream=None) -> None:
+    st = load().fc_compress_blocks(_ptr(x), dtype_code(x.dtype), _strides4(x),
+                                   x.shape[2], ctypes.byref(arc), _ref(tail),
+                                   _stream(stream, x))
+    _check(st, "fc_compress_blocks")
+
+
+def fc_append_step(k_new: torch.Tensor, v_new: torch.Tensor, ka: FcArchive,
+                   va: FcArchive, kt: FcTail, vt: FcTail, stream=None) -> None:
+    if k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must share a dtype")
+    st = load().fc_append_step(_ptr(k_new), _ptr(v_new),
+                               dtype_code(k_new.dtype), _strides4(k_new),
+                               _strides4(v_new), ctypes.byref(ka),
+                               ctypes.byref(va), ctypes.byref(kt),
+                               ctypes.byref(vt), _stream(stream, k_new))
+    _check(st, "fc_append_step")
+
+
+def fc_archive_copy_prefix(src: FcArchive, dst: FcArchive,
+                           stream=None, device=None) -> None:
+    s = _stream(stream) if stream is not None or device is None else \
+        ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = load().fc_archive_copy_prefix(ctypes.byref(src), ctypes.byref(dst),
+                                       s)
+    _check(st, "fc_archive_copy_prefix")
+
+
+def fc_decode_plan(ka: FcArchive, kt: Optional[FcTail], Hq: int) -> int:
+    out = ctypes.c_int32(0)
+    st = load().fc_decode_plan(ctypes.byref(ka), _ref(kt), int(Hq),
+                               ctypes.byref(out))
+    _check(st, "fc_decode_plan")
+    return int(out.value)
+
+
+def fc_decode_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
+    return int(load().fc_decode_workspace_bytes(int(B), int(Hq), int(D),
+                                                int(num_splits)))
+
+
+def fc_decode_attention(q: torch.Tensor, ka: FcArchive, va: FcArchive,
+                        kt: Optional[FcTail], vt: Optional[FcTail],
+                        out: torch.Tensor, workspace: Optional[torch.Tensor],
+                        softmax_scale: float = 0.0, num_splits: int = 0,
+                        fuse_combine: bool = True, stream=None) -> None:
+    ws_ptr = _ptr(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * \
+        workspace.element_size()
+    st = load().fc_decode_attention(
+        _ptr(q), dtype_code(q.dtype), _strides4(q), q.shape[1],
+        ctypes.byref(ka), ctypes.byref(va), _ref(kt), _ref(vt),
+        float(softmax_scale), int(num_splits), 1 if fuse_combine else 0,
+        ws_ptr, ws_bytes, _ptr(out), dtype_code(out.dtype), _strides4(out),
+        _stream(stream, q))
+    _check(st, "fc_decode_attention")
+
+
+def fc_combine(workspace: torch.Tensor, B: int, Hq: int, D: int,
+               num_splits: int, out: torch.Tensor, stream=None) -> None:
+    st = load().fc_combine(_ptr(workspace),
+                           workspace.numel() * workspace.element_size(),
+                           int(B), int(Hq), int(D), int(num_splits),
+                           _ptr(out), dtype_code(out.dtype), _strides4(out),
+                           _stream(stream, out))
+    _check(st, "fc_combine")
+
+
+def fc_workspace_status(workspace: torch.Tensor, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    st = load().fc_workspace_status(
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        ctypes.byref(v), _stream(stream, workspace))
+    if st not in (FC_OK, FC_ERR_DEVICE):
+        _check(st, "fc_workspace_status")
+    return int(v.value)
+
+
+def fc_storage_bytes(arc: FcArchive, tail: Optional[FcTail] = None) -> int:
+    n = int(load().fc_storage_bytes(ctypes.byref(arc), _ref(tail)))
+    if n < 0:
+        raise FcError(FC_ERR_INVALID, "fc_storage_bytes")
+    return n

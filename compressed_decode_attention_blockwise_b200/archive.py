@@ -1,0 +1,217 @@
+"""Device archive of one layer's K and V streams and its decode attention.
+
+Host bookkeeping around libfc (flashcodec/cache.py, ``_CodecStream`` and
+``CodecKVCache``): each stream keeps a raw tail of at most R-1 tokens at the
+input precision and a compressed archive whose capacity starts at 16 blocks
+and doubles when full, the live prefix being copied by libfc's copy kernel.
+Device memory comes from torch; every byte of codec and attention arithmetic
+runs in libfc's kernels.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Optional
+
+import torch
+
+from . import _lib
+
+INITIAL_BLOCKS = 16
+
+_COEFF = {"i8": torch.int8, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+def grown_capacity(capacity: int, need: int) -> int:
+    """Geometric growth: unchanged if ``need`` fits, else the smallest
+    16 * 2^k >= need (flashcodec/cache.py, ``_CodecStream._grow``)."""
+    if need <= capacity:
+        return capacity
+    cap = INITIAL_BLOCKS
+    while cap < need:
+        cap *= 2
+    return cap
+
+
+class CodecStream:
+    """One (B, H, T, D) K or V stream on the device."""
+
+    def __init__(self, B: int, H: int, D: int, R: int, S: int, coeff: str,
+                 token_dtype: torch.dtype, device, capacity: int = 0):
+        self.B, self.H, self.D, self.R, self.S = B, H, D, R, S
+        self.coeff = coeff
+        self.token_dtype = token_dtype
+        self.device = torch.device(device)
+        self.coeffs: Optional[torch.Tensor] = None
+        self.scales: Optional[torch.Tensor] = None
+        self.tail = torch.zeros((B, H, R, D), dtype=token_dtype,
+                                device=self.device)
+        self.arc = _lib.FcArchive()
+        self.arc.coeff_dtype = _lib.dtype_code(_COEFF[coeff])
+        self.arc.R, self.arc.S = R, S
+        self.arc.B, self.arc.H, self.arc.D = B, H, D
+        self.tail_desc = _lib.FcTail()
+        self.tail_desc.data = self.tail.data_ptr()
+        self.tail_desc.dtype = _lib.dtype_code(token_dtype)
+        self.tail_desc.len = 0
+        self.tail_desc.stride_b, self.tail_desc.stride_h = \
+            self.tail.stride(0), self.tail.stride(1)
+        self._alloc(grown_capacity(0, max(capacity, 1)))
+
+    # -- storage -----------------------------------------------------------
+    def _alloc(self, cap: int):
+        coeffs = torch.empty((self.B, self.H, cap, self.S, self.D),
+                             dtype=_COEFF[self.coeff], device=self.device)
+        scales = None
+        if self.coeff == "i8":
+            scales = torch.empty((self.B, self.H, cap, self.S),
+                                 dtype=torch.float32, device=self.device)
+        new = _lib.FcArchive()
+        ctypes_copy(new, self.arc)
+        new.coeffs = coeffs.data_ptr()
+        new.scales = None if scales is None else scales.data_ptr()
+        new.capacity = cap
+        new.n_blocks = 0
+        new.coeff_stride_b, new.coeff_stride_h = coeffs.stride(0), \
+            coeffs.stride(1)
+        if scales is not None:
+            new.scale_stride_b, new.scale_stride_h = scales.stride(0), \
+                scales.stride(1)
+        else:
+            new.scale_stride_b = new.scale_stride_h = 0
+        if self.coeffs is not None and self.arc.n_blocks:
+            _lib.fc_archive_copy_prefix(self.arc, new, device=self.device)
+        else:
+            new.n_blocks = self.arc.n_blocks if self.coeffs is not None else 0
+        self.coeffs, self.scales, self.arc = coeffs, scales, new
+
+    def ensure_capacity(self, need_blocks: int):
+        cap = grown_capacity(int(self.arc.capacity), int(need_blocks))
+        if cap != self.arc.capacity:
+            self._alloc(cap)
+
+    # -- views ---------------------------------------------------------------
+    @property
+    def n_blocks(self) -> int:
+        return int(self.arc.n_blocks)
+
+    @property
+    def tail_len(self) -> int:
+        return int(self.tail_desc.len)
+
+    @property
+    def capacity(self) -> int:
+        return int(self.arc.capacity)
+
+    @property
+    def seq_len(self) -> int:
+        return self.n_blocks * self.R + self.tail_len
+
+    def live_coeffs(self) -> torch.Tensor:
+        return self.coeffs[:, :, : self.n_blocks]
+
+    def live_scales(self) -> Optional[torch.Tensor]:
+        return None if self.scales is None else \
+            self.scales[:, :, : self.n_blocks]
+
+    def live_tail(self) -> torch.Tensor:
+        return self.tail[:, :, : self.tail_len]
+
+    def storage_bytes(self) -> int:
+        return _lib.fc_storage_bytes(self.arc, self.tail_desc)
+
+
+def ctypes_copy(dst, src):
+    for name, _ in src._fields_:
+        setattr(dst, name, getattr(src, name))
+
+
+class CodecKVCache:
+    """K and V streams of one attention layer plus decode attention.
+
+    ``coeff_k`` / ``coeff_v`` choose the archive storage: "i8" (int8 codes
+    with one fp32 scale per (block, frequency)), "bf16" or "f32".
+    """
+
+    def __init__(self, B: int, Hk: int, D: int, R: int = 8, S: int = 2,
+                 coeff_k: str = "i8", coeff_v: str = "i8",
+                 token_dtype: torch.dtype = torch.bfloat16, device="cuda",
+                 capacity: int = 0):
+        self.B, self.Hk, self.D, self.R, self.S = B, Hk, D, R, S
+        self.k = CodecStream(B, Hk, D, R, S, coeff_k, token_dtype, device,
+                             capacity)
+        self.v = CodecStream(B, Hk, D, R, S, coeff_v, token_dtype, device,
+                             capacity)
+        self.device = self.k.device
+        self._ws: Optional[torch.Tensor] = None
+
+    @property
+    def seq_len(self) -> int:
+        return self.k.seq_len
+
+    def _grow_to(self, need_blocks: int):
+        self.k.ensure_capacity(need_blocks)
+        self.v.ensure_capacity(need_blocks)
+
+    # -- writes ------------------------------------------------------------
+    def prefill(self, k: torch.Tensor, v: torch.Tensor):
+        """Append a (B, Hk, T, D) prefill: complete blocks are compressed in
+        one launch per stream, the remainder becomes the raw tail."""
+        if k.shape != v.shape or k.shape[0] != self.B or \
+                k.shape[1] != self.Hk or k.shape[3] != self.D:
+            raise ValueError("prefill shape mismatch")
+        t0 = 0
+        # top up a partial tail token by token first (append semantics)
+        while self.k.tail_len and t0 < k.shape[2]:
+            self.append(k[:, :, t0:t0 + 1], v[:, :, t0:t0 + 1])
+            t0 += 1
+        if t0 >= k.shape[2]:
+            return
+        kk, vv = k[:, :, t0:], v[:, :, t0:]
+        self._grow_to(self.k.n_blocks + kk.shape[2] // self.R)
+        _lib.fc_compress_blocks(kk, self.k.arc, self.k.tail_desc)
+        _lib.fc_compress_blocks(vv, self.v.arc, self.v.tail_desc)
+
+    def append(self, k_new: torch.Tensor, v_new: torch.Tensor):
+        """decode_step: append one (B, Hk, 1, D) token to both streams."""
+        if self.k.tail_len + 1 == self.R:
+            self._grow_to(self.k.n_blocks + 1)
+        _lib.fc_append_step(k_new, v_new, self.k.arc, self.v.arc,
+                            self.k.tail_desc, self.v.tail_desc)
+
+    # -- attention -----------------------------------------------------------
+    def num_splits(self, Hq: int) -> int:
+        return _lib.fc_decode_plan(self.k.arc, self.k.tail_desc, Hq)
+
+    def workspace(self, Hq: int, num_splits: int) -> torch.Tensor:
+        need = _lib.fc_decode_workspace_bytes(self.B, Hq, self.D, num_splits)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.zeros(need, dtype=torch.uint8,
+                                   device=self.device)
+        return self._ws
+
+    def attention(self, q: torch.Tensor, out: Optional[torch.Tensor] = None,
+                  softmax_scale: Optional[float] = None, num_splits: int = 0,
+                  fuse_combine: bool = True,
+                  out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
+        """Decode attention of q (B, Hq, 1, D) over archive + tail."""
+        Hq = q.shape[1]
+        if out is None:
+            out = torch.empty((self.B, Hq, 1, self.D), dtype=out_dtype,
+                              device=q.device)
+        ns = num_splits or self.num_splits(Hq)
+        ws = self.workspace(Hq, ns)
+        _lib.fc_decode_attention(
+            q, self.k.arc, self.v.arc, self.k.tail_desc, self.v.tail_desc,
+            out, ws, softmax_scale=0.0 if softmax_scale is None else
+            float(softmax_scale), num_splits=ns, fuse_combine=fuse_combine)
+        if not fuse_combine:
+            _lib.fc_combine(ws, self.B, Hq, self.D, ns, out)
+        return out
+
+    def storage_bytes(self) -> int:
+        return self.k.storage_bytes() + self.v.storage_bytes()
+
+
+def default_scale(D: int) -> float:
+    return 1.0 / math.sqrt(D)

@@ -1,0 +1,189 @@
+// Entry points of coefficient-domain decode attention: planning, argument
+// validation, kernel selection, and the stand-alone combine.
+#include <cmath>
+
+#include "fc_decode.cuh"
+
+namespace fc {
+namespace {
+
+// Split count: enough (chunk, kv head, batch) CTAs to give every SM about four,
+// but no chunk shorter than 16 blocks (the partials then stay a small fraction
+// of the archive bytes).
+int plan_splits(int64_t nb, int64_t B, int64_t Hk) {
+  if (nb <= 0) return 1;
+  const int64_t units = B * Hk;
+  const int64_t target = int64_t(sm_count()) * 4;
+  int64_t ns = (target + units - 1) / units;
+  const int64_t by_len = nb / 16 > 0 ? nb / 16 : 1;
+  if (ns > by_len) ns = by_len;
+  if (ns > kMaxSplits) ns = kMaxSplits;
+  if (ns < 1) ns = 1;
+  return int(ns);
+}
+
+bool supported_G(int64_t G) { return G == 1 || G == 2 || G == 4 || G == 8 || G == 16; }
+
+__global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
+  extern __shared__ float wts[];  // ns + 1
+  const int hq = blockIdx.x, b = blockIdx.y;
+  const int64_t row = (int64_t(b) * a.Hq + hq) * a.ns;
+  combine_head(a.pm + row, a.pl + row, a.pacc + row * a.D, a.ns, a.D, wts, a.out,
+               b * a.os_b + hq * a.os_h, a.out_dtype);
+}
+
+int check_io(const void* p, int dtype, const int64_t* strides) {
+  if (!p || !strides) return FC_ERR_INVALID;
+  if (dtype != FC_DTYPE_F32 && dtype != FC_DTYPE_BF16) return FC_ERR_INVALID;
+  if (strides[3] != 1 || strides[0] < 0 || strides[1] < 0) return FC_ERR_INVALID;
+  return FC_OK;
+}
+
+}  // namespace
+}  // namespace fc
+
+using namespace fc;
+
+extern "C" int fc_decode_plan(const fc_archive* ka, const fc_tail* kt, int64_t Hq,
+                              int32_t* num_splits_out) {
+  (void)kt;
+  if (!num_splits_out) return FC_ERR_INVALID;
+  const int st = check_archive(ka);
+  if (st != FC_OK) return st;
+  if (Hq < 1 || Hq % ka->H) return FC_ERR_INVALID;
+  *num_splits_out = plan_splits(ka->n_blocks, ka->B, ka->H);
+  return FC_OK;
+}
+
+extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides,
+                                   int64_t Hq, const fc_archive* ka, const fc_archive* va,
+                                   const fc_tail* kt, const fc_tail* vt, float softmax_scale,
+                                   int32_t num_splits, int32_t fuse_combine, void* workspace,
+                                   size_t workspace_bytes, void* out, int32_t out_dtype,
+                                   const int64_t* out_strides, fc_stream stream) {
+  int st = check_archive(ka);
+  if (st != FC_OK) return st;
+  st = check_archive(va);
+  if (st != FC_OK) return st;
+  if (ka->B != va->B || ka->H != va->H || ka->R != va->R || ka->S != va->S || ka->D != va->D ||
+      ka->n_blocks != va->n_blocks)
+    return FC_ERR_INVALID;
+  st = check_io(q, q_dtype, q_strides);
+  if (st != FC_OK) return st;
+  st = check_io(out, out_dtype, out_strides);
+  if (st != FC_OK) return st;
+  if (Hq < 1 || Hq % ka->H) return FC_ERR_INVALID;
+  const int64_t G = Hq / ka->H;
+  if (!supported_G(G)) return FC_ERR_UNSUPPORTED;
+  if (G * (ka->D / 32) > 64) return FC_ERR_UNSUPPORTED;
+  int nr = 0;
+  int t_dtype = FC_DTYPE_BF16;
+  if (kt || vt) {
+    if (!kt || !vt) return FC_ERR_INVALID;
+    st = check_tail(kt, ka, true);
+    if (st != FC_OK) return st;
+    st = check_tail(vt, va, true);
+    if (st != FC_OK) return st;
+    if (kt->len != vt->len || kt->dtype != vt->dtype) return FC_ERR_INVALID;
+    nr = kt->len;
+    t_dtype = kt->dtype;
+  }
+  if (ka->n_blocks == 0 && nr == 0) return FC_ERR_INVALID;
+  int ns = num_splits;
+  if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H);
+  if (ns < 1 || ns > kMaxSplits) return FC_ERR_INVALID;
+  if (ka->B > 65535 || ka->H > 65535) return FC_ERR_UNSUPPORTED;
+  const bool need_ws = !(fuse_combine && ns == 1);
+  const WorkspaceLayout wl = workspace_layout(ka->B, Hq, ka->D, ns);
+  if (need_ws) {
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+        workspace_bytes < wl.total)
+      return FC_ERR_INVALID;
+  }
+  DecodeArgs a;
+  a.q = q;
+  a.q_dtype = q_dtype;
+  a.qs_b = q_strides[0];
+  a.qs_h = q_strides[1];
+  a.kc = ka->coeffs;
+  a.ks = ka->scales;
+  a.kcs_b = ka->coeff_stride_b;
+  a.kcs_h = ka->coeff_stride_h;
+  a.kss_b = ka->scale_stride_b;
+  a.kss_h = ka->scale_stride_h;
+  a.vc = va->coeffs;
+  a.vs = va->scales;
+  a.vcs_b = va->coeff_stride_b;
+  a.vcs_h = va->coeff_stride_h;
+  a.vss_b = va->scale_stride_b;
+  a.vss_h = va->scale_stride_h;
+  a.kt = kt ? kt->data : nullptr;
+  a.vt = vt ? vt->data : nullptr;
+  a.t_dtype = t_dtype;
+  a.kts_b = kt ? kt->stride_b : 0;
+  a.kts_h = kt ? kt->stride_h : 0;
+  a.vts_b = vt ? vt->stride_b : 0;
+  a.vts_h = vt ? vt->stride_h : 0;
+  a.nr = nr;
+  a.B = int(ka->B);
+  a.Hk = int(ka->H);
+  a.G = int(G);
+  a.R = ka->R;
+  a.S = ka->S;
+  a.D = int(ka->D);
+  a.nb = ka->n_blocks;
+  a.ns = ns;
+  a.chunk = ka->n_blocks > 0 ? (ka->n_blocks + ns - 1) / ns : 0;
+  const float sigma = softmax_scale > 0.f ? softmax_scale : float(1.0 / std::sqrt(double(ka->D)));
+  a.qscale = float(double(sigma) * 1.4426950408889634);  // log2(e)
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.status = need_ws ? reinterpret_cast<uint32_t*>(ws + wl.status) : nullptr;
+  a.tickets = need_ws ? reinterpret_cast<uint32_t*>(ws + wl.tickets) : nullptr;
+  a.pm = need_ws ? reinterpret_cast<float*>(ws + wl.m) : nullptr;
+  a.pl = need_ws ? reinterpret_cast<float*>(ws + wl.l) : nullptr;
+  a.pacc = need_ws ? reinterpret_cast<float*>(ws + wl.acc) : nullptr;
+  a.fuse = fuse_combine ? 1 : 0;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.os_b = out_strides[0];
+  a.os_h = out_strides[1];
+  Basis basis;
+  make_basis(ka->R, ka->S, &basis);
+  const int kd = ka->coeff_dtype, vd = va->coeff_dtype;
+  if (kd == FC_DTYPE_I8 && vd == FC_DTYPE_I8) return launch_decode_generic<int8_t, int8_t>(a, basis, stream);
+  if (kd == FC_DTYPE_I8 && vd == FC_DTYPE_BF16)
+    return launch_decode_generic<int8_t, __nv_bfloat16>(a, basis, stream);
+  if (kd == FC_DTYPE_I8 && vd == FC_DTYPE_F32) return launch_decode_generic<int8_t, float>(a, basis, stream);
+  if (kd == FC_DTYPE_BF16 && vd == FC_DTYPE_BF16)
+    return launch_decode_generic<__nv_bfloat16, __nv_bfloat16>(a, basis, stream);
+  if (kd == FC_DTYPE_F32 && vd == FC_DTYPE_F32) return launch_decode_generic<float, float>(a, basis, stream);
+  return FC_ERR_UNSUPPORTED;
+}
+
+extern "C" int fc_combine(const void* workspace, size_t workspace_bytes, int64_t B, int64_t Hq,
+                          int64_t D, int32_t num_splits, void* out, int32_t out_dtype,
+                          const int64_t* out_strides, fc_stream stream) {
+  if (B < 1 || Hq < 1 || num_splits < 1 || num_splits > kMaxSplits) return FC_ERR_INVALID;
+  if (D != 32 && D != 64 && D != 128 && D != 256) return FC_ERR_UNSUPPORTED;
+  int st = check_io(out, out_dtype, out_strides);
+  if (st != FC_OK) return st;
+  const WorkspaceLayout wl = workspace_layout(B, Hq, D, num_splits);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) || workspace_bytes < wl.total)
+    return FC_ERR_INVALID;
+  if (B > 65535 || Hq > 0x7fffffff) return FC_ERR_UNSUPPORTED;
+  const uint8_t* ws = static_cast<const uint8_t*>(workspace);
+  CombineArgs a;
+  a.pm = reinterpret_cast<const float*>(ws + wl.m);
+  a.pl = reinterpret_cast<const float*>(ws + wl.l);
+  a.pacc = reinterpret_cast<const float*>(ws + wl.acc);
+  a.Hq = int(Hq);
+  a.D = int(D);
+  a.ns = num_splits;
+  a.out = out;
+  a.out_dtype = out_dtype;
+  a.os_b = out_strides[0];
+  a.os_h = out_strides[1];
+  const size_t smem = size_t(num_splits + 1) * sizeof(float);
+  combine_kernel<<<dim3(unsigned(Hq), unsigned(B)), 128, smem, stream>>>(a);
+  return cuda_status(cudaGetLastError());
+}

@@ -1,0 +1,503 @@
+// Block-DCT codec kernels: prefill compression, single-token append and the
+// archive's growth copy.
+//
+// flashcodec-kv README "Math": a block X (R x D) is encoded as C = M X with the
+// orthonormal DCT-II rows M; the S lowest frequencies are kept. With int8
+// storage each (block, frequency) row keeps one fp32 scale over D
+// (README, quant_bits=8 paragraph; flashcodec/cache.py, _archive_spec):
+// scale = max_d |C| / 127 and code = clamp(rint(C / scale), -127, 127), an
+// all-zero row storing scale 0 and codes 0. Only complete blocks are archived
+// (flashcodec/cache.py, _CodecStream.append).
+//
+// Work mapping: one warp per (b, h, block); lane l owns the VEC = D / 32
+// consecutive channels [l * VEC, (l + 1) * VEC), so every token row is one
+// coalesced warp-wide load and every coefficient row one coalesced store. The
+// S x VEC coefficients accumulate in registers in fp32 (t ascending, fused
+// multiply-add), the absmax is a warp-shuffle max, and the quantiser divides in
+// fp32 with round-to-nearest-even. Compression of a prefill and of an appended
+// block run the same device code in the same order, so an archive built token
+// by token is bitwise identical to one built in a single call.
+#include <type_traits>
+
+#include "fc_internal.cuh"
+
+namespace fc {
+namespace {
+
+struct StreamOut {
+  void* coeffs;
+  float* scales;
+  int64_t cs_b, cs_h;  // coefficient element strides
+  int64_t ss_b, ss_h;  // scale element strides
+};
+
+template <int VEC, int SMAX>
+__device__ __forceinline__ void accum_row(float (&c)[SMAX][VEC], const float (&x)[VEC],
+                                          const Basis& basis, int t, int S) {
+#pragma unroll
+  for (int j = 0; j < SMAX; ++j) {
+    if (j < S) {
+      const float m = basis.m[j][t];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) c[j][v] = fmaf(m, x[v], c[j][v]);
+    }
+  }
+}
+
+template <int VEC>
+__device__ __forceinline__ void store_codes(int8_t* p, const int (&code)[VEC]) {
+  if constexpr (VEC == 1) {
+    *p = static_cast<int8_t>(code[0]);
+  } else if constexpr (VEC == 2) {
+    const uint32_t w = (uint32_t(code[0]) & 0xffu) | ((uint32_t(code[1]) & 0xffu) << 8);
+    *reinterpret_cast<unsigned short*>(p) = static_cast<unsigned short>(w);
+  } else {
+    uint32_t w[VEC / 4];
+#pragma unroll
+    for (int i = 0; i < VEC / 4; ++i) {
+      w[i] = (uint32_t(code[4 * i]) & 0xffu) | ((uint32_t(code[4 * i + 1]) & 0xffu) << 8) |
+             ((uint32_t(code[4 * i + 2]) & 0xffu) << 16) | ((uint32_t(code[4 * i + 3]) & 0xffu) << 24);
+    }
+    if constexpr (VEC == 4) {
+      *reinterpret_cast<uint32_t*>(p) = w[0];
+    } else {
+      *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+    }
+  }
+}
+
+template <typename T, int VEC>
+__device__ __forceinline__ void store_row(T* p, const float (&x)[VEC]) {
+  if constexpr (std::is_same_v<T, float>) {
+    if constexpr (VEC % 4 == 0) {
+#pragma unroll
+      for (int i = 0; i < VEC / 4; ++i)
+        reinterpret_cast<float4*>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+    } else if constexpr (VEC == 2) {
+      *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
+    } else {
+      p[0] = x[0];
+    }
+  } else {
+    static_assert(std::is_same_v<T, __nv_bfloat16>, "bf16 or f32 rows");
+    if constexpr (VEC == 1) {
+      p[0] = __float2bfloat16_rn(x[0]);
+    } else {
+      uint32_t w[VEC / 2];
+#pragma unroll
+      for (int i = 0; i < VEC / 2; ++i) {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h);
+      }
+      if constexpr (VEC == 2) {
+        *reinterpret_cast<uint32_t*>(p) = w[0];
+      } else if constexpr (VEC == 4) {
+        *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+      } else {
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+}
+
+// Quantises (int8) or rounds (bf16 / f32) the S coefficient rows of one block
+// and stores them at `blk` (S x D elements) / `scl` (S floats).
+template <typename TOut, int VEC, int SMAX>
+__device__ __forceinline__ void store_block(const float (&c)[SMAX][VEC], int S, int D, int lane,
+                                            TOut* blk, float* scl) {
+#pragma unroll
+  for (int j = 0; j < SMAX; ++j) {
+    if (j < S) {
+      if constexpr (std::is_same_v<TOut, int8_t>) {
+        float amax = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) amax = fmaxf(amax, fabsf(c[j][v]));
+        amax = warp_max(amax);
+        const float scale = amax / 127.0f;
+        int code[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          int q = 0;
+          if (scale > 0.f) q = __float2int_rn(c[j][v] / scale);
+          code[v] = max(-127, min(127, q));
+        }
+        store_codes<VEC>(blk + int64_t(j) * D + lane * VEC, code);
+        if (lane == 0) scl[j] = scale;
+      } else {
+        float row[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) row[v] = c[j][v];
+        store_row<TOut, VEC>(blk + int64_t(j) * D + lane * VEC, row);
+      }
+    }
+  }
+}
+
+struct CompressArgs {
+  const void* x;
+  int64_t xs_b, xs_h, xs_t;
+  int B, H, R, S, D;
+  int64_t n_full, slot0;
+  StreamOut out;
+  void* tail;  // may be null
+  int64_t ts_b, ts_h;
+  int n_rem;
+};
+
+template <int VEC, int SMAX, typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) compress_blocks_kernel(CompressArgs a, Basis basis) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_items = int64_t(a.B) * a.H * a.n_full;
+  const TIn* x = static_cast<const TIn*>(a.x);
+  if (w < n_items) {
+    const int64_t n = w % a.n_full;
+    const int64_t bh = w / a.n_full;
+    const int h = int(bh % a.H), b = int(bh / a.H);
+    const TIn* src = x + b * a.xs_b + h * a.xs_h + n * a.R * a.xs_t + lane * VEC;
+    float c[SMAX][VEC];
+#pragma unroll
+    for (int j = 0; j < SMAX; ++j)
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) c[j][v] = 0.f;
+#pragma unroll 4
+    for (int t = 0; t < a.R; ++t) {
+      float xv[VEC];
+      load_vec<TIn, VEC>(src + t * a.xs_t, xv);
+      accum_row<VEC, SMAX>(c, xv, basis, t, a.S);
+    }
+    TOut* blk = static_cast<TOut*>(a.out.coeffs) + b * a.out.cs_b + h * a.out.cs_h +
+                (a.slot0 + n) * a.S * a.D;
+    float* scl = a.out.scales ? a.out.scales + b * a.out.ss_b + h * a.out.ss_h + (a.slot0 + n) * a.S
+                              : nullptr;
+    store_block<TOut, VEC, SMAX>(c, a.S, a.D, lane, blk, scl);
+  } else if (a.tail != nullptr && w < n_items + int64_t(a.B) * a.H) {
+    // copy the T mod R remaining tokens of (b, h) into its raw tail rows
+    const int64_t bh = w - n_items;
+    const int h = int(bh % a.H), b = int(bh / a.H);
+    const TIn* src = x + b * a.xs_b + h * a.xs_h + a.n_full * a.R * a.xs_t + lane * VEC;
+    TIn* dst = static_cast<TIn*>(a.tail) + b * a.ts_b + h * a.ts_h + lane * VEC;
+    for (int i = 0; i < a.n_rem; ++i) {
+      float xv[VEC];
+      load_vec<TIn, VEC>(src + i * a.xs_t, xv);
+      store_row<TIn, VEC>(dst + int64_t(i) * a.D, xv);
+    }
+  }
+}
+
+struct AppendStream {
+  const void* src;  // new token (B, H, 1, D)
+  int64_t src_b, src_h;
+  void* tail;
+  int64_t ts_b, ts_h;
+  StreamOut out;
+};
+
+struct AppendArgs {
+  AppendStream st[2];
+  int B, H, R, S, D;
+  int len;       // tail rows before this token
+  int complete;  // len + 1 == R: archive the block into `slot`
+  int64_t slot;
+};
+
+template <int VEC, int SMAX, typename TIn, typename TOutK, typename TOutV>
+__global__ void __launch_bounds__(256) append_step_kernel(AppendArgs a, Basis basis) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t bh_total = int64_t(a.B) * a.H;
+  if (w >= 2 * bh_total) return;
+  const int s = int(w / bh_total);
+  const int64_t bh = w % bh_total;
+  const int h = int(bh % a.H), b = int(bh / a.H);
+  const AppendStream& st = a.st[s];
+  float xn[VEC];
+  load_vec<TIn, VEC>(static_cast<const TIn*>(st.src) + b * st.src_b + h * st.src_h + lane * VEC, xn);
+  TIn* trow = static_cast<TIn*>(st.tail) + b * st.ts_b + h * st.ts_h + lane * VEC;
+  if (!a.complete) {
+    store_row<TIn, VEC>(trow + int64_t(a.len) * a.D, xn);
+    return;
+  }
+  // the block completes: rows 0..R-2 come from the tail, row R-1 is the new token
+  float c[SMAX][VEC];
+#pragma unroll
+  for (int j = 0; j < SMAX; ++j)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) c[j][v] = 0.f;
+  for (int t = 0; t < a.R - 1; ++t) {
+    float xv[VEC];
+    load_vec<TIn, VEC>(trow + int64_t(t) * a.D, xv);
+    accum_row<VEC, SMAX>(c, xv, basis, t, a.S);
+  }
+  accum_row<VEC, SMAX>(c, xn, basis, a.R - 1, a.S);
+  const StreamOut& o = st.out;
+  float* scl = o.scales ? o.scales + b * o.ss_b + h * o.ss_h + a.slot * a.S : nullptr;
+  if (s == 0) {
+    TOutK* blk = static_cast<TOutK*>(o.coeffs) + b * o.cs_b + h * o.cs_h + a.slot * a.S * a.D;
+    store_block<TOutK, VEC, SMAX>(c, a.S, a.D, lane, blk, scl);
+  } else {
+    TOutV* blk = static_cast<TOutV*>(o.coeffs) + b * o.cs_b + h * o.cs_h + a.slot * a.S * a.D;
+    store_block<TOutV, VEC, SMAX>(c, a.S, a.D, lane, blk, scl);
+  }
+}
+
+struct CopyArgs {
+  const uint8_t* src_c;
+  uint8_t* dst_c;
+  int64_t src_cb, src_ch, dst_cb, dst_ch;  // byte strides
+  int64_t bytes_per_head;                  // multiple of 16
+  const float* src_s;
+  float* dst_s;
+  int64_t src_sb, src_sh, dst_sb, dst_sh;  // element strides
+  int64_t scales_per_head;
+  int H;
+};
+
+__global__ void __launch_bounds__(256) archive_copy_kernel(CopyArgs a) {
+  const int bh = blockIdx.y;
+  const int h = bh % a.H, b = bh / a.H;
+  const uint4* s = reinterpret_cast<const uint4*>(a.src_c + b * a.src_cb + h * a.src_ch);
+  uint4* d = reinterpret_cast<uint4*>(a.dst_c + b * a.dst_cb + h * a.dst_ch);
+  const int64_t n16 = a.bytes_per_head / 16;
+  for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n16;
+       i += int64_t(gridDim.x) * blockDim.x)
+    d[i] = s[i];
+  if (a.src_s) {
+    const float* ss = a.src_s + b * a.src_sb + h * a.src_sh;
+    float* ds = a.dst_s + b * a.dst_sb + h * a.dst_sh;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < a.scales_per_head;
+         i += int64_t(gridDim.x) * blockDim.x)
+      ds[i] = ss[i];
+  }
+}
+
+// ------------------------------------------------------------ dispatch
+
+template <typename F>
+int dispatch_vec(int D, F&& f) {
+  switch (D) {
+    case 32: return f(std::integral_constant<int, 1>{});
+    case 64: return f(std::integral_constant<int, 2>{});
+    case 128: return f(std::integral_constant<int, 4>{});
+    case 256: return f(std::integral_constant<int, 8>{});
+    default: return FC_ERR_UNSUPPORTED;
+  }
+}
+
+template <typename F>
+int dispatch_smax(int S, F&& f) {
+  if (S <= 4) return f(std::integral_constant<int, 4>{});
+  return f(std::integral_constant<int, 16>{});
+}
+
+template <typename F>
+int dispatch_in(int dt, F&& f) {
+  if (dt == FC_DTYPE_BF16) return f(__nv_bfloat16{});
+  if (dt == FC_DTYPE_F32) return f(float{});
+  return FC_ERR_UNSUPPORTED;
+}
+
+template <typename F>
+int dispatch_out(int dt, F&& f) {
+  if (dt == FC_DTYPE_I8) return f(int8_t{});
+  if (dt == FC_DTYPE_BF16) return f(__nv_bfloat16{});
+  if (dt == FC_DTYPE_F32) return f(float{});
+  return FC_ERR_UNSUPPORTED;
+}
+
+StreamOut stream_out(const fc_archive* a) {
+  StreamOut o;
+  o.coeffs = a->coeffs;
+  o.scales = a->scales;
+  o.cs_b = a->coeff_stride_b;
+  o.cs_h = a->coeff_stride_h;
+  o.ss_b = a->scale_stride_b;
+  o.ss_h = a->scale_stride_h;
+  return o;
+}
+
+}  // namespace
+}  // namespace fc
+
+using namespace fc;
+
+extern "C" int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t* x_strides,
+                                  int64_t T, fc_archive* arc, fc_tail* tail, fc_stream stream) {
+  if (!x || !x_strides || T < 0) return FC_ERR_INVALID;
+  int st = check_archive(arc);
+  if (st != FC_OK) return st;
+  if (x_dtype != FC_DTYPE_BF16 && x_dtype != FC_DTYPE_F32) return FC_ERR_INVALID;
+  if (x_strides[3] != 1 || x_strides[0] < 0 || x_strides[1] < 0 || x_strides[2] < 0)
+    return FC_ERR_INVALID;
+  const int esz = dtype_size(x_dtype);
+  if (!aligned16(x) || (x_strides[0] * esz) % 16 || (x_strides[1] * esz) % 16 ||
+      (x_strides[2] * esz) % 16)
+    return FC_ERR_INVALID;
+  const int64_t n_full = T / arc->R;
+  const int n_rem = int(T - n_full * arc->R);
+  if (tail) {
+    st = check_tail(tail, arc, n_rem == 0);
+    if (st != FC_OK) return st;
+    if (tail->len != 0 || tail->dtype != x_dtype) return FC_ERR_INVALID;
+  }
+  if (arc->n_blocks + n_full > arc->capacity) return FC_ERR_CAPACITY;
+  const bool copy_tail = tail && n_rem > 0;
+  if (n_full == 0 && !copy_tail) {
+    return FC_OK;
+  }
+  CompressArgs a;
+  a.x = x;
+  a.xs_b = x_strides[0];
+  a.xs_h = x_strides[1];
+  a.xs_t = x_strides[2];
+  a.B = int(arc->B);
+  a.H = int(arc->H);
+  a.R = arc->R;
+  a.S = arc->S;
+  a.D = int(arc->D);
+  a.n_full = n_full;
+  a.slot0 = arc->n_blocks;
+  a.out = stream_out(arc);
+  a.tail = copy_tail ? tail->data : nullptr;
+  a.ts_b = tail ? tail->stride_b : 0;
+  a.ts_h = tail ? tail->stride_h : 0;
+  a.n_rem = n_rem;
+  Basis basis;
+  make_basis(arc->R, arc->S, &basis);
+  const int64_t warps = arc->B * arc->H * n_full + (copy_tail ? arc->B * arc->H : 0);
+  const int64_t grid = (warps + 7) / 8;
+  if (grid > 0x7fffffffLL) return FC_ERR_UNSUPPORTED;
+  st = dispatch_vec(a.D, [&](auto vec) {
+    return dispatch_smax(a.S, [&](auto smax) {
+      return dispatch_in(x_dtype, [&](auto tin) {
+        return dispatch_out(arc->coeff_dtype, [&](auto tout) {
+          using TIn = decltype(tin);
+          using TOut = decltype(tout);
+          compress_blocks_kernel<decltype(vec)::value, decltype(smax)::value, TIn, TOut>
+              <<<unsigned(grid), 256, 0, stream>>>(a, basis);
+          return cuda_status(cudaGetLastError());
+        });
+      });
+    });
+  });
+  if (st != FC_OK) return st;
+  arc->n_blocks += n_full;
+  if (copy_tail) tail->len = n_rem;
+  return FC_OK;
+}
+
+extern "C" int fc_append_step(const void* k_new, const void* v_new, int32_t dtype,
+                              const int64_t* k_strides, const int64_t* v_strides, fc_archive* ka,
+                              fc_archive* va, fc_tail* kt, fc_tail* vt, fc_stream stream) {
+  if (!k_new || !v_new || !k_strides || !v_strides) return FC_ERR_INVALID;
+  int st = check_archive(ka);
+  if (st != FC_OK) return st;
+  st = check_archive(va);
+  if (st != FC_OK) return st;
+  if (ka->B != va->B || ka->H != va->H || ka->R != va->R || ka->S != va->S || ka->D != va->D ||
+      ka->n_blocks != va->n_blocks)
+    return FC_ERR_INVALID;
+  st = check_tail(kt, ka, false);
+  if (st != FC_OK) return st;
+  st = check_tail(vt, va, false);
+  if (st != FC_OK) return st;
+  if (kt->len != vt->len || kt->dtype != dtype || vt->dtype != dtype) return FC_ERR_INVALID;
+  if (k_strides[3] != 1 || v_strides[3] != 1) return FC_ERR_INVALID;
+  const int esz = dtype_size(dtype);
+  if (!aligned16(k_new) || !aligned16(v_new) || (k_strides[0] * esz) % 16 ||
+      (k_strides[1] * esz) % 16 || (v_strides[0] * esz) % 16 || (v_strides[1] * esz) % 16)
+    return FC_ERR_INVALID;
+  const bool complete = kt->len + 1 == ka->R;
+  if (complete && (ka->n_blocks >= ka->capacity || va->n_blocks >= va->capacity))
+    return FC_ERR_CAPACITY;
+  AppendArgs a;
+  const fc_archive* arcs[2] = {ka, va};
+  const fc_tail* tails[2] = {kt, vt};
+  const void* srcs[2] = {k_new, v_new};
+  const int64_t* strides[2] = {k_strides, v_strides};
+  for (int s = 0; s < 2; ++s) {
+    a.st[s].src = srcs[s];
+    a.st[s].src_b = strides[s][0];
+    a.st[s].src_h = strides[s][1];
+    a.st[s].tail = tails[s]->data;
+    a.st[s].ts_b = tails[s]->stride_b;
+    a.st[s].ts_h = tails[s]->stride_h;
+    a.st[s].out = stream_out(arcs[s]);
+  }
+  a.B = int(ka->B);
+  a.H = int(ka->H);
+  a.R = ka->R;
+  a.S = ka->S;
+  a.D = int(ka->D);
+  a.len = kt->len;
+  a.complete = complete ? 1 : 0;
+  a.slot = ka->n_blocks;
+  Basis basis;
+  make_basis(ka->R, ka->S, &basis);
+  const int64_t warps = 2 * ka->B * ka->H;
+  const int64_t grid = (warps + 7) / 8;
+  st = dispatch_vec(a.D, [&](auto vec) {
+    return dispatch_smax(a.S, [&](auto smax) {
+      return dispatch_in(dtype, [&](auto tin) {
+        return dispatch_out(ka->coeff_dtype, [&](auto tk) {
+          return dispatch_out(va->coeff_dtype, [&](auto tv) {
+            append_step_kernel<decltype(vec)::value, decltype(smax)::value, decltype(tin),
+                               decltype(tk), decltype(tv)><<<unsigned(grid), 256, 0, stream>>>(a, basis);
+            return cuda_status(cudaGetLastError());
+          });
+        });
+      });
+    });
+  });
+  if (st != FC_OK) return st;
+  if (complete) {
+    ka->n_blocks += 1;
+    va->n_blocks += 1;
+    kt->len = 0;
+    vt->len = 0;
+  } else {
+    kt->len += 1;
+    vt->len += 1;
+  }
+  return FC_OK;
+}
+
+extern "C" int fc_archive_copy_prefix(const fc_archive* src, fc_archive* dst, fc_stream stream) {
+  int st = check_archive(src);
+  if (st != FC_OK) return st;
+  st = check_archive(dst);
+  if (st != FC_OK) return st;
+  if (src->B != dst->B || src->H != dst->H || src->R != dst->R || src->S != dst->S ||
+      src->D != dst->D || src->coeff_dtype != dst->coeff_dtype)
+    return FC_ERR_INVALID;
+  if (dst->capacity < src->n_blocks) return FC_ERR_CAPACITY;
+  if (src->n_blocks > 0) {
+    const int64_t esz = dtype_size(src->coeff_dtype);
+    CopyArgs a;
+    a.src_c = static_cast<const uint8_t*>(src->coeffs);
+    a.dst_c = static_cast<uint8_t*>(dst->coeffs);
+    a.src_cb = src->coeff_stride_b * esz;
+    a.src_ch = src->coeff_stride_h * esz;
+    a.dst_cb = dst->coeff_stride_b * esz;
+    a.dst_ch = dst->coeff_stride_h * esz;
+    a.bytes_per_head = src->n_blocks * src->S * src->D * esz;
+    a.src_s = src->scales;
+    a.dst_s = dst->scales;
+    a.src_sb = src->scale_stride_b;
+    a.src_sh = src->scale_stride_h;
+    a.dst_sb = dst->scale_stride_b;
+    a.dst_sh = dst->scale_stride_h;
+    a.scales_per_head = src->scales ? src->n_blocks * src->S : 0;
+    a.H = int(src->H);
+    const int64_t bh = src->B * src->H;
+    if (bh > 65535) return FC_ERR_UNSUPPORTED;
+    int64_t gx = (a.bytes_per_head / 16 + 255) / 256;
+    if (gx > 1024) gx = 1024;
+    if (gx < 1) gx = 1;
+    archive_copy_kernel<<<dim3(unsigned(gx), unsigned(bh)), 256, 0, stream>>>(a);
+    st = cuda_status(cudaGetLastError());
+    if (st != FC_OK) return st;
+  }
+  dst->n_blocks = src->n_blocks;
+  return FC_OK;
+}

@@ -1,0 +1,257 @@
+/*
+ * fc.h -- C ABI of libfc: a block-DCT int8 codec for a transformer KV cache and
+ * single-token decode attention computed directly on the compressed
+ * coefficients, for NVIDIA B200 (sm_100a).
+ *
+ * Method (flashcodec-kv 1.0.0 README, "Math" and "Materialization-free decode
+ * attention"; flashcodec/triton_attention.py; flashcodec/cache.py):
+ *   - every complete block of R tokens of a (B, H, T, D) K or V stream is
+ *     encoded as C = M X_blk with the orthonormal DCT-II rows
+ *     M[j, t] = c_j cos(pi/R (t + 1/2) j), c_0 = sqrt(1/R), c_j = sqrt(2/R),
+ *     keeping the S lowest frequencies; the partial last block stays raw;
+ *   - int8 storage keeps one fp32 scale per (block, frequency):
+ *     scale = max_d |C| / 127, code = clamp(round_half_even(C / scale), -127, 127)
+ *     (an all-zero row stores scale 0 and codes 0);
+ *   - decode attention never reconstructs K or V: per block s = C_k q,
+ *     logits = sigma A s with A = M^T (R x S), an online-softmax update,
+ *     w = p A, acc += w C_v; the raw tail joins the same softmax; the pass is
+ *     split-K over block chunks and a combine merges the (max, sum, acc)
+ *     partials.
+ *
+ * Conventions for every call:
+ *   - All tensors live in device memory owned by the caller. The library never
+ *     allocates device memory; scratch comes in through `workspace`.
+ *   - Element strides are in ELEMENTS of the tensor's dtype. The innermost
+ *     (head_dim) stride is always 1.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and returns an fc_status. Arguments are validated on the
+ *     host before anything is launched; on any error nothing is launched and
+ *     no descriptor is modified. No exception crosses the ABI.
+ *   - Host-side descriptor fields that a call advances (n_blocks, len) are
+ *     updated only when the call returns FC_OK.
+ *   - There is no fallback path: an unsupported shape or dtype is an error.
+ *
+ * Supported sizes: D in {32, 64, 128, 256}; 1 <= S <= R <= 32 and S <= 16;
+ * Hq a multiple of Hk with G = Hq / Hk in {1, 2, 4, 8, 16}.
+ */
+#ifndef FC_H_
+#define FC_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st* fc_stream;
+
+/* Status codes. */
+enum {
+  FC_OK = 0,
+  FC_ERR_INVALID = 1,      /* null pointer, bad shape, stride, alignment or state */
+  FC_ERR_UNSUPPORTED = 2,  /* valid but outside the supported sizes/dtypes above */
+  FC_ERR_CAPACITY = 3,     /* the archive has too few free blocks; nothing written */
+  FC_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+  FC_ERR_DEVICE = 5        /* a kernel reported an error in the workspace status word */
+};
+
+/* Element types. */
+enum {
+  FC_DTYPE_F32 = 0,
+  FC_DTYPE_BF16 = 1,
+  FC_DTYPE_I8 = 2
+};
+
+/*
+ * Compressed archive of one K or V stream (flashcodec/cache.py, _CodecStream:
+ * coefficients (B, H, capacity, K, D), int8 codes with fp32 scales
+ * (B, H, capacity, K, 1) when quantised, else the stream dtype).
+ *
+ *   coeffs  device, (B, H, capacity, S, D) of coeff_dtype. Within one (b, h)
+ *           the (capacity, S, D) block is contiguous: block stride S*D,
+ *           frequency stride D, element stride 1. 16-byte aligned.
+ *   scales  device, (B, H, capacity, S) fp32, contiguous per (b, h); required
+ *           when coeff_dtype == FC_DTYPE_I8, must be NULL otherwise.
+ *   coeff_dtype  FC_DTYPE_I8 (quantised), FC_DTYPE_BF16 or FC_DTYPE_F32.
+ *   n_blocks     archived blocks per (b, h), 0 <= n_blocks <= capacity; the
+ *                library advances it when it archives blocks.
+ *   *_stride_b / *_stride_h  element strides of the batch and head axes;
+ *                coefficient strides times the element size must be multiples
+ *                of 16 bytes.
+ * Archived blocks are never rewritten by any call (causal safety).
+ */
+typedef struct fc_archive {
+  void* coeffs;
+  float* scales;
+  int32_t coeff_dtype;
+  int32_t R;
+  int32_t S;
+  int32_t reserved;
+  int64_t B, H, D;
+  int64_t capacity;
+  int64_t n_blocks;
+  int64_t coeff_stride_b, coeff_stride_h;
+  int64_t scale_stride_b, scale_stride_h;
+} fc_archive;
+
+/*
+ * Raw tail of one stream: the tokens of the incomplete last block, kept at the
+ * input precision (flashcodec/cache.py, _CodecStream.raw).
+ *
+ *   data    device, (B, H, R, D) of dtype; rows [0, len) are live. Token
+ *           stride D, element stride 1. 16-byte aligned.
+ *   dtype   FC_DTYPE_BF16 or FC_DTYPE_F32 (the stream's input dtype).
+ *   len     0 <= len < R; advanced by fc_append_step / fc_compress_blocks.
+ */
+typedef struct fc_tail {
+  void* data;
+  int32_t dtype;
+  int32_t len;
+  int64_t stride_b, stride_h;
+} fc_tail;
+
+/*
+ * fc_compress_blocks -- archive the complete blocks of a prefill
+ * (flashcodec/cache.py, _CodecStream.append and _archive: the full-block head
+ * is compressed and written as one slice; the remainder stays raw).
+ *
+ *   x        device, (B, H, T, D) tokens of x_dtype (FC_DTYPE_BF16 or
+ *            FC_DTYPE_F32) with element strides x_strides[4]
+ *            (x_strides[3] == 1). Read only.
+ *   T        tokens in x, T >= 0.
+ *   arc      archive; the floor(T / R) complete blocks go to slots
+ *            [arc->n_blocks, arc->n_blocks + floor(T / R)), then n_blocks
+ *            advances. Needs capacity for all of them, else FC_ERR_CAPACITY.
+ *   tail     optional (may be NULL). When given it must have len == 0 and the
+ *            same dtype as x; the T mod R remaining tokens are copied into its
+ *            rows [0, T mod R) and len is set to T mod R. When NULL the caller
+ *            keeps the remainder itself.
+ * One kernel launch (none when there is nothing to do).
+ */
+int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t* x_strides,
+                       int64_t T, fc_archive* arc, fc_tail* tail,
+                       fc_stream stream);
+
+/*
+ * fc_append_step -- append one decode token to the K and V streams
+ * (flashcodec/cache.py, CodecKVCache.decode_step / _CodecStream.append with a
+ * single token): the token is written to tail row `len`; when that fills the
+ * block (len + 1 == R) the R tail tokens are compressed into archive slot
+ * n_blocks, n_blocks advances and len returns to 0.
+ *
+ *   k_new, v_new   device, (B, H, 1, D) of `dtype` (the tails' dtype), element
+ *                  strides k_strides[4] / v_strides[4], innermost 1.
+ *   ka, va         K and V archives (same B, H, R, S, D, n_blocks).
+ *   kt, vt         K and V tails (same len).
+ * FC_ERR_CAPACITY (nothing written) when a block would complete with
+ * n_blocks == capacity: grow the archive (fc_archive_copy_prefix) and retry.
+ * One kernel launch for both streams.
+ */
+int fc_append_step(const void* k_new, const void* v_new, int32_t dtype,
+                   const int64_t* k_strides, const int64_t* v_strides,
+                   fc_archive* ka, fc_archive* va, fc_tail* kt, fc_tail* vt,
+                   fc_stream stream);
+
+/*
+ * fc_archive_copy_prefix -- copy the live blocks [0, src->n_blocks) of every
+ * (b, h) from src into dst and set dst->n_blocks = src->n_blocks: the copy
+ * step of the archive's geometric growth (flashcodec/cache.py,
+ * _CodecStream._grow: capacity starts at 16 blocks and doubles; the old data
+ * is copied verbatim). src and dst must agree on B, H, R, S, D and dtype, and
+ * dst->capacity >= src->n_blocks. One kernel launch.
+ */
+int fc_archive_copy_prefix(const fc_archive* src, fc_archive* dst,
+                           fc_stream stream);
+
+/*
+ * fc_decode_plan -- the split count fc_decode_attention uses when called with
+ * num_splits == 0 for these archives on the current device (chosen to fill the
+ * GPU's SMs; results do not depend on it beyond rounding).
+ */
+int fc_decode_plan(const fc_archive* ka, const fc_tail* kt, int64_t Hq,
+                   int32_t* num_splits_out);
+
+/*
+ * fc_decode_workspace_bytes -- bytes of workspace fc_decode_attention and
+ * fc_combine need for (B, Hq, D, num_splits): a status word, one ticket per
+ * (b, kv head), and the fp32 partials (max, sum, acc[D]) per (b, q head,
+ * split). Returns 0 for invalid sizes.
+ */
+size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
+                                 int32_t num_splits);
+
+/*
+ * fc_decode_attention -- single-token decode attention on the compressed
+ * archive plus the raw tail (flashcodec/triton_attention.py, split and combine
+ * kernels; README "Materialization-free decode attention").
+ *
+ *   q          device, (B, Hq, 1, D) of q_dtype (FC_DTYPE_BF16 or FC_DTYPE_F32),
+ *              element strides q_strides[4], innermost 1. Query head hq reads
+ *              kv head hq / G, G = Hq / Hk.
+ *   ka, va     K and V archives; kt, vt their tails (may be NULL when empty).
+ *              Every archived block and every live tail token is attended;
+ *              there is no mask. n_blocks == 0 is allowed (tail-only softmax);
+ *              n_blocks == 0 with an empty tail is FC_ERR_INVALID.
+ *   softmax_scale   sigma; <= 0 selects D^-0.5.
+ *   num_splits      split-K chunk count, 0 = fc_decode_plan's choice. Chunk c
+ *                   covers blocks [c*chunk, min((c+1)*chunk, n_blocks)); the raw
+ *                   tail belongs to the last chunk.
+ *   fuse_combine    nonzero: the last CTA to finish a kv head merges the
+ *                   partials and writes `out` (one launch, no spin-waits: an
+ *                   atomic ticket). Zero: only the partials are written and
+ *                   fc_combine produces `out`.
+ *   workspace       device, >= fc_decode_workspace_bytes(B, Hq, D, splits)
+ *                   bytes, 256-byte aligned. Its first 256 + 4*B*Hq bytes
+ *                   (status word and tickets) must be zero before the first
+ *                   call; every completed call leaves them zero again. Calls
+ *                   that share a workspace must not overlap on the GPU.
+ *   out        device, (B, Hq, 1, D) of out_dtype (FC_DTYPE_F32 or
+ *              FC_DTYPE_BF16), element strides out_strides[4], innermost 1.
+ * One kernel launch.
+ */
+int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides,
+                        int64_t Hq, const fc_archive* ka, const fc_archive* va,
+                        const fc_tail* kt, const fc_tail* vt,
+                        float softmax_scale, int32_t num_splits,
+                        int32_t fuse_combine, void* workspace,
+                        size_t workspace_bytes, void* out, int32_t out_dtype,
+                        const int64_t* out_strides, fc_stream stream);
+
+/*
+ * fc_combine -- merge split-K partials left in `workspace` by
+ * fc_decode_attention(fuse_combine = 0) (flashcodec/triton_attention.py,
+ * combine kernel): M = max_c m_c, L = sum_c l_c e^(m_c - M),
+ * out = sum_c acc_c e^(m_c - M) / L; chunks with l_c = 0 are skipped.
+ * Sizes must match the producing call. One kernel launch.
+ */
+int fc_combine(const void* workspace, size_t workspace_bytes, int64_t B,
+               int64_t Hq, int64_t D, int32_t num_splits, void* out,
+               int32_t out_dtype, const int64_t* out_strides, fc_stream stream);
+
+/*
+ * fc_workspace_status -- synchronise `stream`, read the workspace status word
+ * into *device_status (0 = no kernel reported a problem) and clear it.
+ * Returns FC_ERR_DEVICE when it was nonzero.
+ */
+int fc_workspace_status(void* workspace, size_t workspace_bytes,
+                        uint32_t* device_status, fc_stream stream);
+
+/*
+ * fc_storage_bytes -- logical storage of one stream: the live archive region
+ * (n_blocks blocks of coefficients, plus their fp32 scales when quantised) and
+ * the live raw tail, excluding idle capacity (flashcodec/cache.py,
+ * _CodecStream.storage_bytes). Host arithmetic only; tail may be NULL.
+ * Returns -1 for an invalid descriptor.
+ */
+int64_t fc_storage_bytes(const fc_archive* arc, const fc_tail* tail);
+
+/* fc_status_string -- static description of a status code. */
+const char* fc_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FC_H_ */

@@ -1,0 +1,181 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol,
+and its host-only logic (validation, workspace sizing, storage accounting)
+behaves; no kernel is launched here."""
+
+import ctypes
+import json
+import os
+import re
+from decimal import Decimal, ROUND_HALF_UP
+
+import pytest
+
+from compressed_decode_attention_blockwise_b200 import _lib
+from compressed_decode_attention_blockwise_b200.archive import grown_capacity
+from oracle.stream import grown_capacity as oracle_grown_capacity
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fc.h")
+FAKE = 0x10000  # aligned non-null address; never dereferenced here
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(
+        r"^\s*(?:const\s+)?[A-Za-z_0-9]+\s*\*?\s+(fc_[a-z_0-9]+)\s*\(", src,
+        flags=re.M)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = declared_functions()
+    assert len(names) == 10, names
+    assert sorted(names) == sorted(_lib.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for code in range(6):
+        assert _lib.fc_status_string(code)
+    assert "unknown" in _lib.fc_status_string(99)
+
+
+def _arc(B=1, H=8, D=64, R=8, S=2, dtype=_lib.FC_DTYPE_I8, cap=16, nb=0):
+    a = _lib.FcArchive()
+    a.coeffs = FAKE
+    a.scales = FAKE if dtype == _lib.FC_DTYPE_I8 else None
+    a.coeff_dtype = dtype
+    a.R, a.S = R, S
+    a.B, a.H, a.D = B, H, D
+    a.capacity, a.n_blocks = cap, nb
+    a.coeff_stride_h = cap * S * D
+    a.coeff_stride_b = H * a.coeff_stride_h
+    a.scale_stride_h = cap * S
+    a.scale_stride_b = H * a.scale_stride_h
+    return a
+
+
+def _tail(a, length=0, dtype=_lib.FC_DTYPE_BF16):
+    t = _lib.FcTail()
+    t.data = FAKE
+    t.dtype = dtype
+    t.len = length
+    t.stride_h = a.R * a.D
+    t.stride_b = a.H * t.stride_h
+    return t
+
+
+def test_storage_bytes_matches_oracle_and_pages():
+    """libfc's storage accounting reproduces the README's cache-footprint
+    table (B*H*D = 512 fp32 streams, r = 8, K and V)."""
+    with open(os.path.join(ROOT, "tests", "golden",
+                           "storage_footprint.json")) as f:
+        gold = json.load(f)
+    for row in gold["rows"]:
+        dt = _lib.FC_DTYPE_I8 if row["quant_bits"] == 8 else _lib.FC_DTYPE_F32
+        nb = row["seq"] // 8
+        a = _arc(B=1, H=8, D=64, R=8, S=row["keep"], dtype=dt, cap=nb, nb=nb)
+        total = 2 * _lib.fc_storage_bytes(a, _tail(a, 0, _lib.FC_DTYPE_F32))
+        mb = Decimal(repr(total / 2 ** 20)).quantize(Decimal("0.1"),
+                                                     ROUND_HALF_UP)
+        assert str(mb) == row["storage"], row
+    # raw tail tokens count at the input precision
+    a = _arc(nb=3)
+    assert _lib.fc_storage_bytes(a, _tail(a, 5)) == \
+        _lib.fc_storage_bytes(a, None) + 1 * 8 * 5 * 64 * 2
+
+
+def test_workspace_bytes():
+    n = _lib.fc_decode_workspace_bytes(2, 8, 128, 3)
+    rows = 2 * 8 * 3
+    pad = lambda x: (x + 255) // 256 * 256
+    assert n == 256 + pad(2 * 8 * 4) + 2 * pad(rows * 4) + pad(rows * 128 * 4)
+    assert _lib.fc_decode_workspace_bytes(0, 8, 128, 3) == 0
+
+
+def test_validation_rejects_bad_arguments_without_launching():
+    lib = _lib.load()
+    a = _arc()
+    t = _tail(a)
+    strides = (ctypes.c_int64 * 4)(8 * 100 * 64, 100 * 64, 64, 1)
+    # null input
+    assert lib.fc_compress_blocks(None, _lib.FC_DTYPE_BF16, strides, 100,
+                                  ctypes.byref(a), None, None) == \
+        _lib.FC_ERR_INVALID
+    # capacity: 100 tokens = 12 blocks > 4 free blocks
+    small = _arc(cap=4)
+    assert lib.fc_compress_blocks(FAKE, _lib.FC_DTYPE_BF16, strides, 100,
+                                  ctypes.byref(small), None, None) == \
+        _lib.FC_ERR_CAPACITY
+    assert small.n_blocks == 0
+    # unsupported head dim, S > R, S above the supported maximum
+    for bad, code in ((_arc(D=100), _lib.FC_ERR_UNSUPPORTED),
+                      (_arc(R=4, S=5), _lib.FC_ERR_INVALID),
+                      (_arc(R=32, S=17), _lib.FC_ERR_UNSUPPORTED)):
+        assert lib.fc_compress_blocks(FAKE, _lib.FC_DTYPE_BF16, strides, 100,
+                                      ctypes.byref(bad), None, None) == code
+    # int8 archive without scales
+    noscale = _arc()
+    noscale.scales = None
+    assert lib.fc_storage_bytes(ctypes.byref(noscale), None) == -1
+    # misaligned coefficient pointer
+    mis = _arc()
+    mis.coeffs = FAKE + 4
+    assert lib.fc_storage_bytes(ctypes.byref(mis), None) == -1
+    # decode: Hq not a multiple of Hk, unsupported group size, empty input
+    q_str = (ctypes.c_int64 * 4)(12 * 64, 64, 64, 1)
+    ws = ctypes.c_void_p(FAKE)
+
+    def attn(Hq, ka, kt=None, vt=None, ns=0):
+        return lib.fc_decode_attention(
+            FAKE, _lib.FC_DTYPE_BF16, q_str, Hq, ctypes.byref(ka),
+            ctypes.byref(ka), None if kt is None else ctypes.byref(kt),
+            None if vt is None else ctypes.byref(vt), 0.0, ns, 1, ws,
+            1 << 30, FAKE, _lib.FC_DTYPE_F32, q_str, None)
+
+    full = _arc(nb=5)
+    assert attn(12, full) == _lib.FC_ERR_INVALID          # 12 % 8
+    assert attn(8 * 3, full) == _lib.FC_ERR_UNSUPPORTED   # G = 3
+    assert attn(8, _arc(nb=0)) == _lib.FC_ERR_INVALID     # nothing to attend
+    assert attn(8, full, _tail(full, 1), None) == _lib.FC_ERR_INVALID
+    assert attn(8, full, ns=10000) == _lib.FC_ERR_INVALID
+    # combine: workspace too small
+    out_str = (ctypes.c_int64 * 4)(8 * 64, 64, 64, 1)
+    assert lib.fc_combine(FAKE, 16, 1, 8, 64, 4, FAKE, _lib.FC_DTYPE_F32,
+                          out_str, None) == _lib.FC_ERR_INVALID
+
+
+def test_append_capacity_error_leaves_state():
+    lib = _lib.load()
+    ka, va = _arc(cap=2, nb=2), _arc(cap=2, nb=2)
+    kt, vt = _tail(ka, 7), _tail(va, 7)
+    s = (ctypes.c_int64 * 4)(8 * 64, 64, 64, 1)
+    st = lib.fc_append_step(FAKE, FAKE, _lib.FC_DTYPE_BF16, s, s,
+                            ctypes.byref(ka), ctypes.byref(va),
+                            ctypes.byref(kt), ctypes.byref(vt), None)
+    assert st == _lib.FC_ERR_CAPACITY
+    assert (ka.n_blocks, kt.len, vt.len) == (2, 7, 7)
+    # mismatched tail lengths
+    vt.len = 6
+    st = lib.fc_append_step(FAKE, FAKE, _lib.FC_DTYPE_BF16, s, s,
+                            ctypes.byref(ka), ctypes.byref(va),
+                            ctypes.byref(kt), ctypes.byref(vt), None)
+    assert st == _lib.FC_ERR_INVALID
+
+
+@pytest.mark.parametrize("cap,need", [(0, 1), (0, 16), (16, 17), (32, 100),
+                                      (128, 100), (0, 1000)])
+def test_capacity_policy_matches_oracle(cap, need):
+    assert grown_capacity(cap, need) == oracle_grown_capacity(cap, need)
+
+
+def test_product_path_has_no_oracle_or_fallback():
+    """The package never imports the oracle and has no CPU compute path."""
+    pkg = os.path.join(ROOT, "compressed_decode_attention_blockwise_b200")
+    for fn in os.listdir(pkg):
+        if fn.endswith(".py"):
+            src = open(os.path.join(pkg, fn)).read()
+            assert "oracle" not in src, fn
+            assert "numpy" not in src, fn
