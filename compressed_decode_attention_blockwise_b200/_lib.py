@@ -23,6 +23,9 @@ FC_ERR_CAPACITY = 3
 FC_ERR_CUDA = 4
 FC_ERR_DEVICE = 5
 
+FC_DECODE_FUSE_COMBINE = 1
+FC_DECODE_PORTABLE = 2
+
 FC_DTYPE_F32 = 0
 FC_DTYPE_BF16 = 1
 FC_DTYPE_I8 = 2
@@ -203,14 +206,17 @@ def fc_decode_attention(q: torch.Tensor, ka: FcArchive, va: FcArchive,
                         kt: Optional[FcTail], vt: Optional[FcTail],
                         out: torch.Tensor, workspace: Optional[torch.Tensor],
                         softmax_scale: float = 0.0, num_splits: int = 0,
-                        fuse_combine: bool = True, stream=None) -> None:
+                        fuse_combine: bool = True, portable: bool = False,
+                        stream=None) -> None:
     ws_ptr = _ptr(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * \
         workspace.element_size()
+    flags = (FC_DECODE_FUSE_COMBINE if fuse_combine else 0) | \
+        (FC_DECODE_PORTABLE if portable else 0)
     st = load().fc_decode_attention(
         _ptr(q), dtype_code(q.dtype), _strides4(q), q.shape[1],
         ctypes.byref(ka), ctypes.byref(va), _ref(kt), _ref(vt),
-        float(softmax_scale), int(num_splits), 1 if fuse_combine else 0,
+        float(softmax_scale), int(num_splits), flags,
         ws_ptr, ws_bytes, _ptr(out), dtype_code(out.dtype), _strides4(out),
         _stream(stream, q))
     _check(st, "fc_decode_attention")

@@ -192,9 +192,11 @@ class CodecKVCache:
 
     def attention(self, q: torch.Tensor, out: Optional[torch.Tensor] = None,
                   softmax_scale: Optional[float] = None, num_splits: int = 0,
-                  fuse_combine: bool = True,
+                  fuse_combine: bool = True, portable: bool = False,
                   out_dtype: torch.dtype = torch.float32) -> torch.Tensor:
-        """Decode attention of q (B, Hq, 1, D) over archive + tail."""
+        """Decode attention of q (B, Hq, 1, D) over archive + tail.
+        ``portable`` forces the CUDA-core kernel where the tensor-core kernel
+        would apply."""
         Hq = q.shape[1]
         if out is None:
             out = torch.empty((self.B, Hq, 1, self.D), dtype=out_dtype,
@@ -204,7 +206,8 @@ class CodecKVCache:
         _lib.fc_decode_attention(
             q, self.k.arc, self.v.arc, self.k.tail_desc, self.v.tail_desc,
             out, ws, softmax_scale=0.0 if softmax_scale is None else
-            float(softmax_scale), num_splits=ns, fuse_combine=fuse_combine)
+            float(softmax_scale), num_splits=ns, fuse_combine=fuse_combine,
+            portable=portable)
         if not fuse_combine:
             _lib.fc_combine(ws, self.B, Hq, self.D, ns, out)
         return out

@@ -7,15 +7,18 @@
 namespace fc {
 namespace {
 
-// Split count: enough (chunk, kv head, batch) CTAs to give every SM about four,
-// but no chunk shorter than 16 blocks (the partials then stay a small fraction
-// of the archive bytes).
-int plan_splits(int64_t nb, int64_t B, int64_t Hk) {
+// Split count. The tensor-core kernel runs 128-row tiles at two CTAs per SM:
+// split each kv head into enough tile-aligned chunks to give every SM two
+// CTAs. The portable kernel aims at four CTAs per SM with chunks of at least
+// 16 blocks. Results do not depend on the split beyond rounding.
+int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   if (nb <= 0) return 1;
   const int64_t units = B * Hk;
-  const int64_t target = int64_t(sm_count()) * 4;
+  const bool tiles = D == 128 && S >= 1 && 32 % S == 0;
+  const int64_t per_sm = tiles ? 2 : 4;
+  const int64_t target = int64_t(sm_count()) * per_sm;
   int64_t ns = (target + units - 1) / units;
-  const int64_t by_len = nb / 16 > 0 ? nb / 16 : 1;
+  const int64_t by_len = tiles ? tc_tiles_per_head(nb, S) : (nb / 16 > 0 ? nb / 16 : 1);
   if (ns > by_len) ns = by_len;
   if (ns > kMaxSplits) ns = kMaxSplits;
   if (ns < 1) ns = 1;
@@ -28,8 +31,8 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   extern __shared__ float wts[];  // ns + 1
   const int hq = blockIdx.x, b = blockIdx.y;
   const int64_t row = (int64_t(b) * a.Hq + hq) * a.ns;
-  combine_head(a.pm + row, a.pl + row, a.pacc + row * a.D, a.ns, a.D, wts, a.out,
-               b * a.os_b + hq * a.os_h, a.out_dtype);
+  combine_heads(a.pm + row, a.pl + row, a.pacc + row * a.D, 1, a.ns, a.D, wts, a.out,
+                b * a.os_b + hq * a.os_h, a.os_h, a.out_dtype);
 }
 
 int check_io(const void* p, int dtype, const int64_t* strides) {
@@ -51,14 +54,14 @@ extern "C" int fc_decode_plan(const fc_archive* ka, const fc_tail* kt, int64_t H
   const int st = check_archive(ka);
   if (st != FC_OK) return st;
   if (Hq < 1 || Hq % ka->H) return FC_ERR_INVALID;
-  *num_splits_out = plan_splits(ka->n_blocks, ka->B, ka->H);
+  *num_splits_out = plan_splits(ka->n_blocks, ka->B, ka->H, ka->S, int(ka->D));
   return FC_OK;
 }
 
 extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides,
                                    int64_t Hq, const fc_archive* ka, const fc_archive* va,
                                    const fc_tail* kt, const fc_tail* vt, float softmax_scale,
-                                   int32_t num_splits, int32_t fuse_combine, void* workspace,
+                                   int32_t num_splits, int32_t flags, void* workspace,
                                    size_t workspace_bytes, void* out, int32_t out_dtype,
                                    const int64_t* out_strides, fc_stream stream) {
   int st = check_archive(ka);
@@ -90,8 +93,10 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
   }
   if (ka->n_blocks == 0 && nr == 0) return FC_ERR_INVALID;
   int ns = num_splits;
-  if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H);
+  if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H, ka->S, int(ka->D));
   if (ns < 1 || ns > kMaxSplits) return FC_ERR_INVALID;
+  if (flags & ~(FC_DECODE_FUSE_COMBINE | FC_DECODE_PORTABLE)) return FC_ERR_INVALID;
+  const bool fuse_combine = (flags & FC_DECODE_FUSE_COMBINE) != 0;
   if (ka->B > 65535 || ka->H > 65535) return FC_ERR_UNSUPPORTED;
   const bool need_ws = !(fuse_combine && ns == 1);
   const WorkspaceLayout wl = workspace_layout(ka->B, Hq, ka->D, ns);
@@ -149,6 +154,8 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
   a.os_h = out_strides[1];
   Basis basis;
   make_basis(ka->R, ka->S, &basis);
+  if (!(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, int(G)))
+    return launch_decode_tc(a, ka, va, basis, stream);
   const int kd = ka->coeff_dtype, vd = va->coeff_dtype;
   if (kd == FC_DTYPE_I8 && vd == FC_DTYPE_I8) return launch_decode_generic<int8_t, int8_t>(a, basis, stream);
   if (kd == FC_DTYPE_I8 && vd == FC_DTYPE_BF16)

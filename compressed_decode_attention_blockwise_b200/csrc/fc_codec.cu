@@ -12,11 +12,16 @@
 // Work mapping: one warp per (b, h, block); lane l owns the VEC = D / 32
 // consecutive channels [l * VEC, (l + 1) * VEC), so every token row is one
 // coalesced warp-wide load and every coefficient row one coalesced store. The
-// S x VEC coefficients accumulate in registers in fp32 (t ascending, fused
-// multiply-add), the absmax is a warp-shuffle max, and the quantiser divides in
-// fp32 with round-to-nearest-even. Compression of a prefill and of an appended
-// block run the same device code in the same order, so an archive built token
-// by token is bitwise identical to one built in a single call.
+// coefficients accumulate in registers in fp64 (t ascending, fused
+// multiply-add, four frequencies per pass over the block's rows), the absmax
+// is a warp-shuffle max, and the quantiser takes its rounding decision in fp64
+// (round-to-nearest-even of C times the reciprocal scale), so codes agree with
+// an fp64 evaluation of the definition except where C / scale lies within a
+// few fp64 ulps of a half-integer; unquantised coefficients are rounded from
+// fp64 straight to the storage dtype. The fp64 work stays below the HBM
+// stream's time on sm_100a. Compression of a prefill and of an appended block
+// run the same device code in the same order, so an archive built token by
+// token is bitwise identical to one built in a single call.
 #include <type_traits>
 
 #include "fc_internal.cuh"
@@ -31,17 +36,12 @@ struct StreamOut {
   int64_t ss_b, ss_h;  // scale element strides
 };
 
-template <int VEC, int SMAX>
-__device__ __forceinline__ void accum_row(float (&c)[SMAX][VEC], const float (&x)[VEC],
-                                          const Basis& basis, int t, int S) {
+constexpr int kJC = 4;  // frequencies per pass over a block's rows
+
+__device__ __forceinline__ double warp_max_d(double v) {
 #pragma unroll
-  for (int j = 0; j < SMAX; ++j) {
-    if (j < S) {
-      const float m = basis.m[j][t];
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) c[j][v] = fmaf(m, x[v], c[j][v]);
-    }
-  }
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
 }
 
 template <int VEC>
@@ -100,35 +100,85 @@ __device__ __forceinline__ void store_row(T* p, const float (&x)[VEC]) {
   }
 }
 
-// Quantises (int8) or rounds (bf16 / f32) the S coefficient rows of one block
-// and stores them at `blk` (S x D elements) / `scl` (S floats).
-template <typename TOut, int VEC, int SMAX>
-__device__ __forceinline__ void store_block(const float (&c)[SMAX][VEC], int S, int D, int lane,
-                                            TOut* blk, float* scl) {
+template <int VEC>
+__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* p, const __nv_bfloat16 (&h)[VEC]) {
+  if constexpr (VEC == 1) {
+    p[0] = h[0];
+  } else {
+    uint32_t w[VEC / 2];
 #pragma unroll
-  for (int j = 0; j < SMAX; ++j) {
-    if (j < S) {
-      if constexpr (std::is_same_v<TOut, int8_t>) {
-        float amax = 0.f;
+    for (int i = 0; i < VEC / 2; ++i)
+      w[i] = uint32_t(__bfloat16_as_ushort(h[2 * i])) | (uint32_t(__bfloat16_as_ushort(h[2 * i + 1])) << 16);
+    if constexpr (VEC == 2) {
+      *reinterpret_cast<uint32_t*>(p) = w[0];
+    } else if constexpr (VEC == 4) {
+      *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+    } else {
+      *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+// Quantises (int8) or rounds (bf16 / f32) one coefficient row held in fp64
+// and stores it at `row` (D elements; lane owns VEC) and, for int8, its scale.
+template <typename TOut, int VEC>
+__device__ __forceinline__ void store_coeff_row(const double (&c)[VEC], int lane, TOut* row,
+                                                float* scl) {
+  if constexpr (std::is_same_v<TOut, int8_t>) {
+    double amax = 0.0;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) amax = fmaxf(amax, fabsf(c[j][v]));
-        amax = warp_max(amax);
-        const float scale = amax / 127.0f;
-        int code[VEC];
+    for (int v = 0; v < VEC; ++v) amax = fmax(amax, fabs(c[v]));
+    amax = warp_max_d(amax);
+    const double scale = amax / 127.0;
+    const double inv = amax > 0.0 ? 1.0 / scale : 0.0;
+    int code[VEC];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-          int q = 0;
-          if (scale > 0.f) q = __float2int_rn(c[j][v] / scale);
-          code[v] = max(-127, min(127, q));
+    for (int v = 0; v < VEC; ++v) code[v] = max(-127, min(127, __double2int_rn(c[v] * inv)));
+    store_codes<VEC>(row + lane * VEC, code);
+    if (lane == 0) *scl = __double2float_rn(scale);
+  } else if constexpr (std::is_same_v<TOut, float>) {
+    float x[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) x[v] = __double2float_rn(c[v]);
+    store_row<float, VEC>(row + lane * VEC, x);
+  } else {
+    // direct fp64 -> bf16 rounding, packed in pairs
+    __nv_bfloat16 hb[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) hb[v] = __double2bfloat16(c[v]);
+    store_bf16_row<VEC>(row + lane * VEC, hb);
+  }
+}
+
+// Encodes the S kept frequencies of one block whose R token rows come from
+// `row_at(t, xf)` (VEC floats of row t for this lane), kJC frequencies per
+// pass, and stores them at `blk` (S x D elements) / `scl` (S floats).
+template <typename TOut, int VEC, typename RowAt>
+__device__ __forceinline__ void encode_block(RowAt&& row_at, int R, int S, int D, int lane,
+                                             const BasisF64& basis, TOut* blk, float* scl) {
+  for (int j0 = 0; j0 < S; j0 += kJC) {
+    double c[kJC][VEC];
+#pragma unroll
+    for (int jj = 0; jj < kJC; ++jj)
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) c[jj][v] = 0.0;
+#pragma unroll 4
+    for (int t = 0; t < R; ++t) {
+      float xf[VEC];
+      row_at(t, xf);
+#pragma unroll
+      for (int jj = 0; jj < kJC; ++jj) {
+        if (j0 + jj < S) {
+          const double m = basis.m[j0 + jj][t];
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) c[jj][v] = fma(m, double(xf[v]), c[jj][v]);
         }
-        store_codes<VEC>(blk + int64_t(j) * D + lane * VEC, code);
-        if (lane == 0) scl[j] = scale;
-      } else {
-        float row[VEC];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) row[v] = c[j][v];
-        store_row<TOut, VEC>(blk + int64_t(j) * D + lane * VEC, row);
       }
+    }
+#pragma unroll
+    for (int jj = 0; jj < kJC; ++jj) {
+      const int j = j0 + jj;
+      if (j < S) store_coeff_row<TOut, VEC>(c[jj], lane, blk + int64_t(j) * D, scl ? scl + j : nullptr);
     }
   }
 }
@@ -144,8 +194,8 @@ struct CompressArgs {
   int n_rem;
 };
 
-template <int VEC, int SMAX, typename TIn, typename TOut>
-__global__ void __launch_bounds__(256) compress_blocks_kernel(CompressArgs a, Basis basis) {
+template <int VEC, typename TIn, typename TOut>
+__global__ void __launch_bounds__(256) compress_blocks_kernel(CompressArgs a, BasisF64 basis) {
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t n_items = int64_t(a.B) * a.H * a.n_full;
@@ -155,22 +205,12 @@ __global__ void __launch_bounds__(256) compress_blocks_kernel(CompressArgs a, Ba
     const int64_t bh = w / a.n_full;
     const int h = int(bh % a.H), b = int(bh / a.H);
     const TIn* src = x + b * a.xs_b + h * a.xs_h + n * a.R * a.xs_t + lane * VEC;
-    float c[SMAX][VEC];
-#pragma unroll
-    for (int j = 0; j < SMAX; ++j)
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) c[j][v] = 0.f;
-#pragma unroll 4
-    for (int t = 0; t < a.R; ++t) {
-      float xv[VEC];
-      load_vec<TIn, VEC>(src + t * a.xs_t, xv);
-      accum_row<VEC, SMAX>(c, xv, basis, t, a.S);
-    }
     TOut* blk = static_cast<TOut*>(a.out.coeffs) + b * a.out.cs_b + h * a.out.cs_h +
                 (a.slot0 + n) * a.S * a.D;
     float* scl = a.out.scales ? a.out.scales + b * a.out.ss_b + h * a.out.ss_h + (a.slot0 + n) * a.S
                               : nullptr;
-    store_block<TOut, VEC, SMAX>(c, a.S, a.D, lane, blk, scl);
+    encode_block<TOut, VEC>([&](int t, float (&xf)[VEC]) { load_vec<TIn, VEC>(src + t * a.xs_t, xf); },
+                            a.R, a.S, a.D, lane, basis, blk, scl);
   } else if (a.tail != nullptr && w < n_items + int64_t(a.B) * a.H) {
     // copy the T mod R remaining tokens of (b, h) into its raw tail rows
     const int64_t bh = w - n_items;
@@ -201,8 +241,8 @@ struct AppendArgs {
   int64_t slot;
 };
 
-template <int VEC, int SMAX, typename TIn, typename TOutK, typename TOutV>
-__global__ void __launch_bounds__(256) append_step_kernel(AppendArgs a, Basis basis) {
+template <int VEC, typename TIn, typename TOutK, typename TOutV>
+__global__ void __launch_bounds__(256) append_step_kernel(AppendArgs a, BasisF64 basis) {
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t bh_total = int64_t(a.B) * a.H;
@@ -219,25 +259,22 @@ __global__ void __launch_bounds__(256) append_step_kernel(AppendArgs a, Basis ba
     return;
   }
   // the block completes: rows 0..R-2 come from the tail, row R-1 is the new token
-  float c[SMAX][VEC];
+  auto row_at = [&](int t, float (&xf)[VEC]) {
+    if (t < a.R - 1) {
+      load_vec<TIn, VEC>(trow + int64_t(t) * a.D, xf);
+    } else {
 #pragma unroll
-  for (int j = 0; j < SMAX; ++j)
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) c[j][v] = 0.f;
-  for (int t = 0; t < a.R - 1; ++t) {
-    float xv[VEC];
-    load_vec<TIn, VEC>(trow + int64_t(t) * a.D, xv);
-    accum_row<VEC, SMAX>(c, xv, basis, t, a.S);
-  }
-  accum_row<VEC, SMAX>(c, xn, basis, a.R - 1, a.S);
+      for (int v = 0; v < VEC; ++v) xf[v] = xn[v];
+    }
+  };
   const StreamOut& o = st.out;
   float* scl = o.scales ? o.scales + b * o.ss_b + h * o.ss_h + a.slot * a.S : nullptr;
   if (s == 0) {
     TOutK* blk = static_cast<TOutK*>(o.coeffs) + b * o.cs_b + h * o.cs_h + a.slot * a.S * a.D;
-    store_block<TOutK, VEC, SMAX>(c, a.S, a.D, lane, blk, scl);
+    encode_block<TOutK, VEC>(row_at, a.R, a.S, a.D, lane, basis, blk, scl);
   } else {
     TOutV* blk = static_cast<TOutV*>(o.coeffs) + b * o.cs_b + h * o.cs_h + a.slot * a.S * a.D;
-    store_block<TOutV, VEC, SMAX>(c, a.S, a.D, lane, blk, scl);
+    encode_block<TOutV, VEC>(row_at, a.R, a.S, a.D, lane, basis, blk, scl);
   }
 }
 
@@ -282,12 +319,6 @@ int dispatch_vec(int D, F&& f) {
     case 256: return f(std::integral_constant<int, 8>{});
     default: return FC_ERR_UNSUPPORTED;
   }
-}
-
-template <typename F>
-int dispatch_smax(int S, F&& f) {
-  if (S <= 4) return f(std::integral_constant<int, 4>{});
-  return f(std::integral_constant<int, 16>{});
 }
 
 template <typename F>
@@ -362,21 +393,18 @@ extern "C" int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t*
   a.ts_b = tail ? tail->stride_b : 0;
   a.ts_h = tail ? tail->stride_h : 0;
   a.n_rem = n_rem;
-  Basis basis;
-  make_basis(arc->R, arc->S, &basis);
+  BasisF64 basis;
+  make_basis_f64(arc->R, arc->S, &basis);
   const int64_t warps = arc->B * arc->H * n_full + (copy_tail ? arc->B * arc->H : 0);
   const int64_t grid = (warps + 7) / 8;
   if (grid > 0x7fffffffLL) return FC_ERR_UNSUPPORTED;
   st = dispatch_vec(a.D, [&](auto vec) {
-    return dispatch_smax(a.S, [&](auto smax) {
-      return dispatch_in(x_dtype, [&](auto tin) {
-        return dispatch_out(arc->coeff_dtype, [&](auto tout) {
-          using TIn = decltype(tin);
-          using TOut = decltype(tout);
-          compress_blocks_kernel<decltype(vec)::value, decltype(smax)::value, TIn, TOut>
-              <<<unsigned(grid), 256, 0, stream>>>(a, basis);
-          return cuda_status(cudaGetLastError());
-        });
+    return dispatch_in(x_dtype, [&](auto tin) {
+      return dispatch_out(arc->coeff_dtype, [&](auto tout) {
+        using TIn = decltype(tin);
+        using TOut = decltype(tout);
+        compress_blocks_kernel<decltype(vec)::value, TIn, TOut><<<unsigned(grid), 256, 0, stream>>>(a, basis);
+        return cuda_status(cudaGetLastError());
       });
     });
   });
@@ -432,19 +460,17 @@ extern "C" int fc_append_step(const void* k_new, const void* v_new, int32_t dtyp
   a.len = kt->len;
   a.complete = complete ? 1 : 0;
   a.slot = ka->n_blocks;
-  Basis basis;
-  make_basis(ka->R, ka->S, &basis);
+  BasisF64 basis;
+  make_basis_f64(ka->R, ka->S, &basis);
   const int64_t warps = 2 * ka->B * ka->H;
   const int64_t grid = (warps + 7) / 8;
   st = dispatch_vec(a.D, [&](auto vec) {
-    return dispatch_smax(a.S, [&](auto smax) {
-      return dispatch_in(dtype, [&](auto tin) {
-        return dispatch_out(ka->coeff_dtype, [&](auto tk) {
-          return dispatch_out(va->coeff_dtype, [&](auto tv) {
-            append_step_kernel<decltype(vec)::value, decltype(smax)::value, decltype(tin),
-                               decltype(tk), decltype(tv)><<<unsigned(grid), 256, 0, stream>>>(a, basis);
-            return cuda_status(cudaGetLastError());
-          });
+    return dispatch_in(dtype, [&](auto tin) {
+      return dispatch_out(ka->coeff_dtype, [&](auto tk) {
+        return dispatch_out(va->coeff_dtype, [&](auto tv) {
+          append_step_kernel<decltype(vec)::value, decltype(tin), decltype(tk), decltype(tv)>
+              <<<unsigned(grid), 256, 0, stream>>>(a, basis);
+          return cuda_status(cudaGetLastError());
         });
       });
     });

@@ -71,38 +71,58 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, int dtype, flo
     static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
-// Merges the ns partials of one query head (rows pm[0..ns), pl[0..ns),
-// pacc[0..ns)[D]) into out[0..D). Needs ns + 1 floats of shared scratch
-// `wts`; all threads of the CTA take part. Partials written by other CTAs of
-// the same launch are read through L2 (ld.cg).
-__device__ __forceinline__ void combine_head(const float* pm, const float* pl, const float* pacc,
-                                             int ns, int D, float* wts, void* out, int64_t out_off,
-                                             int out_dtype) {
+// Merges the ns split partials of NH consecutive query heads into their
+// outputs: M = max_c m_c, L = sum_c l_c e^(m_c - M), out = sum_c acc_c
+// e^(m_c - M) / L, chunks with l_c = 0 skipped (base-2 exponentials: the
+// partial maxima are kept in log2 units). Head i's partials are rows
+// pm[i * ns + c], pl[i * ns + c], pacc[(i * ns + c) * D + d]; its output goes to
+// out[out_off + i * out_stride_h + d]. All threads of the CTA take part: warps
+// compute the per-head weights into shared scratch `wts` (NH * (ns + 1)
+// floats), then every thread merges (head, channel) pairs with independent,
+// batched L2 loads. Partials written by other CTAs of the same launch are read
+// through L2 (ld.cg).
+__device__ __forceinline__ void combine_heads(const float* pm, const float* pl, const float* pacc, int NH,
+                                              int ns, int D, float* wts, void* out, int64_t out_off,
+                                              int64_t out_stride_h, int out_dtype) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (warp == 0) {
+  const int nwarps = blockDim.x >> 5;
+  for (int i = warp; i < NH; i += nwarps) {
+    const float* m = pm + int64_t(i) * ns;
+    const float* l = pl + int64_t(i) * ns;
+    float* w = wts + i * (ns + 1);
     float mx = -INFINITY;
     for (int c = lane; c < ns; c += 32)
-      if (__ldcg(pl + c) > 0.f) mx = fmaxf(mx, __ldcg(pm + c));
+      if (__ldcg(l + c) > 0.f) mx = fmaxf(mx, __ldcg(m + c));
     mx = warp_max(mx);
     float L = 0.f;
     for (int c = lane; c < ns; c += 32) {
-      const float lc = __ldcg(pl + c);
-      const float e = lc > 0.f ? exp2f(__ldcg(pm + c) - mx) : 0.f;
-      wts[c] = e;
+      const float lc = __ldcg(l + c);
+      const float e = lc > 0.f ? exp2f(__ldcg(m + c) - mx) : 0.f;
+      w[c] = e;
       L = fmaf(lc, e, L);
     }
     L = warp_sum(L);
-    if (lane == 0) wts[ns] = 1.f / L;
+    if (lane == 0) w[ns] = 1.f / L;
   }
   __syncthreads();
-  const float inv = wts[ns];
-  for (int d = tid; d < D; d += blockDim.x) {
-    float acc = 0.f;
-    for (int c = 0; c < ns; ++c) {
-      const float e = wts[c];
-      if (e != 0.f) acc = fmaf(__ldcg(pacc + int64_t(c) * D + d), e, acc);
+  for (int idx = tid; idx < NH * D; idx += blockDim.x) {
+    const int i = idx / D, d = idx - (idx / D) * D;
+    const float* w = wts + i * (ns + 1);
+    const float* src = pacc + int64_t(i) * ns * D + d;
+    float acc0 = 0.f, acc1 = 0.f;
+    int c = 0;
+    for (; c + 8 <= ns; c += 8) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + int64_t(c + u) * D);
+#pragma unroll
+      for (int u = 0; u < 8; u += 2) {
+        acc0 = fmaf(v[u], w[c + u], acc0);
+        acc1 = fmaf(v[u + 1], w[c + u + 1], acc1);
+      }
     }
-    store_out(out, out_off + d, out_dtype, acc * inv);
+    for (; c < ns; ++c) acc0 = fmaf(__ldcg(src + int64_t(c) * D), w[c], acc0);
+    store_out(out, out_off + i * out_stride_h + d, out_dtype, (acc0 + acc1) * w[ns]);
   }
   __syncthreads();
 }
@@ -160,12 +180,9 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs& a, int b, int h, in
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int g = 0; g < G; ++g) {
-    const int hq = h * G + g;
-    const int64_t row = (int64_t(b) * Hq + hq) * a.ns;
-    combine_head(a.pm + row, a.pl + row, a.pacc + row * D, a.ns, D, scratch, a.out,
-                 b * a.os_b + hq * a.os_h, a.out_dtype);
-  }
+  const int64_t row = (int64_t(b) * Hq + h * G) * a.ns;
+  combine_heads(a.pm + row, a.pl + row, a.pacc + row * D, G, a.ns, D, scratch, a.out,
+                b * a.os_b + (h * G) * a.os_h, a.os_h, a.out_dtype);
   if (tid == 0) a.tickets[b * a.Hk + h] = 0u;
 }
 
@@ -319,14 +336,21 @@ __global__ void __launch_bounds__(kGenericWarps * 32)
   finish_cta<NW>(a, b, h, c, mrg_m, mrg_l, dyn, dyn + NW * G * D);
 }
 
-// Shared memory (bytes) the generic kernel needs beyond its static arrays.
+// Shared memory (bytes) the generic kernel needs beyond its static arrays:
+// the warp-merge buffer, followed by the combine weights.
 inline size_t generic_dyn_smem(int G, int D, int ns) {
-  return size_t(kGenericWarps * G * D + ns + 1) * sizeof(float);
+  return size_t(kGenericWarps * G * D + G * (ns + 1)) * sizeof(float);
 }
 
 // Launchers, one explicit instantiation per (K, V) coefficient type pair.
 template <typename KT, typename VT>
 int launch_decode_generic(const DecodeArgs& a, const Basis& basis, cudaStream_t stream);
+
+// Tensor-core kernel for int8 K and V archives (fc_decode_tc.cu).
+bool decode_tc_eligible(const fc_archive* ka, const fc_archive* va, int G);
+int tc_tiles_per_head(int64_t nb, int S);
+int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive* va, const Basis& basis,
+                     cudaStream_t stream);
 
 // Combine kernel for fc_combine: one CTA per (b, q head).
 struct CombineArgs {

@@ -22,6 +22,19 @@ void make_basis(int R, int S, Basis* out) {
     }
 }
 
+void make_basis_f64(int R, int S, BasisF64* out) {
+  const double pi = 3.14159265358979323846;
+  for (int j = 0; j < kMaxS; ++j)
+    for (int t = 0; t < kMaxR; ++t) {
+      double v = 0.0;
+      if (j < S && t < R) {
+        const double c = (j == 0) ? std::sqrt(1.0 / R) : std::sqrt(2.0 / R);
+        v = c * std::cos(pi / R * (t + 0.5) * j);
+      }
+      out->m[j][t] = v;
+    }
+}
+
 int sm_count() {
   static std::mutex mu;
   static int cache[64] = {0};

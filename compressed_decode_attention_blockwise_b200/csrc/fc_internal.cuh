@@ -22,6 +22,13 @@ struct Basis {
 // Host: fills M[j][t] = c_j cos(pi / R (t + 1/2) j) in double, rounded to fp32.
 void make_basis(int R, int S, Basis* out);
 
+// The same rows in double precision (used by the compression kernels, which
+// take the quantiser's rounding decision in fp64).
+struct BasisF64 {
+  double m[kMaxS][kMaxR];
+};
+void make_basis_f64(int R, int S, BasisF64* out);
+
 // Host: SM count of the current device (cached per device).
 int sm_count();
 

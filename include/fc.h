@@ -57,6 +57,12 @@ enum {
   FC_ERR_DEVICE = 5        /* a kernel reported an error in the workspace status word */
 };
 
+/* fc_decode_attention flags. */
+enum {
+  FC_DECODE_FUSE_COMBINE = 1, /* the last CTA of each kv head writes `out` */
+  FC_DECODE_PORTABLE = 2      /* force the portable CUDA-core kernel */
+};
+
 /* Element types. */
 enum {
   FC_DTYPE_F32 = 0,
@@ -198,10 +204,13 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *   num_splits      split-K chunk count, 0 = fc_decode_plan's choice. Chunk c
  *                   covers blocks [c*chunk, min((c+1)*chunk, n_blocks)); the raw
  *                   tail belongs to the last chunk.
- *   fuse_combine    nonzero: the last CTA to finish a kv head merges the
- *                   partials and writes `out` (one launch, no spin-waits: an
- *                   atomic ticket). Zero: only the partials are written and
- *                   fc_combine produces `out`.
+ *   flags      FC_DECODE_FUSE_COMBINE: the last CTA to finish a kv head
+ *              merges the partials and writes `out` (one launch, no
+ *              spin-waits: an atomic ticket); without it only the partials
+ *              are written and fc_combine produces `out`.
+ *              FC_DECODE_PORTABLE: use the portable CUDA-core kernel even
+ *              where the tensor-core kernel applies (int8 K and V, D = 128,
+ *              S dividing 32, R / S in {2, 4, 8}, G <= 8).
  *   workspace       device, >= fc_decode_workspace_bytes(B, Hq, D, splits)
  *                   bytes, 256-byte aligned. Its first 256 + 4*B*Hq bytes
  *                   (status word and tickets) must be zero before the first
@@ -215,13 +224,13 @@ int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides
                         int64_t Hq, const fc_archive* ka, const fc_archive* va,
                         const fc_tail* kt, const fc_tail* vt,
                         float softmax_scale, int32_t num_splits,
-                        int32_t fuse_combine, void* workspace,
+                        int32_t flags, void* workspace,
                         size_t workspace_bytes, void* out, int32_t out_dtype,
                         const int64_t* out_strides, fc_stream stream);
 
 /*
  * fc_combine -- merge split-K partials left in `workspace` by
- * fc_decode_attention(fuse_combine = 0) (flashcodec/triton_attention.py,
+ * fc_decode_attention without FC_DECODE_FUSE_COMBINE (flashcodec/triton_attention.py,
  * combine kernel): M = max_c m_c, L = sum_c l_c e^(m_c - M),
  * out = sum_c acc_c e^(m_c - M) / L; chunks with l_c = 0 are skipped.
  * Sizes must match the producing call. One kernel launch.

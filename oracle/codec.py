@@ -72,8 +72,10 @@ def quantize(C: np.ndarray, decision: str = "f64"):
 
     Returns ``(codes int8, scale fp64, y)`` where ``y = C / scale`` is the
     pre-rounding value (0 for an all-zero row). ``decision='f64'`` divides in
-    float64; ``decision='f32'`` rounds C and the scale to float32 first and
-    divides in float32, the precision the GPU kernel decides in.
+    float64, the precision the GPU kernel takes the decision in;
+    ``decision='f32'`` rounds C and the scale to float32 first and divides in
+    float32, an alternative reading used only to bound how far the two
+    precisions can disagree.
     The stored scale is ``float32(scale)`` in both cases.
     """
     C = np.asarray(C, dtype=F64)

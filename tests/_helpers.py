@@ -53,7 +53,14 @@ def check_coeffs(gpu: np.ndarray, C: np.ndarray, coeff: str):
         ref = oracle.round_to_dtype(C, "bf16")
         mag = np.maximum(np.abs(ref), np.abs(gpu)) + 1e-300
         ulp = np.ldexp(1.0, np.frexp(mag)[1] - 8)
-        assert np.all(np.abs(gpu - ref) <= ulp), "bf16 coefficient mismatch"
+        bad = np.abs(gpu - ref) > ulp
+        if bad.any():
+            k = tuple(np.argwhere(bad)[0])
+            raise AssertionError(
+                "bf16 coefficient mismatch at %d positions; first %s: gpu %r "
+                "ref %r exact %r (max %.3g ulp)" % (
+                    int(bad.sum()), k, float(gpu[k]), float(ref[k]),
+                    float(C[k]), float(np.max(np.abs(gpu - ref) / ulp))))
     else:
         scale = np.max(np.abs(C), axis=(-2, -1), keepdims=True)
         err = np.abs(gpu - C)

@@ -51,11 +51,14 @@ def test_small_cases_match_oracle(case):
     cache, data = _cache_for(w)
     q = data["q"].to(DEV)
     ref = oracle_on_gpu_archive(cache, q)
-    for ns in (0, 1, 2, 3, 7, nb, nb + 3):
-        for fuse in (True, False):
-            out = cache.attention(q, num_splits=ns, fuse_combine=fuse)
-            torch.cuda.synchronize()
-            check_out(f64(out), ref, "ns=%d fuse=%s" % (ns, fuse))
+    for portable in (False, True):
+        for ns in (0, 1, 2, 3, 7, nb, nb + 3):
+            for fuse in (True, False):
+                out = cache.attention(q, num_splits=ns, fuse_combine=fuse,
+                                      portable=portable)
+                torch.cuda.synchronize()
+                check_out(f64(out), ref, "ns=%d fuse=%s portable=%s"
+                          % (ns, fuse, portable))
     # bf16 output: within one bf16 rounding of the fp32 result
     o32 = cache.attention(q)
     o16 = cache.attention(q, out_dtype=torch.bfloat16)
@@ -154,7 +157,10 @@ def test_full_size_large_sampled_heads():
 
 def test_end_to_end_against_oracle_archive():
     """Oracle's own archive (fp64 encode) through the oracle's attention vs
-    the GPU pipeline: covers codec + attention together."""
+    the GPU pipeline: covers codec + attention together. The two archives may
+    differ by the permitted +-1 code flips near half-integers, each worth one
+    quantisation step of one coefficient, so this cross-archive check holds
+    the relative-L2 bar and a max-abs bound of 1e-2."""
     w = synth.WORKLOADS["gqa"].replace(B=2, T=8 * 120 + 5, seed=8)
     cache, data = _cache_for(w)
     q = data["q"].to(DEV)
@@ -165,4 +171,7 @@ def test_end_to_end_against_oracle_archive():
     ref = oracle.decode_attention_reference(f64(data["q"]), ek["C_hat"],
                                             ev["C_hat"], ek["tail"],
                                             ev["tail"], w.R)
-    check_out(f64(out), ref, "end to end")
+    got = f64(out)
+    err = np.max(np.abs(got - ref))
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    assert rel <= 1e-3 and err <= 1e-2, (err, rel)

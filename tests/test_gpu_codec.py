@@ -125,7 +125,7 @@ def test_prefill_after_partial_tail_matches_oracle_stream():
     X = torch.from_numpy(np.cumsum(rng.standard_normal((B, H, 300, D)),
                                    axis=2)).to(torch.bfloat16)
     cache = CodecKVCache(B, H, D, R, S, device=DEV)
-    ora = oracle.CodecStreamOracle(R, S, "i8", "bf16", decision="f32")
+    ora = oracle.CodecStreamOracle(R, S, "i8", "bf16")
     t = 0
     while t < 300:
         m = int(rng.integers(1, 50))
