@@ -7,19 +7,25 @@
 namespace fc {
 namespace {
 
-// Split count. The tensor-core kernel runs 128-row tiles at two CTAs per SM:
-// split each kv head into enough tile-aligned chunks to give every SM two
-// CTAs. The portable kernel aims at four CTAs per SM with chunks of at least
-// 16 blocks. Results do not depend on the split beyond rounding.
+// Split count. The tensor-core kernel runs one CTA per SM (a six-stage ring
+// of 128-row tiles fills its shared memory): split each kv head into
+// tile-aligned chunks so that all chunks of all kv heads fit in one wave. The
+// portable kernel aims at four CTAs per SM with chunks of at least 16 blocks.
+// Results do not depend on the split beyond rounding.
 int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   if (nb <= 0) return 1;
   const int64_t units = B * Hk;
   const bool tiles = D == 128 && S >= 1 && 32 % S == 0;
-  const int64_t per_sm = tiles ? 2 : 4;
-  const int64_t target = int64_t(sm_count()) * per_sm;
-  int64_t ns = (target + units - 1) / units;
-  const int64_t by_len = tiles ? tc_tiles_per_head(nb, S) : (nb / 16 > 0 ? nb / 16 : 1);
-  if (ns > by_len) ns = by_len;
+  int64_t ns;
+  if (tiles) {
+    ns = int64_t(sm_count()) / units;
+    const int64_t t = tc_tiles_per_head(nb, S);
+    if (ns > t) ns = t;
+  } else {
+    ns = (int64_t(sm_count()) * 4 + units - 1) / units;
+    const int64_t by_len = nb / 16 > 0 ? nb / 16 : 1;
+    if (ns > by_len) ns = by_len;
+  }
   if (ns > kMaxSplits) ns = kMaxSplits;
   if (ns < 1) ns = 1;
   return int(ns);

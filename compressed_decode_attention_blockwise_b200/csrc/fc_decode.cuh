@@ -86,43 +86,78 @@ __device__ __forceinline__ void combine_heads(const float* pm, const float* pl, 
                                               int64_t out_stride_h, int out_dtype) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
+  constexpr int kReg = 4;  // partial rows per lane kept in registers (ns <= 128)
   for (int i = warp; i < NH; i += nwarps) {
     const float* m = pm + int64_t(i) * ns;
     const float* l = pl + int64_t(i) * ns;
     float* w = wts + i * (ns + 1);
-    float mx = -INFINITY;
-    for (int c = lane; c < ns; c += 32)
-      if (__ldcg(l + c) > 0.f) mx = fmaxf(mx, __ldcg(m + c));
-    mx = warp_max(mx);
-    float L = 0.f;
-    for (int c = lane; c < ns; c += 32) {
-      const float lc = __ldcg(l + c);
-      const float e = lc > 0.f ? exp2f(__ldcg(m + c) - mx) : 0.f;
-      w[c] = e;
-      L = fmaf(lc, e, L);
+    float mx = -INFINITY, L = 0.f;
+    if (ns <= 32 * kReg) {
+      float mv[kReg], lv[kReg];
+#pragma unroll
+      for (int r = 0; r < kReg; ++r) {
+        const int c = lane + 32 * r;
+        mv[r] = c < ns ? __ldcg(m + c) : -INFINITY;
+        lv[r] = c < ns ? __ldcg(l + c) : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < kReg; ++r)
+        if (lv[r] > 0.f) mx = fmaxf(mx, mv[r]);
+      mx = warp_max(mx);
+#pragma unroll
+      for (int r = 0; r < kReg; ++r) {
+        const int c = lane + 32 * r;
+        const float e = lv[r] > 0.f ? exp2f(mv[r] - mx) : 0.f;
+        if (c < ns) w[c] = e;
+        L = fmaf(lv[r], e, L);
+      }
+    } else {
+      for (int c = lane; c < ns; c += 32)
+        if (__ldcg(l + c) > 0.f) mx = fmaxf(mx, __ldcg(m + c));
+      mx = warp_max(mx);
+      for (int c = lane; c < ns; c += 32) {
+        const float lc = __ldcg(l + c);
+        const float e = lc > 0.f ? exp2f(__ldcg(m + c) - mx) : 0.f;
+        w[c] = e;
+        L = fmaf(lc, e, L);
+      }
     }
     L = warp_sum(L);
     if (lane == 0) w[ns] = 1.f / L;
   }
   __syncthreads();
-  for (int idx = tid; idx < NH * D; idx += blockDim.x) {
-    const int i = idx / D, d = idx - (idx / D) * D;
-    const float* w = wts + i * (ns + 1);
-    const float* src = pacc + int64_t(i) * ns * D + d;
-    float acc0 = 0.f, acc1 = 0.f;
-    int c = 0;
-    for (; c + 8 <= ns; c += 8) {
-      float v[8];
+  // every thread merges up to two (head, channel) outputs, 16 partials of each
+  // in flight at a time
+  const int n_out = NH * D;
+  for (int o0 = tid; o0 < n_out; o0 += 2 * blockDim.x) {
+    const int o1 = o0 + blockDim.x;
+    const bool has1 = o1 < n_out;
+    const int i0 = o0 / D, d0 = o0 - i0 * D;
+    const int i1 = has1 ? o1 / D : i0, d1 = has1 ? o1 - i1 * D : d0;
+    const float* w0 = wts + i0 * (ns + 1);
+    const float* w1 = wts + i1 * (ns + 1);
+    const float* s0 = pacc + int64_t(i0) * ns * D + d0;
+    const float* s1 = pacc + int64_t(i1) * ns * D + d1;
+    float a0 = 0.f, a1 = 0.f;
+    for (int c0 = 0; c0 < ns; c0 += 16) {
+      float v0[16], v1[16];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(src + int64_t(c + u) * D);
+      for (int u = 0; u < 16; ++u) {
+        const int c = c0 + u;
+        v0[u] = c < ns ? __ldcg(s0 + int64_t(c) * D) : 0.f;
+        v1[u] = (c < ns && has1) ? __ldcg(s1 + int64_t(c) * D) : 0.f;
+      }
 #pragma unroll
-      for (int u = 0; u < 8; u += 2) {
-        acc0 = fmaf(v[u], w[c + u], acc0);
-        acc1 = fmaf(v[u + 1], w[c + u + 1], acc1);
+      for (int u = 0; u < 16; ++u) {
+        const int c = c0 + u;
+        if (c < ns) {
+          a0 = fmaf(v0[u], w0[c], a0);
+          a1 = fmaf(v1[u], w1[c], a1);
+        }
       }
     }
-    for (; c < ns; ++c) acc0 = fmaf(__ldcg(src + int64_t(c) * D), w[c], acc0);
-    store_out(out, out_off + i * out_stride_h + d, out_dtype, (acc0 + acc1) * w[ns]);
+    store_out(out, out_off + i0 * out_stride_h + d0, out_dtype, a0 * w0[ns]);
+    if (has1) store_out(out, out_off + i1 * out_stride_h + d1, out_dtype, a1 * w1[ns]);
   }
   __syncthreads();
 }

@@ -22,15 +22,17 @@
 //           |w_j| <= p_max(tile) sqrt(R) (the columns of A are unit vectors);
 //           the int32 sums are exact.
 //
-// Warp roles. One producer warp issues the TMA loads (128-row tiles of K and
-// V codes with 128-byte swizzle plus their scales, a three-stage ring) and
-// the MMAs, so the tensor core runs ahead of the CUDA cores: the K-side MMA of
-// tile i+1 and the V-side MMA of tile i overlap the softmax work. Two groups
-// of four compute warps split the G query heads of the kv head between them;
+// Warp roles. A TMA warp keeps a six-stage ring of 128-row tiles (K and V
+// codes with 128-byte swizzle, plus their scales) full, refilling a stage as
+// soon as the V-side MMA of its tile completes. Two MMA warps issue the K-side
+// MMA of each tile as soon as it lands and the V-side MMA as soon as its W is
+// written, so neither waits behind the other and both overlap the softmax. Up
+// to four groups of four compute warps split the G query heads of the kv head;
 // in a group, thread t owns coefficient row t on the K side and channel d = t
-// on the V side, so every TMEM load is one warp quadrant. K and V
-// accumulators are double-buffered in TMEM, W is double-buffered in shared
-// memory, and the V epilogue of tile i runs after the softmax of tile i+1.
+// on the V side, so every TMEM load is one warp quadrant. K sums are
+// double-buffered and V sums triple-buffered in TMEM, W is triple-buffered in
+// shared memory, and the V epilogue of tile i runs after the softmax of tile
+// i+2.
 // The online softmax keeps one running max per head for the CTA (one max per
 // tile and group), each thread accumulates its own share of the softmax sum,
 // and the output accumulator lives in registers (thread d, its group's heads).
@@ -51,7 +53,7 @@ namespace tc {
 
 constexpr int kRows = 128;  // coefficient rows per tile
 constexpr int kD = 128;     // head dim served by this kernel
-constexpr int kStages = 3;
+constexpr int kStages = 6;
 constexpr uint32_t kTileBytes = kRows * kD;
 constexpr uint32_t kStageTx = 2 * kTileBytes + 2 * kRows * 4;
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 2 GHz
@@ -63,13 +65,14 @@ __host__ __device__ constexpr int pad16(int x) { return (x + 15) / 16 * 16; }
 // limb columns, each group padded to CS columns.
 template <int G>
 struct Cols {
-  static constexpr int GW = G >= 2 ? 2 : 1;  // compute warp groups
+  static constexpr int GW = G >= 4 ? 4 : G;  // compute warp groups (1, 2 or 4)
   static constexpr int GH = G / GW;          // heads per group
   static constexpr int CS = pad8(3 * GH);    // columns per group (8 or 16)
   static constexpr int NP = pad16(GW * CS);  // MMA N
   static constexpr int kComputeThreads = 128 * GW;
-  static constexpr int kThreads = kComputeThreads + 32;
-  static constexpr uint32_t kTmemCols = 4 * NP <= 64 ? 64 : 128;
+  static constexpr int kThreads = kComputeThreads + 96;  // + TMA, K-MMA and V-MMA warps
+  // K sums double-buffered, V sums triple-buffered
+  static constexpr uint32_t kTmemCols = 5 * NP <= 64 ? 64 : (5 * NP <= 128 ? 128 : 256);
 };
 
 struct TcArgs {
@@ -83,13 +86,13 @@ struct SmemLayout {
   static constexpr uint32_t k = 0;
   static constexpr uint32_t v = k + kStages * kTileBytes;
   static constexpr uint32_t qb = v + kStages * kTileBytes;   // K-major SW128, NP rows x 128 B
-  static constexpr uint32_t wb = qb + NP * 128;               // 2 x (NP/16 x 128 rows x 16 B)
-  static constexpr uint32_t ks = wb + 2 * NP * 128;
+  static constexpr uint32_t wb = qb + NP * 128;               // 3 x (NP/16 x 128 rows x 16 B)
+  static constexpr uint32_t ks = wb + 3 * NP * 128;
   static constexpr uint32_t vs = ks + kStages * kRows * 4;
-  static constexpr uint32_t red = vs + kStages * kRows * 4;   // 2 groups x 4 warps x 32 floats
-  static constexpr uint32_t bars = red + 2 * 4 * 32 * 4;
-  // full[kStages], kfull[2], kempty[2], wready[2], vfull[2], vempty[2]
-  static constexpr int kBars = kStages + 10;
+  static constexpr uint32_t red = vs + kStages * kRows * 4;   // up to 4 groups x 4 warps x 32 floats
+  static constexpr uint32_t bars = red + 4 * 4 * 32 * 4;
+  // full[kStages], vdone[kStages], kfull[2], kempty[2], wready[3], vempty[3], qready
+  static constexpr int kBars = 2 * kStages + 11;
   static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
   static constexpr uint32_t bytes = misc + 16;
   static constexpr uint32_t alloc = bytes + 1024;             // alignment slack
@@ -170,7 +173,7 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CS]) 
 }
 
 template <int G, int S, int TPT>
-__global__ void __launch_bounds__(Cols<G>::kThreads, 2)
+__global__ void __launch_bounds__(Cols<G>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const TcArgs ta, const Basis basis) {
@@ -192,12 +195,13 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
   // 128-byte swizzle atoms need 1024-byte alignment in the shared window
   uint8_t* sm = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
-  uint64_t* full = bars;
-  uint64_t* kfull = bars + kStages;
+  uint64_t* full = bars;               // tile landed (TMA -> MMA)
+  uint64_t* vdone = bars + kStages;    // V-side MMA of the stage's tile done (-> compute, TMA)
+  uint64_t* kfull = bars + 2 * kStages;
   uint64_t* kempty = kfull + 2;
-  uint64_t* wready = kfull + 4;
-  uint64_t* vfull = kfull + 6;
-  uint64_t* vempty = kfull + 8;
+  uint64_t* wready = kfull + 4;        // 3 W buffers
+  uint64_t* vempty = kfull + 7;        // 3 V accumulators
+  uint64_t* qready = kfull + 10;       // query limbs written (compute -> MMA)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::misc);
   int* abort_flag = reinterpret_cast<int*>(sm + L::misc + 4);
   int* last_flag = reinterpret_cast<int*>(sm + L::misc + 8);
@@ -210,24 +214,34 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
   const int tile0 = c * ta.chunk_tiles;
   const int tile1 = min(tile0 + ta.chunk_tiles, ta.tiles_per_head);
   const int ntiles = max(0, tile1 - tile0);
-  const bool producer = warp == NCT / 32;
+  const bool producer = warp >= NCT / 32;  // TMA warp, K-MMA warp, V-MMA warp
+  const bool tma_warp = warp == NCT / 32;
+  const bool mma_warp = warp == NCT / 32 + 1;   // K side; also owns the TMEM allocation
+  const bool mmav_warp = warp == NCT / 32 + 2;  // V side
 
   if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) ptx::mbar_init(&full[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&vdone[i], 1);
+    }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&kfull[i], 1);
       ptx::mbar_init(&kempty[i], NCT);
+    }
+    for (int i = 0; i < 3; ++i) {
       ptx::mbar_init(&wready[i], NCT);
-      ptx::mbar_init(&vfull[i], 1);
       ptx::mbar_init(&vempty[i], NCT);
     }
+    ptx::mbar_init(qready, NCT);
     *abort_flag = 0;
     *last_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (producer) {
+  if (mma_warp) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
+  }
+  if (tma_warp) {
     if (lane == 0) {
       ptx::prefetch_tmap(&tm_k);
       ptx::prefetch_tmap(&tm_v);
@@ -235,6 +249,13 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
       ptx::prefetch_tmap(&tm_vs);
     }
   }
+
+  // barriers and the TMEM address are visible to every warp from here on; the
+  // TMA warp starts streaming while the compute warps prepare the query limbs
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
   // compute-thread identity: group gw, thread t in the group (row / channel)
   const int gw = producer ? 0 : tid / 128;
@@ -276,72 +297,67 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
     if (gw == GW - 1)
       for (int n = GW * CS; n < NP; ++n) qb[sw128_offset(n, t)] = 0;
     ptx::fence_proxy_async_smem();
+    ptx::mbar_arrive(qready);
   }
-  ptx::tc_fence_before();
-  __syncthreads();
-  ptx::tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (producer) {
-    // ================= producer warp: TMA loads and MMA issue (lane 0)
-    if (lane == 0) {
-      auto load_tile = [&](int i) {
-        const int s = i % kStages;
-        const int row0 = (tile0 + i) * kRows;
-        ptx::mbar_arrive_expect_tx(&full[s], kStageTx);
-        ptx::tma_load_4d(sm + L::k + s * kTileBytes, &tm_k, &full[s], 0, row0, h, b);
-        ptx::tma_load_4d(sm + L::v + s * kTileBytes, &tm_v, &full[s], 0, row0, h, b);
-        ptx::tma_load_3d(sm + L::ks + s * kRows * 4, &tm_ks, &full[s], row0, h, b);
-        ptx::tma_load_3d(sm + L::vs + s * kRows * 4, &tm_vs, &full[s], row0, h, b);
-      };
-      auto issue_k = [&](int i) {
-        const int s = i % kStages, bb = i & 1;
-        waiter.wait(&full[s], uint32_t(i / kStages) & 1u);
-        waiter.wait(&kempty[bb], (uint32_t(i >> 1) & 1u) ^ 1u);
-        if (*reinterpret_cast<volatile int*>(abort_flag)) return;
-        ptx::tc_fence_after();
-        const uint32_t ka = ptx::smem_u32(sm + L::k + s * kTileBytes);
-        const uint32_t qa = ptx::smem_u32(sm + L::qb);
-#pragma unroll
-        for (int k = 0; k < kD / 32; ++k)
-          ptx::mma_i8(tmem + bb * NP, ptx::desc_sw128(ka + 32 * k, 16, 1024),
-                      ptx::desc_sw128(qa + 32 * k, 16, 1024), kIdescK, k > 0 ? 1u : 0u);
-        ptx::mma_commit(&kfull[bb]);
-      };
-      int loaded = 0;
-      for (; loaded < kStages && loaded < ntiles; ++loaded) load_tile(loaded);
-      if (ntiles > 0) issue_k(0);
-      for (int i = 0; i < ntiles; ++i) {
-        if (i + 1 < ntiles) issue_k(i + 1);
-        const int s = i % kStages, bb = i & 1;
-        waiter.wait(&wready[bb], uint32_t(i >> 1) & 1u);
-        waiter.wait(&vempty[bb], (uint32_t(i >> 1) & 1u) ^ 1u);
-        if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-        ptx::tc_fence_after();
-        const uint32_t va = ptx::smem_u32(sm + L::v + s * kTileBytes);
-        const uint32_t wa = ptx::smem_u32(sm + L::wb + bb * kWBytes);
-#pragma unroll
-        for (int k = 0; k < kRows / 32; ++k)
-          ptx::mma_i8(tmem + 2 * NP + bb * NP, ptx::desc_sw128(va + 4096 * k, kTileBytes, 1024),
-                      ptx::desc_noswizzle(wa + 512 * k, 128, 2048), kIdescV, k > 0 ? 1u : 0u);
-        ptx::mma_commit(&vfull[bb]);
-        // refill the stage of the previous tile once its V-side MMA (and with
-        // it every earlier MMA of this thread) has completed
-        if (i >= 1 && loaded < ntiles) {
-          waiter.wait(&vfull[(i - 1) & 1], uint32_t((i - 1) >> 1) & 1u);
-          if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-          load_tile(loaded);
-          ++loaded;
+  if (tma_warp && lane == 0) {
+    // ================= TMA warp: keep the ring full. Stage s is refilled as
+    // soon as the V-side MMA of the tile it held has completed.
+    int loaded = 0;
+    for (; loaded < ntiles; ++loaded) {
+      const int s = loaded % kStages;
+      if (loaded >= kStages) waiter.wait(&vdone[s], uint32_t(loaded / kStages - 1) & 1u);
+      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
+      const int row0 = (tile0 + loaded) * kRows;
+      ptx::mbar_arrive_expect_tx(&full[s], kStageTx);
+      ptx::tma_load_4d(sm + L::k + s * kTileBytes, &tm_k, &full[s], 0, row0, h, b);
+      ptx::tma_load_4d(sm + L::v + s * kTileBytes, &tm_v, &full[s], 0, row0, h, b);
+      ptx::tma_load_3d(sm + L::ks + s * kRows * 4, &tm_ks, &full[s], row0, h, b);
+      ptx::tma_load_3d(sm + L::vs + s * kRows * 4, &tm_vs, &full[s], row0, h, b);
+    }
+    // after an abort, every issued load must land before the CTA exits (bounded)
+    if (*reinterpret_cast<volatile int*>(abort_flag)) {
+      const unsigned long long t0 = clock64();
+      for (int i = 0; i < loaded; ++i)
+        while (!ptx::mbar_try_wait(&full[i % kStages], uint32_t(i / kStages) & 1u) &&
+               clock64() - t0 < kWaitCycles) {
         }
-      }
-      // drain: every issued load must land before the CTA exits (bounded)
-      if (*reinterpret_cast<volatile int*>(abort_flag)) {
-        const unsigned long long t0 = clock64();
-        for (int i = 0; i < loaded; ++i)
-          while (!ptx::mbar_try_wait(&full[i % kStages], uint32_t(i / kStages) & 1u) &&
-                 clock64() - t0 < kWaitCycles) {
-          }
-      }
+    }
+  }
+  if (mma_warp && lane == 0) {
+    // ================= K-MMA warp: S_int of each tile as soon as it lands
+    waiter.wait(qready, 0u);
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % kStages, bb = i & 1;
+      waiter.wait(&full[s], uint32_t(i / kStages) & 1u);
+      waiter.wait(&kempty[bb], (uint32_t(i >> 1) & 1u) ^ 1u);
+      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
+      ptx::tc_fence_after();
+      const uint32_t ka = ptx::smem_u32(sm + L::k + s * kTileBytes);
+      const uint32_t qa = ptx::smem_u32(sm + L::qb);
+#pragma unroll
+      for (int k = 0; k < kD / 32; ++k)
+        ptx::mma_i8(tmem + bb * NP, ptx::desc_sw128(ka + 32 * k, 16, 1024),
+                    ptx::desc_sw128(qa + 32 * k, 16, 1024), kIdescK, k > 0 ? 1u : 0u);
+      ptx::mma_commit(&kfull[bb]);
+    }
+  }
+  if (mmav_warp && lane == 0) {
+    // ================= V-MMA warp: Acc_int of each tile as soon as its W is ready
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = i % kStages, vb = i % 3;
+      waiter.wait(&wready[vb], uint32_t(i / 3) & 1u);
+      waiter.wait(&vempty[vb], (uint32_t(i / 3) & 1u) ^ 1u);
+      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
+      ptx::tc_fence_after();
+      const uint32_t va = ptx::smem_u32(sm + L::v + s * kTileBytes);
+      const uint32_t wa = ptx::smem_u32(sm + L::wb + vb * kWBytes);
+#pragma unroll
+      for (int k = 0; k < kRows / 32; ++k)
+        ptx::mma_i8(tmem + 2 * NP + vb * NP, ptx::desc_sw128(va + 4096 * k, kTileBytes, 1024),
+                    ptx::desc_noswizzle(wa + 512 * k, 128, 2048), kIdescV, k > 0 ? 1u : 0u);
+      // completes when this and every earlier V-side MMA has finished; the
+      // K-side MMA of the same tile finished before its W could be written
+      ptx::mma_commit(&vdone[s]);
     }
   }
 
@@ -366,26 +382,28 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
     const float sqrtR = sqrtf(float(R));
     const uint32_t lane_off = uint32_t(wq * 32) << 16;
     const uint32_t col0 = uint32_t(gw * CS);
-    float alpha_prev[GH], wunit_prev[GH];
+    // softmax rescale and W unit of the two tiles whose V epilogue is pending
+    float alpha_p1[GH], wunit_p1[GH], alpha_p2[GH], wunit_p2[GH];
 #pragma unroll
     for (int i = 0; i < GH; ++i) {
-      alpha_prev[i] = 1.f;
-      wunit_prev[i] = 0.f;
+      alpha_p1[i] = alpha_p2[i] = 1.f;
+      wunit_p1[i] = wunit_p2[i] = 0.f;
     }
 
-    // V epilogue of tile i: acc = alpha(i) acc + W-limb sums
-    auto v_epilogue = [&](int i) {
-      const int bb = i & 1;
-      waiter.wait(&vfull[bb], uint32_t(i >> 1) & 1u);
+    // V epilogue of tile i: acc = alpha(i) acc + W-limb sums (run two tiles
+    // late, so the V-side MMA round trip overlaps two softmax passes)
+    auto v_epilogue = [&](int i, const float (&al)[GH], const float (&wu)[GH]) {
+      const int vb = i % 3;
+      waiter.wait(&vdone[i % kStages], uint32_t(i / kStages) & 1u);
       ptx::tc_fence_after();
       uint32_t vr[CS];
-      tmem_ld_cols<CS>(tmem + 2 * NP + bb * NP + col0 + lane_off, vr);
+      tmem_ld_cols<CS>(tmem + 2 * NP + vb * NP + col0 + lane_off, vr);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&vempty[bb]);
+      ptx::mbar_arrive(&vempty[vb]);
 #pragma unroll
       for (int g = 0; g < GH; ++g)
-        acc[g] = fmaf(acc[g], alpha_prev[g], wunit_prev[g] * unlimb3(vr[3 * g], vr[3 * g + 1], vr[3 * g + 2]));
+        acc[g] = fmaf(acc[g], al[g], wu[g] * unlimb3(vr[3 * g], vr[3 * g + 1], vr[3 * g + 2]));
     };
 
     for (int it = 0; it < ntiles; ++it) {
@@ -529,28 +547,33 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
             packed[byte / 4] |= (uint32_t(l[k]) & 0xffu) << (8 * (byte % 4));
           }
         }
-        uint8_t* wrow = sm + L::wb + bb * kWBytes;
+        uint8_t* wrow = sm + L::wb + (it % 3) * kWBytes;
+        // column c of row t lives at (c / 16) * 2048 + t * 16 + c % 16
         if constexpr (CS == 8) {
-          *reinterpret_cast<uint2*>(wrow + t * 16 + gw * 8) = make_uint2(packed[0], packed[1]);
+          *reinterpret_cast<uint2*>(wrow + (gw / 2) * 2048 + t * 16 + (gw % 2) * 8) =
+              make_uint2(packed[0], packed[1]);
         } else {
           *reinterpret_cast<uint4*>(wrow + gw * 2048 + t * 16) =
               make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
       }
       ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(&wready[bb]);
+      ptx::mbar_arrive(&wready[it % 3]);
 #pragma unroll
       for (int g = 0; g < GH; ++g) m_run[g] = m_new[g];
 
-      // ---- V epilogue of the previous tile (its MMA overlapped this softmax)
-      if (it >= 1) v_epilogue(it - 1);
+      // ---- V epilogue of the tile two back (its MMA overlapped two softmaxes)
+      if (it >= 2) v_epilogue(it - 2, alpha_p2, wunit_p2);
 #pragma unroll
       for (int g = 0; g < GH; ++g) {
-        alpha_prev[g] = alpha[g];
-        wunit_prev[g] = wunit[g];
+        alpha_p2[g] = alpha_p1[g];
+        wunit_p2[g] = wunit_p1[g];
+        alpha_p1[g] = alpha[g];
+        wunit_p1[g] = wunit[g];
       }
     }
-    if (ntiles >= 1) v_epilogue(ntiles - 1);
+    if (ntiles >= 2) v_epilogue(ntiles - 2, alpha_p2, wunit_p2);
+    if (ntiles >= 1) v_epilogue(ntiles - 1, alpha_p1, wunit_p1);
 
     // ---- raw tail tokens (last chunk): thread t = channel d
     if (c == a.ns - 1) {
@@ -595,7 +618,7 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 2)
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (producer) {
+  if (mma_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -48,12 +48,15 @@ def check_scales(gpu_scales: np.ndarray, ref_scales: np.ndarray):
 def check_coeffs(gpu: np.ndarray, C: np.ndarray, coeff: str):
     """Unquantised coefficients (..., nb, S, D) against the exact ones:
     bf16 within one bf16 ulp, f32 within 1e-6 of the block's largest
-    coefficient."""
+    coefficient. A coefficient whose exact value vanishes (its block's
+    tokens cancel) is rounding noise of the fp64 sum on both sides, so bf16
+    differences below 1e-12 of the block's largest coefficient also pass."""
     if coeff == "bf16":
         ref = oracle.round_to_dtype(C, "bf16")
         mag = np.maximum(np.abs(ref), np.abs(gpu)) + 1e-300
         ulp = np.ldexp(1.0, np.frexp(mag)[1] - 8)
-        bad = np.abs(gpu - ref) > ulp
+        floor = 1e-12 * np.max(np.abs(C), axis=(-2, -1), keepdims=True)
+        bad = np.abs(gpu - ref) > np.maximum(ulp, floor)
         if bad.any():
             k = tuple(np.argwhere(bad)[0])
             raise AssertionError(
