@@ -22,6 +22,8 @@ FC_ERR_UNSUPPORTED = 2
 FC_ERR_CAPACITY = 3
 FC_ERR_CUDA = 4
 FC_ERR_DEVICE = 5
+FC_ERR_SCRATCH_LIMIT = 6
+FC_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 FC_DECODE_FUSE_COMBINE = 1
 FC_DECODE_PORTABLE = 2
@@ -37,8 +39,8 @@ _DTYPE_CODE = {torch.float32: FC_DTYPE_F32, torch.bfloat16: FC_DTYPE_BF16,
 EXPORTS = (
     "fc_compress_blocks", "fc_append_step", "fc_archive_copy_prefix",
     "fc_decode_plan", "fc_decode_workspace_bytes", "fc_decode_attention",
-    "fc_combine", "fc_workspace_status", "fc_storage_bytes",
-    "fc_status_string",
+    "fc_combine", "fc_decode_attention_noalloc", "fc_workspace_status",
+    "fc_storage_bytes", "fc_status_string",
 )
 
 
@@ -102,6 +104,10 @@ def load() -> ctypes.CDLL:
                                                PI64, P]),
         "fc_combine": (ctypes.c_int, [P, ctypes.c_size_t, I64, I64, I64, I32,
                                       P, I32, PI64, P]),
+        "fc_decode_attention_noalloc": (ctypes.c_int, [P, I32, PI64, I64, PA,
+                                                       PA, PT, PT,
+                                                       ctypes.c_float, I32, P,
+                                                       I32, PI64, P]),
         "fc_workspace_status": (ctypes.c_int, [P, ctypes.c_size_t,
                                                ctypes.POINTER(ctypes.c_uint32),
                                                P]),
@@ -220,6 +226,20 @@ def fc_decode_attention(q: torch.Tensor, ka: FcArchive, va: FcArchive,
         ws_ptr, ws_bytes, _ptr(out), dtype_code(out.dtype), _strides4(out),
         _stream(stream, q))
     _check(st, "fc_decode_attention")
+
+
+def fc_decode_attention_noalloc(q: torch.Tensor, ka: FcArchive, va: FcArchive,
+                                kt: Optional[FcTail], vt: Optional[FcTail],
+                                out: torch.Tensor, softmax_scale: float = 0.0,
+                                num_splits: int = 0, stream=None) -> None:
+    """Decode attention with the library's static scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    st = load().fc_decode_attention_noalloc(
+        _ptr(q), dtype_code(q.dtype), _strides4(q), q.shape[1],
+        ctypes.byref(ka), ctypes.byref(va), _ref(kt), _ref(vt),
+        float(softmax_scale), int(num_splits), _ptr(out),
+        dtype_code(out.dtype), _strides4(out), _stream(stream, q))
+    _check(st, "fc_decode_attention_noalloc")
 
 
 def fc_combine(workspace: torch.Tensor, B: int, Hq: int, D: int,

@@ -1,6 +1,7 @@
 // Entry points of coefficient-domain decode attention: planning, argument
 // validation, kernel selection, and the stand-alone combine.
 #include <cmath>
+#include <mutex>
 
 #include "fc_decode.cuh"
 
@@ -199,4 +200,57 @@ extern "C" int fc_combine(const void* workspace, size_t workspace_bytes, int64_t
   const size_t smem = size_t(num_splits + 1) * sizeof(float);
   combine_kernel<<<dim3(unsigned(Hq), unsigned(B)), 128, smem, stream>>>(a);
   return cuda_status(cudaGetLastError());
+}
+
+// ----------------------------------------------------------------------------
+// Allocation-free decode attention: the scratch is a file-scope device array
+// (FC_NOALLOC_SCRATCH_BYTES, held by every GPU that loads the library until the
+// process exits). Host code cannot use the array's name as a device address,
+// so its address is resolved with cudaGetSymbolAddress once per device, with
+// that device current, on the first call made on the device.
+namespace fc {
+namespace {
+
+__device__ __align__(256) uint8_t g_noalloc_scratch[FC_NOALLOC_SCRATCH_BYTES];
+
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return FC_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FC_OK;
+}
+
+}  // namespace
+}  // namespace fc
+
+extern "C" int fc_decode_attention_noalloc(const void* q, int32_t q_dtype, const int64_t* q_strides,
+                                           int64_t Hq, const fc_archive* ka, const fc_archive* va,
+                                           const fc_tail* kt, const fc_tail* vt, float softmax_scale,
+                                           int32_t num_splits, void* out, int32_t out_dtype,
+                                           const int64_t* out_strides, fc_stream stream) {
+  int st = check_archive(ka);
+  if (st != FC_OK) return st;
+  if (Hq < 1 || Hq % ka->H) return FC_ERR_INVALID;
+  int ns = num_splits;
+  if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H, ka->S, int(ka->D));
+  if (ns < 1 || ns > kMaxSplits) return FC_ERR_INVALID;
+  const WorkspaceLayout wl = workspace_layout(ka->B, Hq, ka->D, ns);
+  if (wl.total > FC_NOALLOC_SCRATCH_BYTES) return FC_ERR_SCRATCH_LIMIT;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != FC_OK) return st;
+  // the status word and the tickets must start at zero; the array keeps
+  // whatever the previous call left
+  if (cudaMemsetAsync(scratch, 0, wl.m, stream) != cudaSuccess) return FC_ERR_CUDA;
+  return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, ns,
+                             FC_DECODE_FUSE_COMBINE, scratch, FC_NOALLOC_SCRATCH_BYTES, out, out_dtype,
+                             out_strides, stream);
 }

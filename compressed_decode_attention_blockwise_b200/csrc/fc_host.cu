@@ -106,6 +106,8 @@ const char* fc_status_string(int status) {
     case FC_ERR_CAPACITY: return "archive capacity exhausted; nothing was written";
     case FC_ERR_CUDA: return "CUDA runtime error or kernel launch failure";
     case FC_ERR_DEVICE: return "a kernel reported an error in the workspace status word";
+    case FC_ERR_SCRATCH_LIMIT:
+      return "request needs more scratch than the library's static array (FC_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }

@@ -54,7 +54,8 @@ enum {
   FC_ERR_UNSUPPORTED = 2,  /* valid but outside the supported sizes/dtypes above */
   FC_ERR_CAPACITY = 3,     /* the archive has too few free blocks; nothing written */
   FC_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
-  FC_ERR_DEVICE = 5        /* a kernel reported an error in the workspace status word */
+  FC_ERR_DEVICE = 5,       /* a kernel reported an error in the workspace status word */
+  FC_ERR_SCRATCH_LIMIT = 6 /* fc_decode_attention_noalloc: request exceeds its static scratch */
 };
 
 /* fc_decode_attention flags. */
@@ -238,6 +239,32 @@ int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides
 int fc_combine(const void* workspace, size_t workspace_bytes, int64_t B,
                int64_t Hq, int64_t D, int32_t num_splits, void* out,
                int32_t out_dtype, const int64_t* out_strides, fc_stream stream);
+
+/*
+ * fc_decode_attention_noalloc -- fc_decode_attention (fused combine) for
+ * callers that cannot hand the library a workspace: a C host that runs inside
+ * a fixed device-memory budget with no allocator of its own, or a serving
+ * loop that must not call cudaMalloc per step because the call synchronises
+ * the device. The paper has no counterpart; this is an interface convenience.
+ *
+ * Instead of a caller workspace the call uses one file-scope device array of
+ * FC_NOALLOC_SCRATCH_BYTES that every GPU loading the library holds until the
+ * process exits. It calls no cudaMalloc, cudaFree or allocating routine. The
+ * first call on a device resolves the array's device address with
+ * cudaGetSymbolAddress (once per device, with that device current); make that
+ * first call before any stream capture. Every call shares the array and
+ * clears its status word and tickets on `stream` before the kernel, so calls
+ * whose executions overlap on the GPU (other streams, other host threads)
+ * race; serialise them. Arguments and results as in fc_decode_attention;
+ * returns FC_ERR_SCRATCH_LIMIT, launching nothing, when
+ * fc_decode_workspace_bytes(B, Hq, D, splits) exceeds the array.
+ */
+#define FC_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+int fc_decode_attention_noalloc(const void* q, int32_t q_dtype, const int64_t* q_strides,
+                                int64_t Hq, const fc_archive* ka, const fc_archive* va,
+                                const fc_tail* kt, const fc_tail* vt, float softmax_scale,
+                                int32_t num_splits, void* out, int32_t out_dtype,
+                                const int64_t* out_strides, fc_stream stream);
 
 /*
  * fc_workspace_status -- synchronise `stream`, read the workspace status word

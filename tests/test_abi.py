@@ -30,14 +30,14 @@ def declared_functions():
 def test_library_exports_every_declared_symbol():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 10, names
+    assert len(names) == 11, names
     assert sorted(names) == sorted(_lib.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
 
 
 def test_status_strings():
-    for code in range(6):
+    for code in range(7):
         assert _lib.fc_status_string(code)
     assert "unknown" in _lib.fc_status_string(99)
 
