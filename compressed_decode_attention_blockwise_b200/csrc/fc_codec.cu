@@ -243,6 +243,10 @@ struct AppendArgs {
 
 template <int VEC, typename TIn, typename TOutK, typename TOutV>
 __global__ void __launch_bounds__(256) append_step_kernel(AppendArgs a, BasisF64 basis) {
+  // a decode attention launched with FC_DECODE_OVERLAP may start streaming
+  // the older archive blocks now: this kernel writes only the tails and the
+  // block it completes, which that attention reads after its dependency wait
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t bh_total = int64_t(a.B) * a.H;

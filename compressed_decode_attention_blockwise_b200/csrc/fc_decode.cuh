@@ -58,7 +58,8 @@ struct DecodeArgs {
   float* pm;
   float* pl;
   float* pacc;
-  int fuse;  // 1: last CTA per kv head writes out
+  int fuse;     // 1: last CTA per kv head writes out
+  int overlap;  // 1: launched as a programmatic dependent (FC_DECODE_OVERLAP)
   void* out;
   int out_dtype;
   int64_t os_b, os_h;
@@ -76,16 +77,28 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, int dtype, flo
 // e^(m_c - M) / L, chunks with l_c = 0 skipped (base-2 exponentials: the
 // partial maxima are kept in log2 units). Head i's partials are rows
 // pm[i * ns + c], pl[i * ns + c], pacc[(i * ns + c) * D + d]; its output goes to
-// out[out_off + i * out_stride_h + d]. All threads of the CTA take part: warps
-// compute the per-head weights into shared scratch `wts` (NH * (ns + 1)
-// floats), then every thread merges (head, channel) pairs with independent,
-// batched L2 loads. Partials written by other CTAs of the same launch are read
-// through L2 (ld.cg).
+// out[out_off + i * out_stride_h + d]. All threads of the CTA take part. Each
+// thread first issues the loads of the partial accumulators of its first
+// (head, channel) output (up to kPre of them) and only then do warps compute
+// the per-head weights into shared scratch `wts` (NH * (ns + 1) floats), so
+// both sets of L2 reads are in flight together; further outputs (more outputs
+// than threads) and partials beyond kPre use batched loads. Partials written
+// by other CTAs of the same launch are read through L2 (ld.cg).
 __device__ __forceinline__ void combine_heads(const float* pm, const float* pl, const float* pacc, int NH,
                                               int ns, int D, float* wts, void* out, int64_t out_off,
                                               int64_t out_stride_h, int out_dtype) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
+  const int n_out = NH * D;
+  constexpr int kPre = 24;
+  // partials of my first output, requested before the weights are known
+  const bool has_first = tid < n_out;
+  const int fi = has_first ? tid / D : 0, fd = has_first ? tid - fi * D : 0;
+  const float* fsrc = pacc + int64_t(fi) * ns * D + fd;
+  float pre[kPre];
+#pragma unroll
+  for (int u = 0; u < kPre; ++u) pre[u] = (has_first && u < ns) ? __ldcg(fsrc + int64_t(u) * D) : 0.f;
+
   constexpr int kReg = 4;  // partial rows per lane kept in registers (ns <= 128)
   for (int i = warp; i < NH; i += nwarps) {
     const float* m = pm + int64_t(i) * ns;
@@ -126,40 +139,49 @@ __device__ __forceinline__ void combine_heads(const float* pm, const float* pl, 
     if (lane == 0) w[ns] = 1.f / L;
   }
   __syncthreads();
-  // every thread merges up to two (head, channel) outputs, 16 partials of each
-  // in flight at a time
-  const int n_out = NH * D;
-  for (int o0 = tid; o0 < n_out; o0 += 2 * blockDim.x) {
-    const int o1 = o0 + blockDim.x;
-    const bool has1 = o1 < n_out;
-    const int i0 = o0 / D, d0 = o0 - i0 * D;
-    const int i1 = has1 ? o1 / D : i0, d1 = has1 ? o1 - i1 * D : d0;
-    const float* w0 = wts + i0 * (ns + 1);
-    const float* w1 = wts + i1 * (ns + 1);
-    const float* s0 = pacc + int64_t(i0) * ns * D + d0;
-    const float* s1 = pacc + int64_t(i1) * ns * D + d1;
-    float a0 = 0.f, a1 = 0.f;
+  if (has_first) {
+    const float* w = wts + fi * (ns + 1);
+    float acc = 0.f;
+#pragma unroll
+    for (int u = 0; u < kPre; ++u)
+      if (u < ns) acc = fmaf(pre[u], w[u], acc);
+    for (int c = kPre; c < ns; ++c) acc = fmaf(__ldcg(fsrc + int64_t(c) * D), w[c], acc);
+    store_out(out, out_off + fi * out_stride_h + fd, out_dtype, acc * w[ns]);
+  }
+  // the remaining outputs, 16 partials in flight at a time
+  for (int o = tid + blockDim.x; o < n_out; o += blockDim.x) {
+    const int i = o / D, d = o - i * D;
+    const float* w = wts + i * (ns + 1);
+    const float* src = pacc + int64_t(i) * ns * D + d;
+    float acc = 0.f;
     for (int c0 = 0; c0 < ns; c0 += 16) {
-      float v0[16], v1[16];
+      float v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int c = c0 + u;
-        v0[u] = c < ns ? __ldcg(s0 + int64_t(c) * D) : 0.f;
-        v1[u] = (c < ns && has1) ? __ldcg(s1 + int64_t(c) * D) : 0.f;
-      }
+      for (int u = 0; u < 16; ++u) v[u] = c0 + u < ns ? __ldcg(src + int64_t(c0 + u) * D) : 0.f;
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const int c = c0 + u;
-        if (c < ns) {
-          a0 = fmaf(v0[u], w0[c], a0);
-          a1 = fmaf(v1[u], w1[c], a1);
-        }
-      }
+      for (int u = 0; u < 16; ++u)
+        if (c0 + u < ns) acc = fmaf(v[u], w[c0 + u], acc);
     }
-    store_out(out, out_off + i0 * out_stride_h + d0, out_dtype, a0 * w0[ns]);
-    if (has1) store_out(out, out_off + i1 * out_stride_h + d1, out_dtype, a1 * w1[ns]);
+    store_out(out, out_off + i * out_stride_h + d, out_dtype, acc * w[ns]);
   }
   __syncthreads();
+}
+
+// The hand-off to the last CTA of a (b, kv head): every thread's partial
+// writes are ordered before thread 0's fence and ticket increment by the CTA
+// barrier; the CTA that draws the last ticket fences again before its threads
+// read the other CTAs' partials. Returns true in that CTA (all threads).
+__device__ __forceinline__ bool last_cta_ticket(uint32_t* ticket, int ns, int* s_flag) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const unsigned t = atomicAdd(ticket, 1u);
+    const int last = (t == unsigned(ns - 1)) ? 1 : 0;
+    if (last) __threadfence();
+    *s_flag = last;
+  }
+  __syncthreads();
+  return *s_flag != 0;
 }
 
 // Writes the CTA's merged state for query head g of its kv head (or the final
@@ -206,15 +228,7 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs& a, int b, int h, in
   // last CTA of this (b, kv head) to arrive merges all chunks: an atomic
   // ticket, no waiting
   __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned t = atomicAdd(a.tickets + (b * a.Hk + h), 1u);
-    s_last = (t == unsigned(a.ns - 1)) ? 1 : 0;
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
+  if (!last_cta_ticket(a.tickets + (b * a.Hk + h), a.ns, &s_last)) return;
   const int64_t row = (int64_t(b) * Hq + h * G) * a.ns;
   combine_heads(a.pm + row, a.pl + row, a.pacc + row * D, G, a.ns, D, scratch, a.out,
                 b * a.os_b + (h * G) * a.os_h, a.os_h, a.out_dtype);

@@ -22,20 +22,27 @@
 //           |w_j| <= p_max(tile) sqrt(R) (the columns of A are unit vectors);
 //           the int32 sums are exact.
 //
-// Warp roles. A TMA warp keeps a six-stage ring of 128-row tiles (K and V
-// codes with 128-byte swizzle, plus their scales) full, refilling a stage as
-// soon as the V-side MMA of its tile completes. Two MMA warps issue the K-side
-// MMA of each tile as soon as it lands and the V-side MMA as soon as its W is
-// written, so neither waits behind the other and both overlap the softmax. Up
-// to four groups of four compute warps split the G query heads of the kv head;
-// in a group, thread t owns coefficient row t on the K side and channel d = t
-// on the V side, so every TMEM load is one warp quadrant. K sums are
-// double-buffered and V sums triple-buffered in TMEM, W is triple-buffered in
-// shared memory, and the V epilogue of tile i runs after the softmax of tile
-// i+2.
-// The online softmax keeps one running max per head for the CTA (one max per
-// tile and group), each thread accumulates its own share of the softmax sum,
-// and the output accumulator lives in registers (thread d, its group's heads).
+// Warp roles. One TMA thread keeps two rings full: K tiles (128 rows x 128
+// codes, 128-byte swizzle), recycled as soon as their K-side MMA completes,
+// and V tiles together with the tile's K and V scales, recycled when the
+// V-side MMA completes. Two MMA warps issue the K-side MMA of each tile as
+// soon as it lands and the V-side MMA as soon as its W is written. NG = 4
+// compute groups of four warps (3 when G or S is 8, for registers) take the
+// tiles in turn (tile i -> group i mod NG), each with its own online-softmax
+// state, so NG tiles are in the softmax at once; the groups' states merge at
+// the end of the chunk.
+//
+// Inside a group, thread t first owns coefficient row t (its TMEM lane) and
+// converts the K sums of all heads; a warp-local transpose through shared
+// memory then gives each lane whole (block, head) items, so a lane computes
+// the R logits of a block from its S scores with the basis as compile-time
+// constant operands, takes the R exponentials, and folds them back into the S
+// weights w_j without any cross-lane reduction. One named barrier per tile
+// exchanges the per-warp maxima. The V epilogue of a tile (thread t = channel
+// d, every head) runs one group iteration later, so the V-side MMA overlaps
+// the group's next softmax. Integer<->float conversions of the limbs use the
+// 1.5 * 2^23 addition (exact for |x| < 2^22), which keeps them on the FMA
+// pipes.
 //
 // Every wait on an mbarrier is bounded; on timeout the kernel records an
 // error in the workspace status word, stops issuing work, drains what it
@@ -53,49 +60,59 @@ namespace tc {
 
 constexpr int kRows = 128;  // coefficient rows per tile
 constexpr int kD = 128;     // head dim served by this kernel
-constexpr int kStages = 6;
 constexpr uint32_t kTileBytes = kRows * kD;
-constexpr uint32_t kStageTx = 2 * kTileBytes + 2 * kRows * 4;
+constexpr uint32_t kScaleBytes = kRows * 4;
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 2 GHz
+constexpr int kFinBar = 8;   // named barrier over every compute warp
+constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
+constexpr int kMagicBits = 0x4B400000;
 
-__host__ __device__ constexpr int pad8(int x) { return (x + 7) / 8 * 8; }
 __host__ __device__ constexpr int pad16(int x) { return (x + 15) / 16 * 16; }
 
-// Column layout of the MMA N dimension: GW groups of GH heads, each head three
-// limb columns, each group padded to CS columns.
-template <int G>
-struct Cols {
-  static constexpr int GW = G >= 4 ? 4 : G;  // compute warp groups (1, 2 or 4)
-  static constexpr int GH = G / GW;          // heads per group
-  static constexpr int CS = pad8(3 * GH);    // columns per group (8 or 16)
-  static constexpr int NP = pad16(GW * CS);  // MMA N
-  static constexpr int kComputeThreads = 128 * GW;
-  static constexpr int kThreads = kComputeThreads + 96;  // + TMA, K-MMA and V-MMA warps
-  // K sums double-buffered, V sums triple-buffered
-  static constexpr uint32_t kTmemCols = 5 * NP <= 64 ? 64 : (5 * NP <= 128 ? 128 : 256);
+template <int G, int S, int TPT>
+struct Cfg {
+  static constexpr int R = S * TPT;
+  static constexpr int TB = kRows / S;             // blocks per tile
+  static constexpr int BW = 32 / S;                // blocks per warp
+  static constexpr int NI = G >= S ? G / S : 1;    // (block, head) items per lane
+  // compute groups of four warps (three where a lane's items need more
+  // registers than four groups leave)
+  static constexpr int NG = (S == 8 || G == 8) ? 3 : 4;
+  static constexpr int HPG = (G + NG - 1) / NG;    // heads per group in the final merge
+  static constexpr int NP = pad16(3 * G);          // MMA N: three limb columns per head
+  static constexpr int NKS = 4;                    // K ring stages
+  static constexpr int NVS = NP == 16 ? 7 : 6;     // V ring stages
+  static constexpr int kThreads = 128 * NG + 96;   // + TMA, K-MMA and V-MMA warps
+  // per group 2 K and 2 V buffers, allocated as a power of two
+  static constexpr uint32_t kTmemCols = 4 * NP * NG <= 256 ? 256 : 512;
+  static constexpr uint32_t LBO = 16 * NP;         // W operand: K-direction core-matrix stride
+  static constexpr int XP = S * (G + 1);           // transpose scratch floats per block
+  static constexpr int XW = BW * XP;               // ... per warp
+  // shared memory (offsets from a 1024-byte aligned base)
+  static constexpr uint32_t kt = 0;
+  static constexpr uint32_t vt = kt + NKS * kTileBytes;
+  static constexpr uint32_t qb = vt + NVS * kTileBytes;       // K-major SW128, NP rows x 128 B
+  static constexpr uint32_t sc = qb + NP * 128;               // per V stage: K scales, V scales
+  static constexpr uint32_t wb = sc + NVS * 2 * kScaleBytes;  // NG x 2 W buffers
+  static constexpr uint32_t xs = wb + NG * 2 * NP * 128;     // transpose scratch, 4 NG warps
+  static constexpr uint32_t red = xs + NG * 4 * XW * 4;      // NG x 2 x (G + 1) x 4 floats
+  static constexpr uint32_t qu = red + NG * 2 * (G + 1) * 16;  // G limb units of q
+  static constexpr uint32_t qs = qu + 64;                     // 4 x G floats: |q| maxima
+  static constexpr uint32_t bars = qs + 128;
+  static constexpr int kBars = 2 * NKS + 2 * NVS + 10 * NG + 1;
+  static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
+  static constexpr uint32_t bytes = misc + 16;
+  static constexpr uint32_t alloc = bytes + 1024;             // alignment slack
+  static_assert(alloc <= 232448, "shared memory");
+  static_assert((NG * G * (kD + 5) + 4) * 4 <= int(NKS * kTileBytes), "merge scratch");
+  static_assert(4 * NP * NG <= 512, "TMEM allocation");
+  static_assert(NI * R <= 32, "logits per lane");
 };
 
 struct TcArgs {
   DecodeArgs d;
   int tiles_per_head;
   int chunk_tiles;
-};
-
-template <int NP>
-struct SmemLayout {
-  static constexpr uint32_t k = 0;
-  static constexpr uint32_t v = k + kStages * kTileBytes;
-  static constexpr uint32_t qb = v + kStages * kTileBytes;   // K-major SW128, NP rows x 128 B
-  static constexpr uint32_t wb = qb + NP * 128;               // 3 x (NP/16 x 128 rows x 16 B)
-  static constexpr uint32_t ks = wb + 3 * NP * 128;
-  static constexpr uint32_t vs = ks + kStages * kRows * 4;
-  static constexpr uint32_t red = vs + kStages * kRows * 4;   // up to 4 groups x 4 warps x 32 floats
-  static constexpr uint32_t bars = red + 4 * 4 * 32 * 4;
-  // full[kStages], vdone[kStages], kfull[2], kempty[2], wready[3], vempty[3], qready
-  static constexpr int kBars = 2 * kStages + 11;
-  static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
-  static constexpr uint32_t bytes = misc + 16;
-  static constexpr uint32_t alloc = bytes + 1024;             // alignment slack
 };
 
 __device__ __forceinline__ float pow2i(int e) {
@@ -109,23 +126,88 @@ __device__ __forceinline__ int exp_above(float x) {
   return ef == 0 ? -126 : ef - 126;
 }
 
-// three 7-bit limbs of x in (-64, 64): x ~ L0 + L1 / 128 + L2 / 16384
-__device__ __forceinline__ void limbs3(float x, int& l0, int& l1, int& l2) {
-  l0 = __float2int_rn(x);
-  const float r1 = (x - float(l0)) * 128.f;
-  l1 = __float2int_rn(r1);
-  const float r2 = (r1 - float(l1)) * 128.f;
-  l2 = __float2int_rn(r2);
+// exact int32 -> float for |v| < 2^22
+__device__ __forceinline__ float i2f_small(uint32_t v) {
+  return __fsub_rn(__int_as_float(int(v) + kMagicBits), kMagic);
+}
+
+// x ~ L0 + L1 / 128 + L2 / 16384 for x in (-64, 64), limbs rounded to nearest
+// even; returns each limb in the low byte of a word
+__device__ __forceinline__ void limb_bytes(float x, uint32_t& b0, uint32_t& b1, uint32_t& b2) {
+  const float t0 = __fadd_rn(x, kMagic);
+  const float y1 = __fmul_rn(__fsub_rn(x, __fsub_rn(t0, kMagic)), 128.f);
+  const float t1 = __fadd_rn(y1, kMagic);
+  const float y2 = __fmul_rn(__fsub_rn(y1, __fsub_rn(t1, kMagic)), 128.f);
+  const float t2 = __fadd_rn(y2, kMagic);
+  b0 = __float_as_uint(t0);
+  b1 = __float_as_uint(t1);
+  b2 = __float_as_uint(t2);
 }
 
 __device__ __forceinline__ float unlimb3(uint32_t c0, uint32_t c1, uint32_t c2) {
-  return fmaf(float(int(c2)), 1.f / 16384.f, fmaf(float(int(c1)), 1.f / 128.f, float(int(c0))));
+  return fmaf(i2f_small(c2), 1.f / 16384.f, fmaf(i2f_small(c1), 1.f / 128.f, i2f_small(c0)));
 }
 
 // byte offset of element (row n, column k) in a 128-byte-swizzled K-major
 // operand whose rows are 128 bytes (1024-byte-aligned atoms of 8 rows)
 __device__ __forceinline__ uint32_t sw128_offset(int n, int k) {
   return uint32_t(n) * 128u + ((uint32_t(k >> 4) ^ uint32_t(n & 7)) << 4) + uint32_t(k & 15);
+}
+
+// byte offset of W[n][k] (column n = head limb, k = tile row) in the K-major
+// operand without swizzle: 8 x 16-byte core matrices, N-adjacent ones 128 B
+// apart, K-adjacent ones LBO apart
+template <uint32_t LBO>
+__device__ __forceinline__ uint32_t w_offset(int n, int k) {
+  return uint32_t(k >> 4) * LBO + uint32_t(n >> 3) * 128u + uint32_t(n & 7) * 16u + uint32_t(k & 15);
+}
+
+// stores the low bytes of S words as S consecutive bytes
+template <int S>
+__device__ __forceinline__ void store_bytes(uint8_t* p, const uint32_t (&v)[S]) {
+  if constexpr (S == 1) {
+    *p = uint8_t(v[0]);
+  } else if constexpr (S == 2) {
+    *reinterpret_cast<uint16_t*>(p) = uint16_t(__byte_perm(v[0], v[1], 0x0040));
+  } else if constexpr (S == 4) {
+    *reinterpret_cast<uint32_t*>(p) =
+        __byte_perm(__byte_perm(v[0], v[1], 0x0040), __byte_perm(v[2], v[3], 0x0040), 0x5410);
+  } else {
+    static_assert(S == 8, "S");
+    const uint32_t lo =
+        __byte_perm(__byte_perm(v[0], v[1], 0x0040), __byte_perm(v[2], v[3], 0x0040), 0x5410);
+    const uint32_t hi =
+        __byte_perm(__byte_perm(v[4], v[5], 0x0040), __byte_perm(v[6], v[7], 0x0040), 0x5410);
+    *reinterpret_cast<uint2*>(p) = make_uint2(lo, hi);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void load_floats(const float* p, float (&v)[N]) {
+  if constexpr (N == 1) {
+    v[0] = p[0];
+  } else if constexpr (N == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x;
+    v[1] = x.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(p + i);
+      v[i] = x.x;
+      v[i + 1] = x.y;
+      v[i + 2] = x.z;
+      v[i + 3] = x.w;
+    }
+  }
+}
+
+template <int N>
+__device__ __forceinline__ float pick(const float (&v)[N], int i) {
+  float r = v[0];
+#pragma unroll
+  for (int k = 1; k < N; ++k) r = (k == i) ? v[k] : r;
+  return r;
 }
 
 struct Waiter {
@@ -147,7 +229,14 @@ struct Waiter {
   }
 };
 
-// Sums G values per thread over the 128 threads of one warp group (named
+// bounded wait that ignores the abort flag (draining after an abort)
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = clock64();
+  while (!ptx::mbar_try_wait(bar, parity) && clock64() - t0 < kWaitCycles) {
+  }
+}
+
+// Sums N values per thread over the 128 threads of one warp group (named
 // barrier `bar_id`; scratch: 4 warps x 32 floats).
 template <int N>
 __device__ __forceinline__ void group_sum(float (&v)[N], float* red, int wq, int lane, int bar_id) {
@@ -163,48 +252,43 @@ __device__ __forceinline__ void group_sum(float (&v)[N], float* red, int wq, int
   ptx::named_bar_sync(bar_id, 128);
 }
 
-template <int CS>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[CS]) {
-  if constexpr (CS == 8) {
-    ptx::tmem_ld8(taddr, r);
-  } else {
+template <int NP>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) {
+  if constexpr (NP == 16) {
     ptx::tmem_ld16(taddr, r);
+  } else {
+    static_assert(NP == 32, "NP");
+    ptx::tmem_ld32(taddr, r);
   }
 }
 
 template <int G, int S, int TPT>
-__global__ void __launch_bounds__(Cols<G>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const TcArgs ta, const Basis basis) {
-  using C = Cols<G>;
-  constexpr int GW = C::GW, GH = C::GH, CS = C::CS, NP = C::NP;
-  constexpr int NCT = C::kComputeThreads;
-  constexpr int R = S * TPT;
-  constexpr int TB = kRows / S;  // blocks per tile
-  using L = SmemLayout<NP>;
-  static_assert(kRows % S == 0 && 32 % S == 0, "blocks must not straddle warps");
-  static_assert(NP == 16 || NP == 32, "N must be 16 or 32");
-  static_assert(GH % 2 == 0 || GH == 1, "heads per group pair up");
+  using C = Cfg<G, S, TPT>;
+  constexpr int R = C::R, NP = C::NP, NI = C::NI, NKS = C::NKS, NVS = C::NVS, XP = C::XP;
+  constexpr int NG = C::NG;
+  constexpr int NCW = 4 * NG;  // compute warps
   constexpr uint32_t kIdescK = ptx::idesc_i8(128, NP, false, false);
-  constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, true);
+  constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
   constexpr uint32_t kWBytes = NP * 128;  // one W buffer
 
   const DecodeArgs& a = ta.d;
   extern __shared__ uint8_t smem_raw[];
   // 128-byte swizzle atoms need 1024-byte alignment in the shared window
   uint8_t* sm = smem_raw + ((1024u - (ptx::smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::bars);
-  uint64_t* full = bars;               // tile landed (TMA -> MMA)
-  uint64_t* vdone = bars + kStages;    // V-side MMA of the stage's tile done (-> compute, TMA)
-  uint64_t* kfull = bars + 2 * kStages;
-  uint64_t* kempty = kfull + 2;
-  uint64_t* wready = kfull + 4;        // 3 W buffers
-  uint64_t* vempty = kfull + 7;        // 3 V accumulators
-  uint64_t* qready = kfull + 10;       // query limbs written (compute -> MMA)
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::misc);
-  int* abort_flag = reinterpret_cast<int*>(sm + L::misc + 4);
-  int* last_flag = reinterpret_cast<int*>(sm + L::misc + 8);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::bars);
+  uint64_t* kfull = bars;         // K tile landed (TMA -> K-MMA)
+  uint64_t* kfree = kfull + NKS;  // K-side MMA done with the stage (-> TMA)
+  uint64_t* vfull = kfree + NKS;  // V tile and both scale rows landed (TMA -> compute, V-MMA)
+  uint64_t* vfree = vfull + NVS;  // V-side MMA done with the stage (-> TMA)
+  uint64_t* gbar = vfree + NVS;   // per group: kres[2] kemp[2] wrdy[2] vres[2] vemp[2]
+  uint64_t* qready = gbar + 10 * NG;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::misc);
+  int* abort_flag = reinterpret_cast<int*>(sm + C::misc + 4);
+  int* last_flag = reinterpret_cast<int*>(sm + C::misc + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -214,426 +298,503 @@ __global__ void __launch_bounds__(Cols<G>::kThreads, 1)
   const int tile0 = c * ta.chunk_tiles;
   const int tile1 = min(tile0 + ta.chunk_tiles, ta.tiles_per_head);
   const int ntiles = max(0, tile1 - tile0);
-  const bool producer = warp >= NCT / 32;  // TMA warp, K-MMA warp, V-MMA warp
-  const bool tma_warp = warp == NCT / 32;
-  const bool mma_warp = warp == NCT / 32 + 1;   // K side; also owns the TMEM allocation
-  const bool mmav_warp = warp == NCT / 32 + 2;  // V side
+  const bool producer = warp >= NCW;
+  const bool tma_warp = warp == NCW;
+  const bool kmma_warp = warp == NCW + 1;  // also owns the TMEM allocation
+  const bool vmma_warp = warp == NCW + 2;
 
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      ptx::mbar_init(&full[i], 1);
-      ptx::mbar_init(&vdone[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
+  const int grp = producer ? 0 : warp >> 2;  // compute group
+  const int w = warp & 3;                    // warp in the group = TMEM lane quadrant
+  const int t = tid & 127;                   // thread in the group
+  // group 0 reads the query (thread t = channel d). Without FC_DECODE_OVERLAP
+  // it does so before anything else, so that these loads do not queue behind
+  // the ring fill; with it, after the setup barrier and the dependency wait
+  // (q comes from the preceding work), while the fill has long been running.
+  float qd[G];
+  auto load_q = [&]() {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      qd[g] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
+  };
+  if (!producer && grp == 0 && !a.overlap) load_q();
+
+  // TMA thread: issues a K load into stage nk % NKS / a V load (codes and both
+  // scale rows) into stage nv % NVS
+  // (under FC_DECODE_OVERLAP the head's last tile, which holds the block the
+  // preceding work may have just written, waits for that work)
+  auto load_k = [&](int nk) {
+    if (a.overlap && tile0 + nk == ta.tiles_per_head - 1) ptx::grid_dep_wait();
+    const int s = nk % NKS;
+    ptx::mbar_arrive_expect_tx(&kfull[s], kTileBytes);
+    ptx::tma_load_4d(sm + C::kt + s * kTileBytes, &tm_k, &kfull[s], 0, (tile0 + nk) * kRows, h, b);
+  };
+  auto load_v = [&](int nv) {
+    if (a.overlap && tile0 + nv == ta.tiles_per_head - 1) ptx::grid_dep_wait();
+    const int s = nv % NVS;
+    const int row0 = (tile0 + nv) * kRows;
+    uint8_t* scs = sm + C::sc + s * 2 * kScaleBytes;
+    ptx::mbar_arrive_expect_tx(&vfull[s], kTileBytes + 2 * kScaleBytes);
+    ptx::tma_load_4d(sm + C::vt + s * kTileBytes, &tm_v, &vfull[s], 0, row0, h, b);
+    ptx::tma_load_3d(scs, &tm_ks, &vfull[s], row0, h, b);
+    ptx::tma_load_3d(scs + kScaleBytes, &tm_vs, &vfull[s], row0, h, b);
+  };
+  int nk = 0, nv = 0;  // loads issued (TMA thread)
+  if (tma_warp && lane == 0) {
+    for (int i = 0; i < NKS; ++i) {
       ptx::mbar_init(&kfull[i], 1);
-      ptx::mbar_init(&kempty[i], NCT);
+      ptx::mbar_init(&kfree[i], 1);
     }
-    for (int i = 0; i < 3; ++i) {
-      ptx::mbar_init(&wready[i], NCT);
-      ptx::mbar_init(&vempty[i], NCT);
+    for (int i = 0; i < NVS; ++i) {
+      ptx::mbar_init(&vfull[i], 1);
+      ptx::mbar_init(&vfree[i], 1);
     }
-    ptx::mbar_init(qready, NCT);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tm_k);
+    ptx::prefetch_tmap(&tm_v);
+    ptx::prefetch_tmap(&tm_ks);
+    ptx::prefetch_tmap(&tm_vs);
+  }
+  if (tid == 0) {
+    for (int g = 0; g < NG; ++g)
+      for (int x = 0; x < 2; ++x) {
+        ptx::mbar_init(&gbar[10 * g + 0 + x], 1);    // kres: K-side MMA committed
+        ptx::mbar_init(&gbar[10 * g + 2 + x], 128);  // kemp: the group read the K sums
+        ptx::mbar_init(&gbar[10 * g + 4 + x], 128);  // wrdy: the group wrote W
+        ptx::mbar_init(&gbar[10 * g + 6 + x], 1);    // vres: V-side MMA committed
+        ptx::mbar_init(&gbar[10 * g + 8 + x], 128);  // vemp: the group read the V sums
+      }
+    ptx::mbar_init(qready, 128);
     *abort_flag = 0;
     *last_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (mma_warp) {
+  if (kmma_warp) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
   }
-  if (tma_warp) {
-    if (lane == 0) {
-      ptx::prefetch_tmap(&tm_k);
-      ptx::prefetch_tmap(&tm_v);
-      ptx::prefetch_tmap(&tm_ks);
-      ptx::prefetch_tmap(&tm_vs);
-    }
-  }
 
-  // barriers and the TMEM address are visible to every warp from here on; the
-  // TMA warp starts streaming while the compute warps prepare the query limbs
+  // barriers and the TMEM address are visible to every warp from here on
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  // compute-thread identity: group gw, thread t in the group (row / channel)
-  const int gw = producer ? 0 : tid / 128;
-  const int t = tid & 127;
-  const int wq = warp & 3;  // TMEM lane quadrant of this warp
-  const int g0 = gw * GH;   // first head of my group
-  const int bar_id = 1 + gw;
-  float* red = reinterpret_cast<float*>(sm + L::red) + gw * 128;
-
-  // ---- query limbs: thread t = channel d, heads of its group
-  float qd[GH];
-  float qunit[GH];  // 2^(E_q - 6): weight of limb 0
-  if (!producer) {
-#pragma unroll
-    for (int i = 0; i < GH; ++i)
-      qd[i] = load_any(a.q, b * a.qs_b + (h * G + g0 + i) * a.qs_h + t, a.q_dtype) * a.qscale;
-    float qmax[GH];
-#pragma unroll
-    for (int i = 0; i < GH; ++i) qmax[i] = warp_max(fabsf(qd[i]));
-    if (lane == 0) {
-#pragma unroll
-      for (int i = 0; i < GH; ++i) red[wq * 32 + i] = qmax[i];
+  // a dependent launch may be scheduled as SMs free up: it only streams the
+  // archive until this grid has completed
+  if (a.overlap) ptx::grid_dep_launch();
+  if (tma_warp && lane == 0) {
+    // fill every stage at once, K and V of a tile together, while group 0
+    // prepares the query limbs
+    const int fk = min(NKS, ntiles), fv = min(NVS, ntiles);
+    for (int i = 0; i < fk || i < fv; ++i) {
+      if (i < fk) load_k(i);
+      if (i < fv) load_v(i);
     }
-    ptx::named_bar_sync(bar_id, 128);
-    uint8_t* qb = sm + L::qb;
+    nk = fk;
+    nv = fv;
+  }
+
+  uint64_t* kres = gbar + 10 * grp;
+  uint64_t* kemp = kres + 2;
+  uint64_t* wrdy = kres + 4;
+  uint64_t* vres = kres + 6;
+  uint64_t* vemp = kres + 8;
+  const uint32_t tm_grp = tmem + uint32_t(grp * 4 * NP);  // K buffers, then V buffers
+
+  // ---- group 0: the query as three int8 limbs per head (thread t = channel d)
+  if (!producer && grp == 0) {
+    if (a.overlap) {
+      ptx::grid_dep_wait();
+      load_q();
+    }
+    float* qmx = reinterpret_cast<float*>(sm + C::qs);
 #pragma unroll
-    for (int i = 0; i < GH; ++i) {
-      const float mx = fmaxf(fmaxf(red[i], red[32 + i]), fmaxf(red[64 + i], red[96 + i]));
+    for (int g = 0; g < G; ++g) {
+      const float mx = warp_max(fabsf(qd[g]));
+      if (lane == 0) qmx[w * G + g] = mx;
+    }
+    ptx::named_bar_sync(1, 128);
+    uint8_t* qb = sm + C::qb;
+    float* qu = reinterpret_cast<float*>(sm + C::qu);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float mx = fmaxf(fmaxf(qmx[g], qmx[G + g]), fmaxf(qmx[2 * G + g], qmx[3 * G + g]));
       const int e = exp_above(mx);
-      qunit[i] = pow2i(e - 6);
-      int l0, l1, l2;
-      limbs3(qd[i] * pow2i(6 - e), l0, l1, l2);
-      const int n = gw * CS + 3 * i;
-      qb[sw128_offset(n + 0, t)] = static_cast<uint8_t>(l0);
-      qb[sw128_offset(n + 1, t)] = static_cast<uint8_t>(l1);
-      qb[sw128_offset(n + 2, t)] = static_cast<uint8_t>(l2);
+      if (t == 0) qu[g] = pow2i(e - 6);
+      uint32_t l0, l1, l2;
+      limb_bytes(qd[g] * pow2i(6 - e), l0, l1, l2);
+      qb[sw128_offset(3 * g + 0, t)] = uint8_t(l0);
+      qb[sw128_offset(3 * g + 1, t)] = uint8_t(l1);
+      qb[sw128_offset(3 * g + 2, t)] = uint8_t(l2);
     }
-    for (int n = gw * CS + 3 * GH; n < (gw + 1) * CS; ++n) qb[sw128_offset(n, t)] = 0;
-    if (gw == GW - 1)
-      for (int n = GW * CS; n < NP; ++n) qb[sw128_offset(n, t)] = 0;
+    for (int n = 3 * G; n < NP; ++n) qb[sw128_offset(n, t)] = 0;
     ptx::fence_proxy_async_smem();
     ptx::mbar_arrive(qready);
   }
+
   if (tma_warp && lane == 0) {
-    // ================= TMA warp: keep the ring full. Stage s is refilled as
-    // soon as the V-side MMA of the tile it held has completed.
-    int loaded = 0;
-    for (; loaded < ntiles; ++loaded) {
-      const int s = loaded % kStages;
-      if (loaded >= kStages) waiter.wait(&vdone[s], uint32_t(loaded / kStages - 1) & 1u);
-      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-      const int row0 = (tile0 + loaded) * kRows;
-      ptx::mbar_arrive_expect_tx(&full[s], kStageTx);
-      ptx::tma_load_4d(sm + L::k + s * kTileBytes, &tm_k, &full[s], 0, row0, h, b);
-      ptx::tma_load_4d(sm + L::v + s * kTileBytes, &tm_v, &full[s], 0, row0, h, b);
-      ptx::tma_load_3d(sm + L::ks + s * kRows * 4, &tm_ks, &full[s], row0, h, b);
-      ptx::tma_load_3d(sm + L::vs + s * kRows * 4, &tm_vs, &full[s], row0, h, b);
-    }
-    // after an abort, every issued load must land before the CTA exits (bounded)
-    if (*reinterpret_cast<volatile int*>(abort_flag)) {
-      const unsigned long long t0 = clock64();
-      for (int i = 0; i < loaded; ++i)
-        while (!ptx::mbar_try_wait(&full[i % kStages], uint32_t(i / kStages) & 1u) &&
-               clock64() - t0 < kWaitCycles) {
-        }
-    }
-  }
-  if (mma_warp && lane == 0) {
-    // ================= K-MMA warp: S_int of each tile as soon as it lands
-    waiter.wait(qready, 0u);
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % kStages, bb = i & 1;
-      waiter.wait(&full[s], uint32_t(i / kStages) & 1u);
-      waiter.wait(&kempty[bb], (uint32_t(i >> 1) & 1u) ^ 1u);
-      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-      ptx::tc_fence_after();
-      const uint32_t ka = ptx::smem_u32(sm + L::k + s * kTileBytes);
-      const uint32_t qa = ptx::smem_u32(sm + L::qb);
-#pragma unroll
-      for (int k = 0; k < kD / 32; ++k)
-        ptx::mma_i8(tmem + bb * NP, ptx::desc_sw128(ka + 32 * k, 16, 1024),
-                    ptx::desc_sw128(qa + 32 * k, 16, 1024), kIdescK, k > 0 ? 1u : 0u);
-      ptx::mma_commit(&kfull[bb]);
-    }
-  }
-  if (mmav_warp && lane == 0) {
-    // ================= V-MMA warp: Acc_int of each tile as soon as its W is ready
-    for (int i = 0; i < ntiles; ++i) {
-      const int s = i % kStages, vb = i % 3;
-      waiter.wait(&wready[vb], uint32_t(i / 3) & 1u);
-      waiter.wait(&vempty[vb], (uint32_t(i / 3) & 1u) ^ 1u);
-      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-      ptx::tc_fence_after();
-      const uint32_t va = ptx::smem_u32(sm + L::v + s * kTileBytes);
-      const uint32_t wa = ptx::smem_u32(sm + L::wb + vb * kWBytes);
-#pragma unroll
-      for (int k = 0; k < kRows / 32; ++k)
-        ptx::mma_i8(tmem + 2 * NP + vb * NP, ptx::desc_sw128(va + 4096 * k, kTileBytes, 1024),
-                    ptx::desc_noswizzle(wa + 512 * k, 128, 2048), kIdescV, k > 0 ? 1u : 0u);
-      // completes when this and every earlier V-side MMA has finished; the
-      // K-side MMA of the same tile finished before its W could be written
-      ptx::mma_commit(&vdone[s]);
-    }
-  }
-
-  // ================= compute warps
-  float m_run[GH], lsum[GH], acc[GH];
-#pragma unroll
-  for (int i = 0; i < GH; ++i) {
-    m_run[i] = -INFINITY;
-    lsum[i] = 0.f;
-    acc[i] = 0.f;
-  }
-  if (!producer) {
-    const int j = lane % S;
-    float2 areg[TPT][S];  // (A[t][jj], A[t][jj]) for my tokens t = j * TPT + i
-#pragma unroll
-    for (int i = 0; i < TPT; ++i)
-#pragma unroll
-      for (int jj = 0; jj < S; ++jj) {
-        const float av = basis.m[jj][j * TPT + i];
-        areg[i][jj] = make_float2(av, av);
+    // ================= TMA thread: both rings, in tile order each, whichever
+    // has a free stage (every stage was filled once before the setup barrier)
+    unsigned long long t_last = clock64();
+    while (nk < ntiles || nv < ntiles) {
+      bool prog = false;
+      if (nk < ntiles && ptx::mbar_test_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u)) {
+        load_k(nk++);
+        prog = true;
       }
-    const float sqrtR = sqrtf(float(R));
-    const uint32_t lane_off = uint32_t(wq * 32) << 16;
-    const uint32_t col0 = uint32_t(gw * CS);
-    // softmax rescale and W unit of the two tiles whose V epilogue is pending
-    float alpha_p1[GH], wunit_p1[GH], alpha_p2[GH], wunit_p2[GH];
+      if (nv < ntiles && ptx::mbar_test_wait(&vfree[nv % NVS], uint32_t(nv / NVS - 1) & 1u)) {
+        load_v(nv++);
+        prog = true;
+      }
+      if (prog) {
+        t_last = clock64();
+        continue;
+      }
+      if (*reinterpret_cast<volatile int*>(abort_flag)) break;
+      if (clock64() - t_last > kWaitCycles) {
+        *reinterpret_cast<volatile int*>(abort_flag) = 1;
+        if (a.status) atomicOr(a.status, 1u);
+        break;
+      }
+      __nanosleep(32);
+    }
+    // after an abort, the newest load of every stage must land before the
+    // CTA exits (older ones completed before their stage was reissued)
+    if (*reinterpret_cast<volatile int*>(abort_flag)) {
+      for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
+      for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
+    }
+  }
+  if (kmma_warp && lane == 0) {
+    // ================= K-MMA thread: S_int of each tile into its group's
+    // TMEM buffer as soon as it lands
+    waiter.wait(qready, 0u);
+    int i = 0;
+    for (; i < ntiles; ++i) {
+      const int s = i % NKS, g = i % NG, k = i / NG, x = k & 1;
+      uint64_t* gq = gbar + 10 * g;
+      if (!waiter.wait(&kfull[s], uint32_t(i / NKS) & 1u)) break;
+      if (!waiter.wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+      ptx::tc_fence_after();
+      const uint32_t ka = ptx::smem_u32(sm + C::kt + s * kTileBytes);
+      const uint32_t qa = ptx::smem_u32(sm + C::qb);
+      const uint32_t d = tmem + uint32_t(g * 4 * NP + x * NP);
 #pragma unroll
-    for (int i = 0; i < GH; ++i) {
-      alpha_p1[i] = alpha_p2[i] = 1.f;
-      wunit_p1[i] = wunit_p2[i] = 0.f;
+      for (int kk = 0; kk < kD / 32; ++kk)
+        ptx::mma_i8(d, ptx::desc_sw128(ka + 32 * kk, 16, 1024), ptx::desc_sw128(qa + 32 * kk, 16, 1024),
+                    kIdescK, kk > 0 ? 1u : 0u);
+      ptx::mma_commit(&kfree[s]);
+      ptx::mma_commit(&gq[x]);
+    }
+    // after an abort, the MMAs already issued finish before TMEM is freed
+    if (i < ntiles && i > 0) drain_wait(&kfree[(i - 1) % NKS], uint32_t((i - 1) / NKS) & 1u);
+  }
+  if (vmma_warp && lane == 0) {
+    // ================= V-MMA thread: Acc_int of each tile as soon as its W is
+    // written
+    int i = 0;
+    for (; i < ntiles; ++i) {
+      const int s = i % NVS, g = i % NG, k = i / NG, x = k & 1;
+      uint64_t* gq = gbar + 10 * g;
+      if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) break;
+      if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) break;
+      if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+      ptx::tc_fence_after();
+      const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
+      const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
+      const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
+#pragma unroll
+      for (int kk = 0; kk < kRows / 32; ++kk)
+        ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
+                    ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
+      ptx::mma_commit(&vfree[s]);
+      ptx::mma_commit(&gq[6 + x]);
+    }
+    if (i < ntiles && i > 0) drain_wait(&vfree[(i - 1) % NVS], uint32_t((i - 1) / NVS) & 1u);
+  }
+
+  // ================= compute groups
+  float m_run[G], acc[G];
+  float lsum[NI];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m_run[g] = -INFINITY;
+    acc[g] = 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < NI; ++i) lsum[i] = 0.f;
+  const int bl = lane / S, jj = lane % S;  // block in the warp, row of the block
+  const bool own = G >= S || jj < G;       // lane owns (block, head) items
+  if (!producer) {
+    // zero this group's W buffers once: the pad columns are never written
+    {
+      uint4* wz = reinterpret_cast<uint4*>(sm + C::wb + grp * 2 * kWBytes);
+      for (int x = t; x < int(2 * kWBytes / 16); x += 128) wz[x] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    waiter.wait(qready, 0u);
+    float qunit[G];  // weight of limb 0 of each head
+#pragma unroll
+    for (int g = 0; g < G; ++g) qunit[g] = reinterpret_cast<const float*>(sm + C::qu)[g];
+    const int bt = w * C::BW + bl;  // block in the tile
+    float* xw = reinterpret_cast<float*>(sm + C::xs) + (grp * 4 + w) * C::XW + bl * XP;
+    float* rdbase = reinterpret_cast<float*>(sm + C::red) + grp * 2 * (G + 1) * 4;
+    uint8_t* wbase = sm + C::wb + grp * 2 * kWBytes;
+    const float sqrtR = sqrtf(float(R));
+    const uint32_t lane_off = uint32_t(w * 32) << 16;
+    float alpha_p[G], wunit_p[G];  // of the tile whose V epilogue is pending
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      alpha_p[g] = 1.f;
+      wunit_p[g] = 0.f;
     }
 
-    // V epilogue of tile i: acc = alpha(i) acc + W-limb sums (run two tiles
-    // late, so the V-side MMA round trip overlaps two softmax passes)
-    auto v_epilogue = [&](int i, const float (&al)[GH], const float (&wu)[GH]) {
-      const int vb = i % 3;
-      waiter.wait(&vdone[i % kStages], uint32_t(i / kStages) & 1u);
+    // V epilogue of group iteration kk: acc = alpha acc + W-limb sums
+    auto v_epilogue = [&](int kk, const float (&al)[G], const float (&wu)[G]) {
+      const int x = kk & 1;
+      waiter.wait(&vres[x], uint32_t(kk >> 1) & 1u);
       ptx::tc_fence_after();
-      uint32_t vr[CS];
-      tmem_ld_cols<CS>(tmem + 2 * NP + vb * NP + col0 + lane_off, vr);
+      uint32_t vr[NP];
+      tmem_ld_cols<NP>(tm_grp + 2 * NP + x * NP + lane_off, vr);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&vempty[vb]);
+      ptx::mbar_arrive(&vemp[x]);
 #pragma unroll
-      for (int g = 0; g < GH; ++g)
+      for (int g = 0; g < G; ++g)
         acc[g] = fmaf(acc[g], al[g], wu[g] * unlimb3(vr[3 * g], vr[3 * g + 1], vr[3 * g + 2]));
     };
 
-    for (int it = 0; it < ntiles; ++it) {
-      const int s = it % kStages, bb = it & 1;
-      const int tile = tile0 + it;
-      // ---- K side results
-      waiter.wait(&kfull[bb], uint32_t(it >> 1) & 1u);
+    int k = 0;
+    for (; grp + k * NG < ntiles; ++k) {
+      const int i = grp + k * NG;  // tile of the chunk
+      const int x = k & 1;
+      const int sv = i % NVS;
+      const int64_t tile = tile0 + i;
+      // ---- K sums of my row, every head
+      waiter.wait(&kres[x], uint32_t(k >> 1) & 1u);
       ptx::tc_fence_after();
-      uint32_t cr[CS];
-      tmem_ld_cols<CS>(tmem + bb * NP + col0 + lane_off, cr);
+      uint32_t cr[NP];
+      tmem_ld_cols<NP>(tm_grp + x * NP + lane_off, cr);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&kempty[bb]);
-      const float sk = reinterpret_cast<const float*>(sm + L::ks)[s * kRows + t];
-      const float sv = reinterpret_cast<const float*>(sm + L::vs)[s * kRows + t];
-      float sval[GH];
+      ptx::mbar_arrive(&kemp[x]);
+      waiter.wait(&vfull[sv], uint32_t(i / NVS) & 1u);
+      const float* scs = reinterpret_cast<const float*>(sm + C::sc + sv * 2 * kScaleBytes);
+      const float sk = scs[t];
+      // s = scale_k C_k q of my row for every head, transposed through shared
+      // memory to (block, head) items: the S scores of each of my blocks' heads
 #pragma unroll
-      for (int g = 0; g < GH; ++g) sval[g] = sk * qunit[g] * unlimb3(cr[3 * g], cr[3 * g + 1], cr[3 * g + 2]);
+      for (int g = 0; g < G; ++g)
+        xw[g * S + jj] = (sk * qunit[g]) * unlimb3(cr[3 * g], cr[3 * g + 1], cr[3 * g + 2]);
+      __syncwarp();
+      float sb[NI][S];
+#pragma unroll
+      for (int ii = 0; ii < NI; ++ii) load_floats<S>(xw + (own ? jj * NI + ii : 0) * S, sb[ii]);
+      float vsc[S];  // V scales of my block
+      load_floats<S>(scs + kRows + bt * S, vsc);
 
-      // gather the S rows of my block
-      float sb[S][GH];
+      // logits of my items (basis entries are compile-time constant operands)
+      const bool live = tile * C::TB + bt < a.nb;
+      float lg[NI][R];
+      float mx[NI];
 #pragma unroll
-      for (int jj = 0; jj < S; ++jj)
+      for (int ii = 0; ii < NI; ++ii) {
+        float m = -INFINITY;
 #pragma unroll
-        for (int g = 0; g < GH; ++g) sb[jj][g] = __shfl_sync(0xffffffffu, sval[g], (lane - j) + jj);
-
-      const bool live = int64_t(tile) * TB + t / S < a.nb;
-      // logits of my TPT tokens, heads in pairs (packed fp32x2 FMA)
-      float lg[TPT][GH];
+        for (int tk = 0; tk < R; ++tk) {
+          float v = basis.m[0][tk] * sb[ii][0];
 #pragma unroll
-      for (int i = 0; i < TPT; ++i) {
-        if constexpr (GH == 1) {
-          float x = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < S; ++jj) x = fmaf(areg[i][jj].x, sb[jj][0], x);
-          lg[i][0] = x;
-        } else {
-#pragma unroll
-          for (int g = 0; g < GH; g += 2) {
-            float2 x = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int jj = 0; jj < S; ++jj) x = __ffma2_rn(areg[i][jj], make_float2(sb[jj][g], sb[jj][g + 1]), x);
-            lg[i][g] = x.x;
-            lg[i][g + 1] = x.y;
-          }
+          for (int q = 1; q < S; ++q) v = fmaf(basis.m[q][tk], sb[ii][q], v);
+          lg[ii][tk] = v;
+          m = fmaxf(m, v);
         }
+        m = live && own ? m : -INFINITY;
+#pragma unroll
+        for (int o = S; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        mx[ii] = m;
       }
-      float tmax[GH];
+      // the tile's largest V scale (scales are >= 0, so their bit patterns
+      // order like their values)
+      float vm = vsc[0];
 #pragma unroll
-      for (int g = 0; g < GH; ++g) {
-        float mx = -INFINITY;
+      for (int q = 1; q < S; ++q) vm = fmaxf(vm, vsc[q]);
+      vm = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(vm)));
+      // per-warp maxima -> tile maxima (one barrier; slots alternate by tile)
+      float* rd = rdbase + x * (G + 1) * 4;
+      if (bl == 0 && own) {
 #pragma unroll
-        for (int i = 0; i < TPT; ++i) mx = fmaxf(mx, lg[i][g]);
-        tmax[g] = live ? mx : -INFINITY;
+        for (int ii = 0; ii < NI; ++ii) rd[(jj * NI + ii) * 4 + w] = mx[ii];
       }
-      // tile-wide max per head and the largest V scale of the tile
-      float vmax = sv;
-#pragma unroll
-      for (int g = 0; g < GH; ++g) tmax[g] = warp_max(tmax[g]);
-      vmax = warp_max(vmax);
-      if (lane == 0) {
-#pragma unroll
-        for (int g = 0; g < GH; ++g) red[wq * 32 + g] = tmax[g];
-        red[wq * 32 + 31] = vmax;
-      }
-      ptx::named_bar_sync(bar_id, 128);
-#pragma unroll
-      for (int g = 0; g < GH; ++g) tmax[g] = fmaxf(fmaxf(red[g], red[32 + g]), fmaxf(red[64 + g], red[96 + g]));
-      vmax = fmaxf(fmaxf(red[31], red[63]), fmaxf(red[95], red[127]));
-      ptx::named_bar_sync(bar_id, 128);  // red is rewritten next tile
-
-      float m_new[GH], alpha[GH], wunit[GH], winv[GH];
-#pragma unroll
-      for (int g = 0; g < GH; ++g) {
-        m_new[g] = fmaxf(m_run[g], tmax[g]);
-        alpha[g] = ptx::ex2(m_run[g] - m_new[g]);
-        const int e = exp_above(ptx::ex2(tmax[g] - m_new[g]) * sqrtR * vmax);
-        wunit[g] = pow2i(e - 6);
-        winv[g] = pow2i(6 - e);
-      }
-      // p, the softmax sum, and my tokens' share of w_jj = sum_t p_t A[t][jj]
-      float2 wpart[S][(GH + 1) / 2];
-#pragma unroll
-      for (int jj = 0; jj < S; ++jj)
-#pragma unroll
-        for (int g2 = 0; g2 < (GH + 1) / 2; ++g2) wpart[jj][g2] = make_float2(0.f, 0.f);
-      float ps[GH];
-#pragma unroll
-      for (int g = 0; g < GH; ++g) ps[g] = 0.f;
-#pragma unroll
-      for (int i = 0; i < TPT; ++i) {
-        float p[GH];
-#pragma unroll
-        for (int g = 0; g < GH; ++g) {
-          p[g] = live ? ptx::ex2(lg[i][g] - m_new[g]) : 0.f;
-          ps[g] += p[g];
-        }
-        if constexpr (GH == 1) {
-#pragma unroll
-          for (int jj = 0; jj < S; ++jj) wpart[jj][0].x = fmaf(p[0], areg[i][jj].x, wpart[jj][0].x);
-        } else {
-#pragma unroll
-          for (int g = 0; g < GH; g += 2)
-#pragma unroll
-            for (int jj = 0; jj < S; ++jj)
-              wpart[jj][g / 2] = __ffma2_rn(make_float2(p[g], p[g + 1]), areg[i][jj], wpart[jj][g / 2]);
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < GH; ++g) lsum[g] = fmaf(lsum[g], alpha[g], ps[g]);
-      // sum the shares over the S lanes of the block
-#pragma unroll
-      for (int o = 1; o < S; o <<= 1)
-#pragma unroll
-        for (int jj = 0; jj < S; ++jj)
-#pragma unroll
-          for (int g2 = 0; g2 < (GH + 1) / 2; ++g2) {
-            float2 other;
-            other.x = __shfl_xor_sync(0xffffffffu, wpart[jj][g2].x, o);
-            other.y = GH == 1 ? 0.f : __shfl_xor_sync(0xffffffffu, wpart[jj][g2].y, o);
-            wpart[jj][g2] = __fadd2_rn(wpart[jj][g2], other);
-          }
-      // W = w_j * scale_v as three int8 limbs: this group's CS bytes of row t
+      if (lane == 0) rd[G * 4 + w] = vm;
+      ptx::named_bar_sync(1 + grp, 128);
+      float m_new[G], alpha[G], wunit[G], winv[G];
       {
-        uint32_t packed[CS / 4];
+        const float4 v4 = reinterpret_cast<const float4*>(rd)[G];
+        const float vmax = fmaxf(fmaxf(v4.x, v4.y), fmaxf(v4.z, v4.w));
 #pragma unroll
-        for (int q = 0; q < CS / 4; ++q) packed[q] = 0u;
-#pragma unroll
-        for (int g = 0; g < GH; ++g) {
-          float wj = 0.f;
-#pragma unroll
-          for (int jj = 0; jj < S; ++jj) {
-            const float cand = (g & 1) ? wpart[jj][g / 2].y : wpart[jj][g / 2].x;
-            wj = (jj == j) ? cand : wj;
-          }
-          int l[3];
-          limbs3(wj * sv * winv[g], l[0], l[1], l[2]);
-#pragma unroll
-          for (int k = 0; k < 3; ++k) {
-            const int byte = 3 * g + k;
-            packed[byte / 4] |= (uint32_t(l[k]) & 0xffu) << (8 * (byte % 4));
-          }
+        for (int g = 0; g < G; ++g) {
+          const float4 r4 = reinterpret_cast<const float4*>(rd)[g];
+          const float tmax = fmaxf(fmaxf(r4.x, r4.y), fmaxf(r4.z, r4.w));
+          m_new[g] = fmaxf(m_run[g], tmax);
+          alpha[g] = ptx::ex2(m_run[g] - m_new[g]);
+          const int e = exp_above(ptx::ex2(tmax - m_new[g]) * sqrtR * vmax);
+          wunit[g] = pow2i(e - 6);
+          winv[g] = pow2i(6 - e);
         }
-        uint8_t* wrow = sm + L::wb + (it % 3) * kWBytes;
-        // column c of row t lives at (c / 16) * 2048 + t * 16 + c % 16
-        if constexpr (CS == 8) {
-          *reinterpret_cast<uint2*>(wrow + (gw / 2) * 2048 + t * 16 + (gw % 2) * 8) =
-              make_uint2(packed[0], packed[1]);
-        } else {
-          *reinterpret_cast<uint4*>(wrow + gw * 2048 + t * 16) =
-              make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+      // p, softmax sums, w_j = sum_t p_t A[t][j], and W = w * scale_v as
+      // three int8 limbs: S bytes (my block's rows) of each limb column
+      uint8_t* wbuf = wbase + x * kWBytes;
+#pragma unroll
+      for (int ii = 0; ii < NI; ++ii) {
+        if (!own) continue;
+        const int hh = jj * NI + ii;
+        const float me = live ? pick(m_new, hh) : INFINITY;  // dead blocks: p = 0
+        float p[R];
+        float ps = 0.f;
+#pragma unroll
+        for (int tk = 0; tk < R; ++tk) {
+          p[tk] = ptx::ex2(lg[ii][tk] - me);
+          ps += p[tk];
         }
+        lsum[ii] = fmaf(lsum[ii], pick(alpha, hh), ps);
+        const float wi = pick(winv, hh);
+        uint32_t by[3][S];
+#pragma unroll
+        for (int q = 0; q < S; ++q) {
+          float wq = p[0] * basis.m[q][0];
+#pragma unroll
+          for (int tk = 1; tk < R; ++tk) wq = fmaf(p[tk], basis.m[q][tk], wq);
+          limb_bytes(wq * vsc[q] * wi, by[0][q], by[1][q], by[2][q]);
+        }
+#pragma unroll
+        for (int l = 0; l < 3; ++l) store_bytes<S>(wbuf + w_offset<C::LBO>(3 * hh + l, bt * S), by[l]);
       }
       ptx::fence_proxy_async_smem();
-      ptx::mbar_arrive(&wready[it % 3]);
+      ptx::mbar_arrive(&wrdy[x]);
 #pragma unroll
-      for (int g = 0; g < GH; ++g) m_run[g] = m_new[g];
+      for (int g = 0; g < G; ++g) m_run[g] = m_new[g];
 
-      // ---- V epilogue of the tile two back (its MMA overlapped two softmaxes)
-      if (it >= 2) v_epilogue(it - 2, alpha_p2, wunit_p2);
+      // ---- V epilogue of my previous tile (its MMA overlapped this softmax)
+      if (k >= 1) v_epilogue(k - 1, alpha_p, wunit_p);
 #pragma unroll
-      for (int g = 0; g < GH; ++g) {
-        alpha_p2[g] = alpha_p1[g];
-        wunit_p2[g] = wunit_p1[g];
-        alpha_p1[g] = alpha[g];
-        wunit_p1[g] = wunit[g];
+      for (int g = 0; g < G; ++g) {
+        alpha_p[g] = alpha[g];
+        wunit_p[g] = wunit[g];
       }
     }
-    if (ntiles >= 2) v_epilogue(ntiles - 2, alpha_p2, wunit_p2);
-    if (ntiles >= 1) v_epilogue(ntiles - 1, alpha_p1, wunit_p1);
+    if (k >= 1) v_epilogue(k - 1, alpha_p, wunit_p);
+  }
 
-    // ---- raw tail tokens (last chunk): thread t = channel d
-    if (c == a.ns - 1) {
+  // ---- merge the four groups' states, fold the raw tail, write the partials
+  const bool direct = a.fuse && a.ns == 1;
+  if (!producer) {
+    // softmax sums of my items over the warp's blocks
+#pragma unroll
+    for (int ii = 0; ii < NI; ++ii)
+#pragma unroll
+      for (int o = S; o < 32; o <<= 1) lsum[ii] += __shfl_xor_sync(0xffffffffu, lsum[ii], o);
+    // the tails, the workspace and out: after the preceding work
+    if (a.overlap) ptx::grid_dep_wait();
+    // every group is done with both rings: the K ring becomes merge scratch
+    ptx::named_bar_sync(kFinBar, 128 * NG);
+    float* fm = reinterpret_cast<float*>(sm + C::kt);  // [group][head] running max
+    float* fl = fm + (NG * G + 3) / 4 * 4;              // [group][head][warp] sums (16-B aligned)
+    float* fa = fl + NG * G * 4;                        // [group][head][channel] acc
+    if (t == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) fm[grp * G + g] = m_run[g];
+    }
+    if (bl == 0 && own) {
+#pragma unroll
+      for (int ii = 0; ii < NI; ++ii) fl[(grp * G + jj * NI + ii) * 4 + w] = lsum[ii];
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) fa[(grp * G + g) * kD + t] = acc[g];
+    ptx::named_bar_sync(kFinBar, 128 * NG);
+
+    // group grp finishes heads grp, grp + 4, ...: thread t = channel d
+    constexpr int HPG = C::HPG;
+    float Mh[HPG], Lh[HPG], Ah[HPG];
+#pragma unroll
+    for (int y = 0; y < HPG; ++y) {
+      const int g = min(grp + NG * y, G - 1);
+      float M = -INFINITY;
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        const float4 l4 = reinterpret_cast<const float4*>(fl)[gg * G + g];
+        if (l4.x + l4.y + l4.z + l4.w > 0.f) M = fmaxf(M, fm[gg * G + g]);
+      }
+      float Ls = 0.f, As = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < NG; ++gg) {
+        const float4 l4 = reinterpret_cast<const float4*>(fl)[gg * G + g];
+        const float lt = l4.x + l4.y + l4.z + l4.w;
+        if (lt > 0.f) {
+          const float e = ptx::ex2(fm[gg * G + g] - M);
+          Ls = fmaf(lt, e, Ls);
+          As = fmaf(fa[(gg * G + g) * kD + t], e, As);
+        }
+      }
+      Mh[y] = M;
+      Lh[y] = Ls;
+      Ah[y] = As;
+    }
+    const bool active = grp < G;  // uniform per group
+    // raw tail tokens (last chunk)
+    if (active && c == a.ns - 1 && a.nr > 0) {
+      float* red2 = reinterpret_cast<float*>(sm + C::xs) + grp * 4 * C::XW;
+      float qh[HPG];
+#pragma unroll
+      for (int y = 0; y < HPG; ++y) {
+        const int g = min(grp + NG * y, G - 1);
+        qh[y] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
+      }
       for (int tt = 0; tt < a.nr; ++tt) {
         const float kd = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, a.t_dtype);
         const float vd = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, a.t_dtype);
-        float lgt[GH];
+        float lgt[HPG];
 #pragma unroll
-        for (int g = 0; g < GH; ++g) lgt[g] = qd[g] * kd;
-        group_sum<GH>(lgt, red, wq, lane, bar_id);
+        for (int y = 0; y < HPG; ++y) lgt[y] = qh[y] * kd;
+        group_sum<HPG>(lgt, red2, w, lane, 1 + grp);
 #pragma unroll
-        for (int g = 0; g < GH; ++g) {
-          const float mn = fmaxf(m_run[g], lgt[g]);
-          const float al = ptx::ex2(m_run[g] - mn);
-          const float p = ptx::ex2(lgt[g] - mn);
-          acc[g] = fmaf(acc[g], al, p * vd);
-          lsum[g] = fmaf(lsum[g], al, t == 0 ? p : 0.f);
-          m_run[g] = mn;
+        for (int y = 0; y < HPG; ++y) {
+          const float mn = fmaxf(Mh[y], lgt[y]);
+          const float al = ptx::ex2(Mh[y] - mn);
+          const float p = ptx::ex2(lgt[y] - mn);
+          Ah[y] = fmaf(Ah[y], al, p * vd);
+          Lh[y] = fmaf(Lh[y], al, p);
+          Mh[y] = mn;
         }
       }
     }
-    group_sum<GH>(lsum, red, wq, lane, bar_id);
-  }
-
-  // ---- partials (or the output)
-  const bool direct = a.fuse && a.ns == 1;
-  if (!producer) {
+    if (active) {
 #pragma unroll
-    for (int g = 0; g < GH; ++g) {
-      const int hq = h * G + g0 + g;
-      if (direct) {
-        store_out(a.out, b * a.os_b + hq * a.os_h + t, a.out_dtype, acc[g] / lsum[g]);
-      } else {
-        const int64_t row = (int64_t(b) * Hq + hq) * a.ns + c;
-        a.pacc[row * kD + t] = acc[g];
-        if (t == 0) {
-          a.pm[row] = lsum[g] > 0.f ? m_run[g] : -INFINITY;
-          a.pl[row] = lsum[g];
+      for (int y = 0; y < HPG; ++y) {
+        const int g = grp + NG * y;
+        if (g >= G) continue;
+        const int hq = h * G + g;
+        if (direct) {
+          store_out(a.out, b * a.os_b + hq * a.os_h + t, a.out_dtype, Ah[y] / Lh[y]);
+        } else {
+          const int64_t row = (int64_t(b) * Hq + hq) * a.ns + c;
+          a.pacc[row * kD + t] = Ah[y];
+          if (t == 0) {
+            a.pm[row] = Lh[y] > 0.f ? Mh[y] : -INFINITY;
+            a.pl[row] = Lh[y];
+          }
         }
       }
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (mma_warp) {
+  if (kmma_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
 
   if (direct || !a.fuse) return;
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const unsigned tk = atomicAdd(a.tickets + (b * a.Hk + h), 1u);
-    *last_flag = (tk == unsigned(a.ns - 1)) ? 1 : 0;
-  }
-  __syncthreads();
-  if (!*last_flag) return;
-  __threadfence();
-  float* wts = reinterpret_cast<float*>(sm);  // stage buffers are free now
+  if (!last_cta_ticket(a.tickets + (b * a.Hk + h), a.ns, last_flag)) return;
+  float* wts = reinterpret_cast<float*>(sm);  // the rings are free now
   const int64_t row = (int64_t(b) * Hq + h * G) * a.ns;
   combine_heads(a.pm + row, a.pl + row, a.pacc + row * kD, G, a.ns, kD, wts, a.out,
                 b * a.os_b + (h * G) * a.os_h, a.os_h, a.out_dtype);
@@ -689,14 +850,22 @@ bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
 
 template <int G, int S, int TPT>
 int launch(const TcArgs& ta, const Basis& basis, const CUtensorMap* maps, cudaStream_t stream) {
-  using Cl = Cols<G>;
-  const size_t smem = SmemLayout<Cl::NP>::alloc;
+  using C = Cfg<G, S, TPT>;
+  const size_t smem = C::alloc;
   auto kern = decode_tc_kernel<G, S, TPT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return FC_ERR_CUDA;
-  const dim3 grid(unsigned(ta.d.ns), unsigned(ta.d.Hk), unsigned(ta.d.B));
-  kern<<<grid, Cl::kThreads, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], ta, basis);
-  return cuda_status(cudaGetLastError());
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(ta.d.ns), unsigned(ta.d.Hk), unsigned(ta.d.B));
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ta.d.overlap ? 1 : 0;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], ta, basis));
 }
 
 }  // namespace tc
@@ -710,10 +879,11 @@ bool decode_tc_eligible(const fc_archive* ka, const fc_archive* va, int G) {
   const int tpt = R / S;
   if (!(G == 1 || G == 2 || G == 4 || G == 8)) return false;
   switch (S * 100 + tpt) {
-    case 204: case 208: case 402: case 404: case 802: case 104: case 108: break;
+    case 104: case 108: case 204: case 208: case 402: case 404: case 802: break;
     default: return false;
   }
-  return S * G <= 32 && tpt * G <= 32;
+  const int ni = G >= S ? G / S : 1;
+  return ni * R <= 32;
 }
 
 int tc_tiles_per_head(int64_t nb, int S) { return int((nb + (tc::kRows / S) - 1) / (tc::kRows / S)); }
@@ -733,13 +903,13 @@ int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive
   switch (key) {
 #define FC_TC_CASE(G, S, T) \
   case G * 10000 + S * 100 + T: return tc::launch<G, S, T>(ta, basis, maps, stream);
+    FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
+    FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
     FC_TC_CASE(1, 2, 4) FC_TC_CASE(2, 2, 4) FC_TC_CASE(4, 2, 4) FC_TC_CASE(8, 2, 4)
     FC_TC_CASE(1, 2, 8) FC_TC_CASE(2, 2, 8) FC_TC_CASE(4, 2, 8)
     FC_TC_CASE(1, 4, 2) FC_TC_CASE(2, 4, 2) FC_TC_CASE(4, 4, 2) FC_TC_CASE(8, 4, 2)
     FC_TC_CASE(1, 4, 4) FC_TC_CASE(2, 4, 4) FC_TC_CASE(4, 4, 4) FC_TC_CASE(8, 4, 4)
-    FC_TC_CASE(1, 8, 2) FC_TC_CASE(2, 8, 2) FC_TC_CASE(4, 8, 2)
-    FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
-    FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
+    FC_TC_CASE(1, 8, 2) FC_TC_CASE(2, 8, 2) FC_TC_CASE(4, 8, 2) FC_TC_CASE(8, 8, 2)
 #undef FC_TC_CASE
     default: return FC_ERR_UNSUPPORTED;
   }

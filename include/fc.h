@@ -61,7 +61,8 @@ enum {
 /* fc_decode_attention flags. */
 enum {
   FC_DECODE_FUSE_COMBINE = 1, /* the last CTA of each kv head writes `out` */
-  FC_DECODE_PORTABLE = 2      /* force the portable CUDA-core kernel */
+  FC_DECODE_PORTABLE = 2,     /* force the portable CUDA-core kernel */
+  FC_DECODE_OVERLAP = 4       /* start before the preceding stream work ends */
 };
 
 /* Element types. */
@@ -212,6 +213,18 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *              FC_DECODE_PORTABLE: use the portable CUDA-core kernel even
  *              where the tensor-core kernel applies (int8 K and V, D = 128,
  *              S dividing 32, R / S in {2, 4, 8}, G <= 8).
+ *              FC_DECODE_OVERLAP (tensor-core kernel; ignored otherwise):
+ *              launch as a programmatic dependent of the preceding work on
+ *              `stream`. The kernel then streams archive blocks
+ *              [0, n_blocks - 1) while that work is still running, and waits
+ *              for it before it reads q, the tails or block n_blocks - 1 and
+ *              before it writes the workspace or `out`. Precondition: no
+ *              work still in flight on the stream writes archive blocks
+ *              below n_blocks - 1. A decode loop of fc_append_step and
+ *              fc_decode_attention meets it (an append writes at most block
+ *              n_blocks - 1 and the tails); a fc_compress_blocks of the same
+ *              archive queued just before does not. Pure scheduling: the
+ *              results are those of a launch without the flag.
  *   workspace       device, >= fc_decode_workspace_bytes(B, Hq, D, splits)
  *                   bytes, 256-byte aligned. Its first 256 + 4*B*Hq bytes
  *                   (status word and tickets) must be zero before the first

@@ -175,3 +175,76 @@ def test_end_to_end_against_oracle_archive():
     err = np.max(np.abs(got - ref))
     rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
     assert rel <= 1e-3 and err <= 1e-2, (err, rel)
+
+
+# every (G, S, R / S) the tensor-core kernel is instantiated for: lanes with
+# several heads (G > S), idle lanes (G < S), one coefficient per block (S = 1),
+# three compute groups (G = 8 or S = 8); 8+ tiles with a partial last tile
+TC_CONFIGS = [(G, S, T) for (S, T) in ((1, 4), (1, 8), (2, 4), (2, 8), (4, 2),
+                                       (4, 4), (8, 2))
+              for G in (1, 2, 4, 8) if max(1, G // S) * S * T <= 32]
+
+
+@pytest.mark.parametrize("cfg", TC_CONFIGS,
+                         ids=lambda c: "G%d-S%d-R%d" % (c[0], c[1], c[1] * c[2]))
+def test_tensor_core_configurations(cfg):
+    G, S, T = cfg
+    R = S * T
+    tb = 128 // S
+    nb = 7 * tb + 5
+    Hk = 2
+    w = synth.Workload("tc", B=1, Hq=Hk * G, Hk=Hk, D=128, T=nb * R + 3, R=R,
+                       S=S, k_coeff="i8", v_coeff="i8", in_dtype="bf16",
+                       rho=0.9, outlier_frac=0.01, seed=G * 100 + R)
+    cache, data = _cache_for(w)
+    q = data["q"].to(DEV)
+    ref = oracle_on_gpu_archive(cache, q)
+    for ns in (0, 1, 3):
+        out = cache.attention(q, num_splits=ns)
+        torch.cuda.synchronize()
+        check_out(f64(out), ref, "ns=%d" % ns)
+    assert _lib.fc_workspace_status(cache._ws) == 0
+
+
+def test_overlap_launch_matches_plain_launch():
+    """FC_DECODE_OVERLAP is scheduling only: a decode loop of appends and
+    overlapped attentions (and back-to-back overlapped attentions on two
+    caches, captured in a CUDA graph) gives bit-identical outputs to plain
+    launches."""
+    w = synth.WORKLOADS["gqa"].replace(B=2, T=8 * 300 + 6, seed=31)
+    data = synth.generate(w.replace(steps=12), q_steps=12)
+    caches = []
+    for _ in range(2):
+        c = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV)
+        c.prefill(data["k"][:, :, :w.T].to(DEV), data["v"][:, :, :w.T].to(DEV))
+        caches.append(c)
+    torch.cuda.synchronize()
+    kd, vd, qs = data["k"].to(DEV), data["v"].to(DEV), data["q"].to(DEV)
+    plain, over = [], []
+    for step in range(12):       # crosses a block boundary (T % 8 = 6)
+        t = w.T + step
+        for i, c in enumerate(caches):
+            c.append(kd[:, :, t:t + 1], vd[:, :, t:t + 1])
+            if i == 0:
+                plain.append(c.attention(qs[step]))
+            else:
+                over.append(c.attention(qs[step], overlap=True))
+    torch.cuda.synchronize()
+    for a, b in zip(plain, over):
+        assert torch.equal(a, b)
+    check_out(f64(over[-1]), oracle_on_gpu_archive(caches[1], qs[11]), "loop")
+    # back to back on alternating caches inside a graph
+    outs = [torch.empty_like(plain[0]) for _ in range(4)]
+    for i in range(4):
+        caches[i % 2].attention(qs[i], out=outs[i], overlap=True)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(4):
+            caches[i % 2].attention(qs[i], out=outs[i], overlap=True)
+    g.replay()
+    torch.cuda.synchronize()
+    for i in range(4):
+        ref = caches[i % 2].attention(qs[i])
+        torch.cuda.synchronize()
+        assert torch.equal(outs[i], ref)
