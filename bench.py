@@ -254,7 +254,7 @@ def run_fc(args, world, rank, local):
         for i in range(K):
             c = i % copies
             caches[c].attention(q_pool[i % Q_POOL], out=out_bufs[c],
-                                overlap=True)
+                                overlap=True, q_final=True)
     for _ in range(max(W, 3)):
         g_att.replay()
     torch.cuda.synchronize()
@@ -278,7 +278,7 @@ def run_fc(args, world, rank, local):
             pos[c] += 1
             step_bytes.append(attention_bytes(caches[c], Hq, esz, 4))
             caches[c].attention(q_pool[i % Q_POOL], out=out_bufs[c],
-                                overlap=True)
+                                overlap=True, q_final=True)
     assert [c.k.capacity for c in caches] == caps, "archive grew in capture"
     for _ in range(max(W, 3)):
         g_step.replay()
@@ -317,7 +317,7 @@ def run_fc(args, world, rank, local):
         caches[c].append(dk, dv)
         pos[c] += 1
         e2e_bytes += attention_bytes(caches[c], Hq, esz, 4)
-        caches[c].attention(dq, out=out_bufs[c], overlap=True)
+        caches[c].attention(dq, out=out_bufs[c], overlap=True, q_final=True)
         host_out[c].copy_(out_bufs[c], non_blocking=True)
     ev1.record()
     torch.cuda.synchronize()
@@ -355,7 +355,7 @@ def run_fc(args, world, rank, local):
             "l2": "inputs larger than L2: %d archive copies (%.0f MB) visited "
                   "round-robin" % (copies, copies * arc_bytes / 1e6),
             "timing": "one CUDA-graph replay of K captured steps, CUDA events",
-            "launch": "attention with FC_DECODE_OVERLAP (programmatic dependent launch after the append or the previous attention)",
+            "launch": "attention with FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL (programmatic dependent launch after the append or the previous attention; q is written before the preceding kernel starts)",
             "parallelism": "replicas" if world > 1 else "single",
         },
         "roofline": {

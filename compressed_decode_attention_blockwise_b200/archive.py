@@ -194,13 +194,15 @@ class CodecKVCache:
                   softmax_scale: Optional[float] = None, num_splits: int = 0,
                   fuse_combine: bool = True, portable: bool = False,
                   out_dtype: torch.dtype = torch.float32,
-                  overlap: bool = False) -> torch.Tensor:
+                  overlap: bool = False, q_final: bool = False) -> torch.Tensor:
         """Decode attention of q (B, Hq, 1, D) over archive + tail.
         ``portable`` forces the CUDA-core kernel where the tensor-core kernel
         would apply. ``overlap`` launches it as a programmatic dependent of
         the preceding stream work (FC_DECODE_OVERLAP): valid in a decode loop
         where that work is an append or another attention, not right after a
-        prefill of this cache."""
+        prefill of this cache. ``q_final`` (FC_DECODE_Q_FINAL, with
+        ``overlap``) states that q was final before that preceding kernel
+        started, which lets the kernel compute before it completes."""
         Hq = q.shape[1]
         if out is None:
             out = torch.empty((self.B, Hq, 1, self.D), dtype=out_dtype,
@@ -211,7 +213,7 @@ class CodecKVCache:
             q, self.k.arc, self.v.arc, self.k.tail_desc, self.v.tail_desc,
             out, ws, softmax_scale=0.0 if softmax_scale is None else
             float(softmax_scale), num_splits=ns, fuse_combine=fuse_combine,
-            portable=portable, overlap=overlap)
+            portable=portable, overlap=overlap, q_final=q_final)
         if not fuse_combine:
             _lib.fc_combine(ws, self.B, Hq, self.D, ns, out)
         return out

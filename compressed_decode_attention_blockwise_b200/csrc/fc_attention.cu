@@ -102,7 +102,8 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
   int ns = num_splits;
   if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H, ka->S, int(ka->D));
   if (ns < 1 || ns > kMaxSplits) return FC_ERR_INVALID;
-  if (flags & ~(FC_DECODE_FUSE_COMBINE | FC_DECODE_PORTABLE | FC_DECODE_OVERLAP)) return FC_ERR_INVALID;
+  if (flags & ~(FC_DECODE_FUSE_COMBINE | FC_DECODE_PORTABLE | FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL))
+    return FC_ERR_INVALID;
   const bool fuse_combine = (flags & FC_DECODE_FUSE_COMBINE) != 0;
   if (ka->B > 65535 || ka->H > 65535) return FC_ERR_UNSUPPORTED;
   const bool need_ws = !(fuse_combine && ns == 1);
@@ -156,6 +157,7 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
   a.pacc = need_ws ? reinterpret_cast<float*>(ws + wl.acc) : nullptr;
   a.fuse = fuse_combine ? 1 : 0;
   a.overlap = (flags & FC_DECODE_OVERLAP) ? 1 : 0;
+  a.q_final = (a.overlap && (flags & FC_DECODE_Q_FINAL)) ? 1 : 0;
   a.out = out;
   a.out_dtype = out_dtype;
   a.os_b = out_strides[0];

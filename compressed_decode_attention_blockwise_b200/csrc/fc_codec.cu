@@ -247,6 +247,9 @@ __global__ void __launch_bounds__(256) append_step_kernel(AppendArgs a, BasisF64
   // the older archive blocks now: this kernel writes only the tails and the
   // block it completes, which that attention reads after its dependency wait
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // launched as a programmatic dependent: nothing is read or written before
+  // the preceding work has completed
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t bh_total = int64_t(a.B) * a.H;
@@ -472,9 +475,23 @@ extern "C" int fc_append_step(const void* k_new, const void* v_new, int32_t dtyp
     return dispatch_in(dtype, [&](auto tin) {
       return dispatch_out(ka->coeff_dtype, [&](auto tk) {
         return dispatch_out(va->coeff_dtype, [&](auto tv) {
-          append_step_kernel<decltype(vec)::value, decltype(tin), decltype(tk), decltype(tv)>
-              <<<unsigned(grid), 256, 0, stream>>>(a, basis);
-          return cuda_status(cudaGetLastError());
+          // a programmatic dependent launch whose first action is the
+          // dependency wait: same ordering as a plain launch, but the kernel
+          // (and, through its early trigger, a decode attention queued after
+          // it with FC_DECODE_OVERLAP) can be scheduled while the preceding
+          // kernel drains
+          cudaLaunchConfig_t cfg = {};
+          cfg.gridDim = dim3(unsigned(grid));
+          cfg.blockDim = dim3(256);
+          cfg.stream = stream;
+          cudaLaunchAttribute attr[1];
+          attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+          attr[0].val.programmaticStreamSerializationAllowed = 1;
+          cfg.attrs = attr;
+          cfg.numAttrs = 1;
+          return cuda_status(cudaLaunchKernelEx(
+              &cfg, append_step_kernel<decltype(vec)::value, decltype(tin), decltype(tk), decltype(tv)>, a,
+              basis));
         });
       });
     });

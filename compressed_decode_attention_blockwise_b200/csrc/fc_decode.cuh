@@ -60,6 +60,7 @@ struct DecodeArgs {
   float* pacc;
   int fuse;     // 1: last CTA per kv head writes out
   int overlap;  // 1: launched as a programmatic dependent (FC_DECODE_OVERLAP)
+  int q_final;  // 1: q may be read before the dependency wait (FC_DECODE_Q_FINAL)
   void* out;
   int out_dtype;
   int64_t os_b, os_h;

@@ -307,16 +307,18 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   const int w = warp & 3;                    // warp in the group = TMEM lane quadrant
   const int t = tid & 127;                   // thread in the group
   // group 0 reads the query (thread t = channel d). Without FC_DECODE_OVERLAP
-  // it does so before anything else, so that these loads do not queue behind
-  // the ring fill; with it, after the setup barrier and the dependency wait
-  // (q comes from the preceding work), while the fill has long been running.
+  // (or with FC_DECODE_Q_FINAL) it does so before anything else, so that these
+  // loads do not queue behind the ring fill; otherwise after the setup barrier
+  // and the dependency wait (q comes from the preceding work), while the fill
+  // has long been running.
   float qd[G];
   auto load_q = [&]() {
 #pragma unroll
     for (int g = 0; g < G; ++g)
       qd[g] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
   };
-  if (!producer && grp == 0 && !a.overlap) load_q();
+  const bool q_after_wait = a.overlap && !a.q_final;
+  if (!producer && grp == 0 && !q_after_wait) load_q();
 
   // TMA thread: issues a K load into stage nk % NKS / a V load (codes and both
   // scale rows) into stage nv % NVS
@@ -402,7 +404,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
 
   // ---- group 0: the query as three int8 limbs per head (thread t = channel d)
   if (!producer && grp == 0) {
-    if (a.overlap) {
+    if (q_after_wait) {
       ptx::grid_dep_wait();
       load_q();
     }
@@ -568,6 +570,10 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       const int x = k & 1;
       const int sv = i % NVS;
       const int64_t tile = tile0 + i;
+      // the groups start one after another (group g once group g - 1 has
+      // written its first W), so the first stages are released early and the
+      // rings refill while the other groups work
+      if (k == 0 && grp > 0) waiter.wait(&gbar[10 * (grp - 1) + 4], 0u);
       // ---- K sums of my row, every head
       waiter.wait(&kres[x], uint32_t(k >> 1) & 1u);
       ptx::tc_fence_after();

@@ -62,7 +62,8 @@ enum {
 enum {
   FC_DECODE_FUSE_COMBINE = 1, /* the last CTA of each kv head writes `out` */
   FC_DECODE_PORTABLE = 2,     /* force the portable CUDA-core kernel */
-  FC_DECODE_OVERLAP = 4       /* start before the preceding stream work ends */
+  FC_DECODE_OVERLAP = 4,      /* start before the preceding stream work ends */
+  FC_DECODE_Q_FINAL = 8       /* with OVERLAP: q was final before that work began */
 };
 
 /* Element types. */
@@ -225,6 +226,15 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *              n_blocks - 1 and the tails); a fc_compress_blocks of the same
  *              archive queued just before does not. Pure scheduling: the
  *              results are those of a launch without the flag.
+ *              FC_DECODE_Q_FINAL (with FC_DECODE_OVERLAP): q already held its
+ *              final values when the preceding kernel on the stream began
+ *              executing (it was written by work that completed before that
+ *              kernel started, e.g. a projection followed by a plain
+ *              fc_append_step launch). The kernel then also reads q and
+ *              computes over blocks [0, n_blocks - 1) before the preceding
+ *              work completes; it still waits before block n_blocks - 1,
+ *              the tails, the workspace and `out`. Ignored without
+ *              FC_DECODE_OVERLAP.
  *   workspace       device, >= fc_decode_workspace_bytes(B, Hq, D, splits)
  *                   bytes, 256-byte aligned. Its first 256 + 4*B*Hq bytes
  *                   (status word and tickets) must be zero before the first

@@ -228,7 +228,8 @@ def test_overlap_launch_matches_plain_launch():
             if i == 0:
                 plain.append(c.attention(qs[step]))
             else:
-                over.append(c.attention(qs[step], overlap=True))
+                over.append(c.attention(qs[step], overlap=True,
+                                        q_final=step % 2 == 1))
     torch.cuda.synchronize()
     for a, b in zip(plain, over):
         assert torch.equal(a, b)
@@ -236,12 +237,13 @@ def test_overlap_launch_matches_plain_launch():
     # back to back on alternating caches inside a graph
     outs = [torch.empty_like(plain[0]) for _ in range(4)]
     for i in range(4):
-        caches[i % 2].attention(qs[i], out=outs[i], overlap=True)
+        caches[i % 2].attention(qs[i], out=outs[i], overlap=True, q_final=True)
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         for i in range(4):
-            caches[i % 2].attention(qs[i], out=outs[i], overlap=True)
+            caches[i % 2].attention(qs[i], out=outs[i], overlap=True,
+                                    q_final=i % 2 == 0)
     g.replay()
     torch.cuda.synchronize()
     for i in range(4):
