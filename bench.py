@@ -57,13 +57,19 @@ def dist_env():
     return world, rank, local
 
 
-def init_dist(world, local):
+def init_dist(world, local, backend="nccl"):
+    """One process per GPU; the process group only carries the barrier and
+    the max-over-ranks timing (the replicas exchange no data)."""
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(
-            seconds=120), device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(
+                seconds=120), device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(
+                seconds=120))
 
 
 def barrier(world):
@@ -76,9 +82,18 @@ def max_over_ranks(x: float, world: int) -> float:
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank_step: float, world: int,
+                  max_step_s: float) -> float:
+    """Weak scaling: every rank streams its own replica of the workload, so
+    the job moves world x the per-rank bytes per step in the slowest rank's
+    step time."""
+    return world * bytes_per_rank_step / max_step_s / 1e9
 
 
 def measured_hbm_gbs():
@@ -331,7 +346,7 @@ def run_fc(args, world, rank, local):
 
     peak, peak_kind = measured_hbm_gbs()
     achieved = att_bytes_mean / att_launch_s / 1e9
-    value = world * bytes_per_step / step_s / 1e9
+    value = whole_job_gbs(bytes_per_step, world, step_s)
     res = {
         "metric": "decode-attn archive GB/s (coefficient-domain split-K "
                   "decode step: append + attention)",
@@ -378,7 +393,7 @@ def run_fc(args, world, rank, local):
             "frac_of_peak": round(comp_bytes / comp_s / 1e9 / peak, 4),
         },
         "us_per_layer": round(step_s * 1e6, 3),
-        "e2e": {"value": round(world * e2e_bytes / e2e_s / 1e9, 2),
+        "e2e": {"value": round(whole_job_gbs(e2e_bytes, world, e2e_s), 2),
                 "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "us_per_step": round(e2e_s * 1e6, 2), "steps": n_e2e},
