@@ -158,13 +158,19 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# the files the tensor-core decode-attention kernel is compiled from
+DECODE_SOURCES = ("include/fc.h",
+                  "compressed_decode_attention_blockwise_b200/csrc/fc_internal.cuh",
+                  "compressed_decode_attention_blockwise_b200/csrc/fc_decode.cuh",
+                  "compressed_decode_attention_blockwise_b200/csrc/fc_tc_ptx.cuh",
+                  "compressed_decode_attention_blockwise_b200/csrc/fc_decode_tc.cu")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "compressed_decode_attention_blockwise_b200",
-                        "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, fn), "rb") as f:
-            h.update(fn.encode() + f.read())
+    for rel in DECODE_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(rel.encode() + f.read())
     return h.hexdigest()[:16]
 
 

@@ -225,6 +225,118 @@ __global__ void __launch_bounds__(256) compress_blocks_kernel(CompressArgs a, Ba
   }
 }
 
+// As load_vec, from memory this thread may also write (shared memory): plain
+// loads instead of the read-only path.
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec_plain(const T* p, float (&out)[VEC]) {
+  constexpr int kBytes = VEC * int(sizeof(T));
+  constexpr int kPerWord = 4 / int(sizeof(T));
+  static_assert(kBytes >= 4, "at least one word");
+  if constexpr (kBytes >= 16) {
+#pragma unroll
+    for (int c = 0; c < kBytes / 16; ++c) {
+      const uint4 u = reinterpret_cast<const uint4*>(p)[c];
+      unpack_word<T>(u.x, &out[c * 4 * kPerWord + 0 * kPerWord]);
+      unpack_word<T>(u.y, &out[c * 4 * kPerWord + 1 * kPerWord]);
+      unpack_word<T>(u.z, &out[c * 4 * kPerWord + 2 * kPerWord]);
+      unpack_word<T>(u.w, &out[c * 4 * kPerWord + 3 * kPerWord]);
+    }
+  } else if constexpr (kBytes == 8) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    unpack_word<T>(u.x, &out[0]);
+    unpack_word<T>(u.y, &out[kPerWord]);
+  } else {
+    unpack_word<T>(*reinterpret_cast<const unsigned int*>(p), &out[0]);
+  }
+}
+
+// cp.async of `kBytes` (4, 8, 16 or 32) from global to shared memory, both
+// aligned to min(kBytes, 16)
+template <int kBytes>
+__device__ __forceinline__ void cp_async_row(void* dst, const void* src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  if constexpr (kBytes <= 16) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(d), "l"(src), "n"(kBytes) : "memory");
+  } else {
+    static_assert(kBytes == 32, "row bytes per lane");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + 16),
+                 "l"(static_cast<const char*>(src) + 16)
+                 : "memory");
+  }
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int kStreamWarps = 8;  // warps per CTA of the pipelined compressor
+
+// Prefill compression with the stream kept in flight: each warp walks its
+// blocks (grid stride over (b, h, block)) through an NST-stage ring of
+// shared-memory copies of the blocks' R token rows, NST - 1 blocks ahead of
+// the one it encodes. Lane l copies and later reads only its own VEC channels
+// of every row, so its own cp.async completion orders its reads. The
+// arithmetic is encode_block, unchanged: codes are bitwise those of the
+// unpipelined path and of the append kernel. The first B * H warps also copy
+// their (b, h)'s T mod R remaining tokens into the raw tail.
+template <int VEC, typename TIn, typename TOut, int NST>
+__global__ void __launch_bounds__(kStreamWarps * 32, 2) compress_stream_kernel(CompressArgs a, BasisF64 basis) {
+  extern __shared__ __align__(16) uint8_t csm[];
+  constexpr int kLaneBytes = VEC * int(sizeof(TIn));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t nw = int64_t(gridDim.x) * kStreamWarps;
+  const int64_t w0 = int64_t(blockIdx.x) * kStreamWarps + warp;
+  const int64_t items = int64_t(a.B) * a.H * a.n_full;
+  const int64_t stage_bytes = int64_t(a.R) * a.D * int64_t(sizeof(TIn));
+  uint8_t* ring = csm + warp * NST * stage_bytes;
+  const TIn* x = static_cast<const TIn*>(a.x);
+
+  auto issue = [&](int64_t it, int st) {
+    if (it < items) {
+      const int64_t n = it % a.n_full, bh = it / a.n_full;
+      const int h = int(bh % a.H), b = int(bh / a.H);
+      const TIn* src = x + b * a.xs_b + h * a.xs_h + n * a.R * a.xs_t + lane * VEC;
+      uint8_t* dst = ring + st * stage_bytes + lane * kLaneBytes;
+      for (int t = 0; t < a.R; ++t)
+        cp_async_row<kLaneBytes>(dst + int64_t(t) * a.D * int64_t(sizeof(TIn)), src + t * a.xs_t);
+    }
+    cp_async_commit();  // possibly empty: keeps one group per ring slot
+  };
+
+#pragma unroll
+  for (int s = 0; s < NST - 1; ++s) issue(w0 + s * nw, s);
+  for (int64_t k = 0;; ++k) {
+    const int64_t it = w0 + k * nw;
+    if (it >= items) break;
+    issue(w0 + (k + NST - 1) * nw, int((k + NST - 1) % NST));
+    cp_async_wait<NST - 1>();
+    const int64_t n = it % a.n_full, bh = it / a.n_full;
+    const int h = int(bh % a.H), b = int(bh / a.H);
+    const TIn* rows = reinterpret_cast<const TIn*>(ring + (k % NST) * stage_bytes) + lane * VEC;
+    TOut* blk = static_cast<TOut*>(a.out.coeffs) + b * a.out.cs_b + h * a.out.cs_h +
+                (a.slot0 + n) * a.S * a.D;
+    float* scl = a.out.scales ? a.out.scales + b * a.out.ss_b + h * a.out.ss_h + (a.slot0 + n) * a.S
+                              : nullptr;
+    encode_block<TOut, VEC>([&](int t, float (&xf)[VEC]) { load_vec_plain<TIn, VEC>(rows + t * a.D, xf); },
+                            a.R, a.S, a.D, lane, basis, blk, scl);
+  }
+  cp_async_wait<0>();
+  if (a.tail != nullptr && w0 < int64_t(a.B) * a.H) {
+    const int h = int(w0 % a.H), b = int(w0 / a.H);
+    const TIn* src = x + b * a.xs_b + h * a.xs_h + a.n_full * a.R * a.xs_t + lane * VEC;
+    TIn* dst = static_cast<TIn*>(a.tail) + b * a.ts_b + h * a.ts_h + lane * VEC;
+    for (int i = 0; i < a.n_rem; ++i) {
+      float xv[VEC];
+      load_vec<TIn, VEC>(src + i * a.xs_t, xv);
+      store_row<TIn, VEC>(dst + int64_t(i) * a.D, xv);
+    }
+  }
+}
+
 struct AppendStream {
   const void* src;  // new token (B, H, 1, D)
   int64_t src_b, src_h;
@@ -405,12 +517,37 @@ extern "C" int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t*
   const int64_t warps = arc->B * arc->H * n_full + (copy_tail ? arc->B * arc->H : 0);
   const int64_t grid = (warps + 7) / 8;
   if (grid > 0x7fffffffLL) return FC_ERR_UNSUPPORTED;
+  // the pipelined compressor when a lane's share of a row is a whole word and
+  // its ring fits (three stages, two CTAs per SM; else two stages); the
+  // direct-load kernel otherwise
+  const int64_t stage_bytes = int64_t(arc->R) * arc->D * esz;
+  const int lane_bytes = int(arc->D / 32) * esz;
+  const int nst = 3 * kStreamWarps * stage_bytes <= 100 * 1024 ? 3
+                  : 2 * kStreamWarps * stage_bytes <= 200 * 1024 ? 2 : 0;
+  const bool pipelined = nst > 0 && lane_bytes >= 4 && n_full > 0;
   st = dispatch_vec(a.D, [&](auto vec) {
     return dispatch_in(x_dtype, [&](auto tin) {
       return dispatch_out(arc->coeff_dtype, [&](auto tout) {
         using TIn = decltype(tin);
         using TOut = decltype(tout);
-        compress_blocks_kernel<decltype(vec)::value, TIn, TOut><<<unsigned(grid), 256, 0, stream>>>(a, basis);
+        constexpr int VEC = decltype(vec)::value;
+        if constexpr (VEC * sizeof(TIn) >= 4) {
+          if (pipelined) {
+            const size_t smem = size_t(kStreamWarps) * nst * stage_bytes;
+            const int64_t need = (arc->B * arc->H * n_full + kStreamWarps - 1) / kStreamWarps;
+            const int64_t cap = int64_t(sm_count()) * (nst == 3 ? 2 : 1);  // one resident wave
+            const int64_t g = need < cap ? need : cap;
+            const int64_t g_tail = (copy_tail ? (arc->B * arc->H + kStreamWarps - 1) / kStreamWarps : 0);
+            const unsigned grid_p = unsigned(g > g_tail ? g : g_tail);
+            auto kern = nst == 3 ? compress_stream_kernel<VEC, TIn, TOut, 3> : compress_stream_kernel<VEC, TIn, TOut, 2>;
+            if (smem > 48 * 1024 &&
+                cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+              return int(FC_ERR_CUDA);
+            kern<<<grid_p, kStreamWarps * 32, smem, stream>>>(a, basis);
+            return cuda_status(cudaGetLastError());
+          }
+        }
+        compress_blocks_kernel<VEC, TIn, TOut><<<unsigned(grid), 256, 0, stream>>>(a, basis);
         return cuda_status(cudaGetLastError());
       });
     });
