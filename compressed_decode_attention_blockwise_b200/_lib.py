@@ -42,7 +42,7 @@ EXPORTS = (
     "fc_compress_blocks", "fc_append_step", "fc_archive_copy_prefix",
     "fc_decode_plan", "fc_decode_workspace_bytes", "fc_decode_attention",
     "fc_combine", "fc_decode_attention_noalloc", "fc_workspace_status",
-    "fc_storage_bytes", "fc_status_string",
+    "fc_storage_bytes", "fc_status_string", "fc_decode_step",
 )
 
 
@@ -104,6 +104,10 @@ def load() -> ctypes.CDLL:
                                                PT, ctypes.c_float, I32, I32,
                                                P, ctypes.c_size_t, P, I32,
                                                PI64, P]),
+        "fc_decode_step": (ctypes.c_int, [P, I32, PI64, I64, P, P, I32, PI64,
+                                          PI64, PA, PA, PT, PT,
+                                          ctypes.c_float, I32, I32, P,
+                                          ctypes.c_size_t, P, I32, PI64, P]),
         "fc_combine": (ctypes.c_int, [P, ctypes.c_size_t, I64, I64, I64, I32,
                                       P, I32, PI64, P]),
         "fc_decode_attention_noalloc": (ctypes.c_int, [P, I32, PI64, I64, PA,
@@ -231,6 +235,32 @@ def fc_decode_attention(q: torch.Tensor, ka: FcArchive, va: FcArchive,
         ws_ptr, ws_bytes, _ptr(out), dtype_code(out.dtype), _strides4(out),
         _stream(stream, q))
     _check(st, "fc_decode_attention")
+
+
+def fc_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                   ka: FcArchive, va: FcArchive, kt: FcTail, vt: FcTail,
+                   out: torch.Tensor, workspace: Optional[torch.Tensor],
+                   softmax_scale: float = 0.0, num_splits: int = 0,
+                   fuse_combine: bool = True, portable: bool = False,
+                   overlap: bool = False, q_final: bool = False,
+                   stream=None) -> None:
+    if k_new.dtype != v_new.dtype:
+        raise ValueError("k_new and v_new must share a dtype")
+    ws_ptr = _ptr(workspace)
+    ws_bytes = 0 if workspace is None else workspace.numel() * \
+        workspace.element_size()
+    flags = (FC_DECODE_FUSE_COMBINE if fuse_combine else 0) | \
+        (FC_DECODE_PORTABLE if portable else 0) | \
+        (FC_DECODE_OVERLAP if overlap else 0) | \
+        (FC_DECODE_Q_FINAL if q_final else 0)
+    st = load().fc_decode_step(
+        _ptr(q), dtype_code(q.dtype), _strides4(q), q.shape[1],
+        _ptr(k_new), _ptr(v_new), dtype_code(k_new.dtype), _strides4(k_new),
+        _strides4(v_new), ctypes.byref(ka), ctypes.byref(va),
+        ctypes.byref(kt), ctypes.byref(vt), float(softmax_scale),
+        int(num_splits), flags, ws_ptr, ws_bytes, _ptr(out),
+        dtype_code(out.dtype), _strides4(out), _stream(stream, q))
+    _check(st, "fc_decode_step")
 
 
 def fc_decode_attention_noalloc(q: torch.Tensor, ka: FcArchive, va: FcArchive,

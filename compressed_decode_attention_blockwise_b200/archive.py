@@ -144,6 +144,8 @@ class CodecKVCache:
                              capacity)
         self.device = self.k.device
         self._ws: Optional[torch.Tensor] = None
+        self._plans: dict = {}      # (Hq, n_blocks) -> split count
+        self._ws_need: dict = {}    # (Hq, splits) -> workspace bytes
 
     @property
     def seq_len(self) -> int:
@@ -179,12 +181,49 @@ class CodecKVCache:
         _lib.fc_append_step(k_new, v_new, self.k.arc, self.v.arc,
                             self.k.tail_desc, self.v.tail_desc)
 
+    def step(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+             out: Optional[torch.Tensor] = None,
+             softmax_scale: Optional[float] = None, num_splits: int = 0,
+             fuse_combine: bool = True, portable: bool = False,
+             out_dtype: torch.dtype = torch.float32, overlap: bool = False,
+             q_final: bool = False) -> torch.Tensor:
+        """One decode step: append the (B, Hk, 1, D) token to both streams,
+        then attend q over the updated cache (fc_decode_step: one launch on
+        the tensor-core path). Flags as in ``attention``."""
+        if self.k.tail_len + 1 == self.R:
+            self._grow_to(self.k.n_blocks + 1)
+        Hq = q.shape[1]
+        if out is None:
+            out = torch.empty((self.B, Hq, 1, self.D), dtype=out_dtype,
+                              device=q.device)
+        ns = num_splits or self.num_splits(Hq)
+        ws = self.workspace(Hq, ns)
+        _lib.fc_decode_step(
+            q, k_new, v_new, self.k.arc, self.v.arc, self.k.tail_desc,
+            self.v.tail_desc, out, ws, softmax_scale=0.0 if softmax_scale is
+            None else float(softmax_scale), num_splits=ns,
+            fuse_combine=fuse_combine, portable=portable, overlap=overlap,
+            q_final=q_final)
+        if not fuse_combine:
+            _lib.fc_combine(ws, self.B, Hq, self.D, ns, out)
+        return out
+
     # -- attention -----------------------------------------------------------
     def num_splits(self, Hq: int) -> int:
-        return _lib.fc_decode_plan(self.k.arc, self.k.tail_desc, Hq)
+        key = (Hq, self.k.n_blocks)     # the plan depends on nothing else
+        ns = self._plans.get(key)
+        if ns is None:
+            ns = _lib.fc_decode_plan(self.k.arc, self.k.tail_desc, Hq)
+            self._plans[key] = ns
+        return ns
 
     def workspace(self, Hq: int, num_splits: int) -> torch.Tensor:
-        need = _lib.fc_decode_workspace_bytes(self.B, Hq, self.D, num_splits)
+        key = (Hq, num_splits)
+        need = self._ws_need.get(key)
+        if need is None:
+            need = _lib.fc_decode_workspace_bytes(self.B, Hq, self.D,
+                                                  num_splits)
+            self._ws_need[key] = need
         if self._ws is None or self._ws.numel() < need:
             self._ws = torch.zeros(need, dtype=torch.uint8,
                                    device=self.device)

@@ -65,12 +65,17 @@ extern "C" int fc_decode_plan(const fc_archive* ka, const fc_tail* kt, int64_t H
   return FC_OK;
 }
 
-extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides,
-                                   int64_t Hq, const fc_archive* ka, const fc_archive* va,
-                                   const fc_tail* kt, const fc_tail* vt, float softmax_scale,
-                                   int32_t num_splits, int32_t flags, void* workspace,
-                                   size_t workspace_bytes, void* out, int32_t out_dtype,
-                                   const int64_t* out_strides, fc_stream stream) {
+namespace fc {
+namespace {
+
+// Validation and argument set-up shared by fc_decode_attention and
+// fc_decode_step. `extra_token`: a new token joins the softmax (the step), so
+// an empty archive with an empty tail is valid.
+int prepare_decode(const void* q, int32_t q_dtype, const int64_t* q_strides, int64_t Hq,
+                   const fc_archive* ka, const fc_archive* va, const fc_tail* kt, const fc_tail* vt,
+                   float softmax_scale, int32_t num_splits, int32_t flags, void* workspace,
+                   size_t workspace_bytes, void* out, int32_t out_dtype, const int64_t* out_strides,
+                   bool extra_token, DecodeArgs* ap) {
   int st = check_archive(ka);
   if (st != FC_OK) return st;
   st = check_archive(va);
@@ -98,7 +103,7 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
     nr = kt->len;
     t_dtype = kt->dtype;
   }
-  if (ka->n_blocks == 0 && nr == 0) return FC_ERR_INVALID;
+  if (ka->n_blocks == 0 && nr == 0 && !extra_token) return FC_ERR_INVALID;
   int ns = num_splits;
   if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H, ka->S, int(ka->D));
   if (ns < 1 || ns > kMaxSplits) return FC_ERR_INVALID;
@@ -113,7 +118,7 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
         workspace_bytes < wl.total)
       return FC_ERR_INVALID;
   }
-  DecodeArgs a;
+  DecodeArgs a = {};
   a.q = q;
   a.q_dtype = q_dtype;
   a.qs_b = q_strides[0];
@@ -162,9 +167,16 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
   a.out_dtype = out_dtype;
   a.os_b = out_strides[0];
   a.os_h = out_strides[1];
+  a.step = 0;
+  *ap = a;
+  return FC_OK;
+}
+
+int launch_prepared(const DecodeArgs& a, const fc_archive* ka, const fc_archive* va, int32_t flags,
+                    cudaStream_t stream) {
   Basis basis;
   make_basis(ka->R, ka->S, &basis);
-  if (!(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, int(G)))
+  if (!(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, a.G))
     return launch_decode_tc(a, ka, va, basis, stream);
   const int kd = ka->coeff_dtype, vd = va->coeff_dtype;
   if (kd == FC_DTYPE_I8 && vd == FC_DTYPE_I8) return launch_decode_generic<int8_t, int8_t>(a, basis, stream);
@@ -175,6 +187,87 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
     return launch_decode_generic<__nv_bfloat16, __nv_bfloat16>(a, basis, stream);
   if (kd == FC_DTYPE_F32 && vd == FC_DTYPE_F32) return launch_decode_generic<float, float>(a, basis, stream);
   return FC_ERR_UNSUPPORTED;
+}
+
+StreamOut out_of(const fc_archive* a) {
+  StreamOut o;
+  o.coeffs = a->coeffs;
+  o.scales = a->scales;
+  o.cs_b = a->coeff_stride_b;
+  o.cs_h = a->coeff_stride_h;
+  o.ss_b = a->scale_stride_b;
+  o.ss_h = a->scale_stride_h;
+  return o;
+}
+
+}  // namespace
+}  // namespace fc
+
+extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides,
+                                   int64_t Hq, const fc_archive* ka, const fc_archive* va,
+                                   const fc_tail* kt, const fc_tail* vt, float softmax_scale,
+                                   int32_t num_splits, int32_t flags, void* workspace,
+                                   size_t workspace_bytes, void* out, int32_t out_dtype,
+                                   const int64_t* out_strides, fc_stream stream) {
+  DecodeArgs a;
+  const int st = prepare_decode(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
+                                workspace, workspace_bytes, out, out_dtype, out_strides, false, &a);
+  if (st != FC_OK) return st;
+  return launch_prepared(a, ka, va, flags, stream);
+}
+
+extern "C" int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int64_t Hq,
+                              const void* k_new, const void* v_new, int32_t new_dtype,
+                              const int64_t* k_strides, const int64_t* v_strides, fc_archive* ka,
+                              fc_archive* va, fc_tail* kt, fc_tail* vt, float softmax_scale,
+                              int32_t num_splits, int32_t flags, void* workspace,
+                              size_t workspace_bytes, void* out, int32_t out_dtype,
+                              const int64_t* out_strides, fc_stream stream) {
+  if (!k_new || !v_new || !k_strides || !v_strides || !kt || !vt || !kt->data || !vt->data)
+    return FC_ERR_INVALID;
+  DecodeArgs a;
+  int st = prepare_decode(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
+                          workspace, workspace_bytes, out, out_dtype, out_strides, true, &a);
+  if (st != FC_OK) return st;
+  const bool fused = !(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, a.G) &&
+                     new_dtype == kt->dtype && k_strides[3] == 1 && v_strides[3] == 1 &&
+                     aligned16(k_new) && aligned16(v_new) && k_strides[0] >= 0 && k_strides[1] >= 0 &&
+                     v_strides[0] >= 0 && v_strides[1] >= 0;
+  if (!fused) {
+    // two launches: the append, then the attention over the updated stream
+    st = fc_append_step(k_new, v_new, new_dtype, k_strides, v_strides, ka, va, kt, vt, stream);
+    if (st != FC_OK) return st;
+    return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
+                               workspace, workspace_bytes, out, out_dtype, out_strides, stream);
+  }
+  const int esz = dtype_size(new_dtype);
+  if ((k_strides[0] * esz) % 16 || (k_strides[1] * esz) % 16 || (v_strides[0] * esz) % 16 ||
+      (v_strides[1] * esz) % 16)
+    return FC_ERR_INVALID;
+  const bool complete = kt->len + 1 == ka->R;
+  if (complete && (ka->n_blocks >= ka->capacity || va->n_blocks >= va->capacity)) return FC_ERR_CAPACITY;
+  a.step = complete ? 2 : 1;
+  a.kn = k_new;
+  a.vn = v_new;
+  a.kns_b = k_strides[0];
+  a.kns_h = k_strides[1];
+  a.vns_b = v_strides[0];
+  a.vns_h = v_strides[1];
+  a.kout = out_of(ka);
+  a.vout = out_of(va);
+  a.new_slot = ka->n_blocks;
+  st = launch_prepared(a, ka, va, flags, stream);
+  if (st != FC_OK) return st;
+  if (complete) {
+    ka->n_blocks += 1;
+    va->n_blocks += 1;
+    kt->len = 0;
+    vt->len = 0;
+  } else {
+    kt->len += 1;
+    vt->len += 1;
+  }
+  return FC_OK;
 }
 
 extern "C" int fc_combine(const void* workspace, size_t workspace_bytes, int64_t B, int64_t Hq,

@@ -24,164 +24,10 @@
 // token is bitwise identical to one built in a single call.
 #include <type_traits>
 
-#include "fc_internal.cuh"
+#include "fc_encode.cuh"
 
 namespace fc {
 namespace {
-
-struct StreamOut {
-  void* coeffs;
-  float* scales;
-  int64_t cs_b, cs_h;  // coefficient element strides
-  int64_t ss_b, ss_h;  // scale element strides
-};
-
-constexpr int kJC = 4;  // frequencies per pass over a block's rows
-
-__device__ __forceinline__ double warp_max_d(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-template <int VEC>
-__device__ __forceinline__ void store_codes(int8_t* p, const int (&code)[VEC]) {
-  if constexpr (VEC == 1) {
-    *p = static_cast<int8_t>(code[0]);
-  } else if constexpr (VEC == 2) {
-    const uint32_t w = (uint32_t(code[0]) & 0xffu) | ((uint32_t(code[1]) & 0xffu) << 8);
-    *reinterpret_cast<unsigned short*>(p) = static_cast<unsigned short>(w);
-  } else {
-    uint32_t w[VEC / 4];
-#pragma unroll
-    for (int i = 0; i < VEC / 4; ++i) {
-      w[i] = (uint32_t(code[4 * i]) & 0xffu) | ((uint32_t(code[4 * i + 1]) & 0xffu) << 8) |
-             ((uint32_t(code[4 * i + 2]) & 0xffu) << 16) | ((uint32_t(code[4 * i + 3]) & 0xffu) << 24);
-    }
-    if constexpr (VEC == 4) {
-      *reinterpret_cast<uint32_t*>(p) = w[0];
-    } else {
-      *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
-    }
-  }
-}
-
-template <typename T, int VEC>
-__device__ __forceinline__ void store_row(T* p, const float (&x)[VEC]) {
-  if constexpr (std::is_same_v<T, float>) {
-    if constexpr (VEC % 4 == 0) {
-#pragma unroll
-      for (int i = 0; i < VEC / 4; ++i)
-        reinterpret_cast<float4*>(p)[i] = make_float4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
-    } else if constexpr (VEC == 2) {
-      *reinterpret_cast<float2*>(p) = make_float2(x[0], x[1]);
-    } else {
-      p[0] = x[0];
-    }
-  } else {
-    static_assert(std::is_same_v<T, __nv_bfloat16>, "bf16 or f32 rows");
-    if constexpr (VEC == 1) {
-      p[0] = __float2bfloat16_rn(x[0]);
-    } else {
-      uint32_t w[VEC / 2];
-#pragma unroll
-      for (int i = 0; i < VEC / 2; ++i) {
-        const __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-        w[i] = *reinterpret_cast<const uint32_t*>(&h);
-      }
-      if constexpr (VEC == 2) {
-        *reinterpret_cast<uint32_t*>(p) = w[0];
-      } else if constexpr (VEC == 4) {
-        *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
-      } else {
-        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-  }
-}
-
-template <int VEC>
-__device__ __forceinline__ void store_bf16_row(__nv_bfloat16* p, const __nv_bfloat16 (&h)[VEC]) {
-  if constexpr (VEC == 1) {
-    p[0] = h[0];
-  } else {
-    uint32_t w[VEC / 2];
-#pragma unroll
-    for (int i = 0; i < VEC / 2; ++i)
-      w[i] = uint32_t(__bfloat16_as_ushort(h[2 * i])) | (uint32_t(__bfloat16_as_ushort(h[2 * i + 1])) << 16);
-    if constexpr (VEC == 2) {
-      *reinterpret_cast<uint32_t*>(p) = w[0];
-    } else if constexpr (VEC == 4) {
-      *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
-    } else {
-      *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  }
-}
-
-// Quantises (int8) or rounds (bf16 / f32) one coefficient row held in fp64
-// and stores it at `row` (D elements; lane owns VEC) and, for int8, its scale.
-template <typename TOut, int VEC>
-__device__ __forceinline__ void store_coeff_row(const double (&c)[VEC], int lane, TOut* row,
-                                                float* scl) {
-  if constexpr (std::is_same_v<TOut, int8_t>) {
-    double amax = 0.0;
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) amax = fmax(amax, fabs(c[v]));
-    amax = warp_max_d(amax);
-    const double scale = amax / 127.0;
-    const double inv = amax > 0.0 ? 1.0 / scale : 0.0;
-    int code[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) code[v] = max(-127, min(127, __double2int_rn(c[v] * inv)));
-    store_codes<VEC>(row + lane * VEC, code);
-    if (lane == 0) *scl = __double2float_rn(scale);
-  } else if constexpr (std::is_same_v<TOut, float>) {
-    float x[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) x[v] = __double2float_rn(c[v]);
-    store_row<float, VEC>(row + lane * VEC, x);
-  } else {
-    // direct fp64 -> bf16 rounding, packed in pairs
-    __nv_bfloat16 hb[VEC];
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) hb[v] = __double2bfloat16(c[v]);
-    store_bf16_row<VEC>(row + lane * VEC, hb);
-  }
-}
-
-// Encodes the S kept frequencies of one block whose R token rows come from
-// `row_at(t, xf)` (VEC floats of row t for this lane), kJC frequencies per
-// pass, and stores them at `blk` (S x D elements) / `scl` (S floats).
-template <typename TOut, int VEC, typename RowAt>
-__device__ __forceinline__ void encode_block(RowAt&& row_at, int R, int S, int D, int lane,
-                                             const BasisF64& basis, TOut* blk, float* scl) {
-  for (int j0 = 0; j0 < S; j0 += kJC) {
-    double c[kJC][VEC];
-#pragma unroll
-    for (int jj = 0; jj < kJC; ++jj)
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) c[jj][v] = 0.0;
-#pragma unroll 4
-    for (int t = 0; t < R; ++t) {
-      float xf[VEC];
-      row_at(t, xf);
-#pragma unroll
-      for (int jj = 0; jj < kJC; ++jj) {
-        if (j0 + jj < S) {
-          const double m = basis.m[j0 + jj][t];
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) c[jj][v] = fma(m, double(xf[v]), c[jj][v]);
-        }
-      }
-    }
-#pragma unroll
-    for (int jj = 0; jj < kJC; ++jj) {
-      const int j = j0 + jj;
-      if (j < S) store_coeff_row<TOut, VEC>(c[jj], lane, blk + int64_t(j) * D, scl ? scl + j : nullptr);
-    }
-  }
-}
 
 struct CompressArgs {
   const void* x;

@@ -26,7 +26,7 @@
 
 #include <type_traits>
 
-#include "fc_internal.cuh"
+#include "fc_encode.cuh"
 
 namespace fc {
 
@@ -61,6 +61,15 @@ struct DecodeArgs {
   int fuse;     // 1: last CTA per kv head writes out
   int overlap;  // 1: launched as a programmatic dependent (FC_DECODE_OVERLAP)
   int q_final;  // 1: q may be read before the dependency wait (FC_DECODE_Q_FINAL)
+  // fused decode step (fc_decode_step): 0 plain attention; 1 the new token
+  // joins the tail at row nr; 2 it completes the block formed by the nr = R - 1
+  // tail rows, which is encoded into archive slot new_slot (= nb)
+  int step;
+  const void* kn;
+  const void* vn;
+  int64_t kns_b, kns_h, vns_b, vns_h;
+  StreamOut kout, vout;
+  int64_t new_slot;
   void* out;
   int out_dtype;
   int64_t os_b, os_h;

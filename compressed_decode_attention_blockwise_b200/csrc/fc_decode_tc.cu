@@ -107,12 +107,28 @@ struct Cfg {
   static_assert((NG * G * (kD + 5) + 4) * 4 <= int(NKS * kTileBytes), "merge scratch");
   static_assert(4 * NP * NG <= 512, "TMEM allocation");
   static_assert(NI * R <= 32, "logits per lane");
+  static_assert(R * HPG <= XW, "tail batch scratch");
 };
 
 struct TcArgs {
   DecodeArgs d;
   int tiles_per_head;
   int chunk_tiles;
+};
+
+// The DCT basis rows the kernel needs, sized for its (S, R): fp32 for the
+// attention arithmetic, fp64 for encoding a block in the fused decode step
+// (the same values as the codec's). A small parameter block keeps launches
+// cheap.
+template <int S, int R>
+struct TcBasis {
+  float m[S][R];
+  double m64[S][R];
+};
+
+template <int S, int R>
+struct Basis64View {  // encode_block indexes basis.m[j][t]
+  const double (&m)[S][R];
 };
 
 __device__ __forceinline__ float pow2i(int e) {
@@ -252,6 +268,51 @@ __device__ __forceinline__ void group_sum(float (&v)[N], float* red, int wq, int
   ptx::named_bar_sync(bar_id, 128);
 }
 
+// dst[di] = src[si] for a runtime dtype (FC_DTYPE_F32 or FC_DTYPE_BF16), bits copied
+__device__ __forceinline__ void copy_elem(const void* dst, int64_t di, const void* src, int64_t si, int dtype) {
+  if (dtype == FC_DTYPE_F32)
+    const_cast<float*>(static_cast<const float*>(dst))[di] = static_cast<const float*>(src)[si];
+  else
+    const_cast<unsigned short*>(static_cast<const unsigned short*>(dst))[di] =
+        static_cast<const unsigned short*>(src)[si];
+}
+
+// Fused decode step: the block completed by the new token (rows 0..R-2 from
+// the tail, row R-1 the token) encoded by one warp into archive slot new_slot
+// of K (which = 0) or V (which = 1), exactly as the append kernel does.
+template <int S, int R>
+__device__ __forceinline__ void encode_new_block(const DecodeArgs& a, int which, int lane,
+                                                 const TcBasis<S, R>& basis, int b, int h) {
+  const Basis64View<S, R> basis64{basis.m64};
+  constexpr int VEC = kD / 32;
+  const StreamOut& o = which ? a.vout : a.kout;
+  const void* tail = which ? a.vt : a.kt;
+  const int64_t tb = which ? a.vts_b : a.kts_b, th = which ? a.vts_h : a.kts_h;
+  const void* nw = which ? a.vn : a.kn;
+  const int64_t nb_ = which ? a.vns_b : a.kns_b, nh = which ? a.vns_h : a.kns_h;
+  int8_t* blk = static_cast<int8_t*>(o.coeffs) + b * o.cs_b + h * o.cs_h + a.new_slot * a.S * kD;
+  float* scl = o.scales + b * o.ss_b + h * o.ss_h + a.new_slot * a.S;
+  auto run = [&](auto tag) {
+    using T = decltype(tag);
+    const T* trow = static_cast<const T*>(tail) + b * tb + h * th + lane * VEC;
+    float xn[VEC];
+    load_vec<T, VEC>(static_cast<const T*>(nw) + b * nb_ + h * nh + lane * VEC, xn);
+    auto row_at = [&](int t, float (&xf)[VEC]) {
+      if (t < R - 1) {
+        load_vec<T, VEC>(trow + int64_t(t) * kD, xf);
+      } else {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) xf[v] = xn[v];
+      }
+    };
+    encode_block<int8_t, VEC>(row_at, R, a.S, kD, lane, basis64, blk, scl);
+  };
+  if (a.t_dtype == FC_DTYPE_F32)
+    run(float(0));
+  else
+    run(__nv_bfloat16());
+}
+
 template <int NP>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) {
   if constexpr (NP == 16) {
@@ -266,7 +327,7 @@ template <int G, int S, int TPT>
 __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
-                     const TcArgs ta, const Basis basis) {
+                     const TcArgs ta, const TcBasis<S, S * TPT> basis) {
   using C = Cfg<G, S, TPT>;
   constexpr int R = C::R, NP = C::NP, NI = C::NI, NKS = C::NKS, NVS = C::NVS, XP = C::XP;
   constexpr int NG = C::NG;
@@ -745,8 +806,18 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       Ah[y] = As;
     }
     const bool active = grp < G;  // uniform per group
-    // raw tail tokens (last chunk)
-    if (active && c == a.ns - 1 && a.nr > 0) {
+    const bool last_chunk = c == a.ns - 1;
+    // fused decode step whose token completes a block: warps 0 and 1 of group
+    // 0 encode it (tail rows 0..R-2 and the new token) into archive slot
+    // new_slot with the codec's own device code, so the archive is bitwise
+    // what fc_append_step writes; the barrier publishes codes and scales to
+    // the CTA
+    if (last_chunk && a.step == 2) {
+      if (grp == 0 && w < 2) encode_new_block<S, S * TPT>(a, w, lane, basis, b, h);
+      ptx::named_bar_sync(kFinBar, 128 * NG);
+    }
+    // raw tail tokens, then the step's new token or block (last chunk)
+    if (active && last_chunk && (a.nr > 0 || a.step != 0)) {
       float* red2 = reinterpret_cast<float*>(sm + C::xs) + grp * 4 * C::XW;
       float qh[HPG];
 #pragma unroll
@@ -754,21 +825,128 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
         const int g = min(grp + NG * y, G - 1);
         qh[y] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
       }
-      for (int tt = 0; tt < a.nr; ++tt) {
-        const float kd = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, a.t_dtype);
-        const float vd = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, a.t_dtype);
-        float lgt[HPG];
+      // the raw tokens of the tail, and the step's new token, in one batch:
+      // one reduction over the group for every logit, then one online-softmax
+      // update (thread t = channel d)
+      const int n_raw = a.step == 2 ? 0 : a.nr;  // a completed block is folded coded
+      const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
+      constexpr int kTok = S * TPT;  // at most R tokens: R - 1 tail rows + the new one
+      if (n_tok > 0) {
+        float kv[kTok], vv[kTok];
 #pragma unroll
-        for (int y = 0; y < HPG; ++y) lgt[y] = qh[y] * kd;
-        group_sum<HPG>(lgt, red2, w, lane, 1 + grp);
+        for (int tt = 0; tt < kTok; ++tt) {
+          kv[tt] = 0.f;
+          vv[tt] = 0.f;
+          if (tt < n_raw) {
+            kv[tt] = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, a.t_dtype);
+            vv[tt] = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, a.t_dtype);
+          } else if (tt == n_raw && a.step == 1) {
+            kv[tt] = load_any(a.kn, b * a.kns_b + h * a.kns_h + t, a.t_dtype);
+            vv[tt] = load_any(a.vn, b * a.vns_b + h * a.vns_h + t, a.t_dtype);
+          }
+        }
+        float lgt[kTok][HPG];
+#pragma unroll
+        for (int tt = 0; tt < kTok; ++tt)
+#pragma unroll
+          for (int y = 0; y < HPG; ++y) lgt[tt][y] = tt < n_tok ? warp_sum(qh[y] * kv[tt]) : 0.f;
+        if (lane == 0) {
+#pragma unroll
+          for (int tt = 0; tt < kTok; ++tt)
+#pragma unroll
+            for (int y = 0; y < HPG; ++y) red2[(w * kTok + tt) * HPG + y] = lgt[tt][y];
+        }
+        ptx::named_bar_sync(1 + grp, 128);
+#pragma unroll
+        for (int tt = 0; tt < kTok; ++tt)
+#pragma unroll
+          for (int y = 0; y < HPG; ++y)
+            lgt[tt][y] = red2[(0 * kTok + tt) * HPG + y] + red2[(1 * kTok + tt) * HPG + y] +
+                         red2[(2 * kTok + tt) * HPG + y] + red2[(3 * kTok + tt) * HPG + y];
+        ptx::named_bar_sync(1 + grp, 128);  // red2 is reused below
 #pragma unroll
         for (int y = 0; y < HPG; ++y) {
-          const float mn = fmaxf(Mh[y], lgt[y]);
+          float mn = Mh[y];
+#pragma unroll
+          for (int tt = 0; tt < kTok; ++tt)
+            if (tt < n_tok) mn = fmaxf(mn, lgt[tt][y]);
           const float al = ptx::ex2(Mh[y] - mn);
-          const float p = ptx::ex2(lgt[y] - mn);
-          Ah[y] = fmaf(Ah[y], al, p * vd);
-          Lh[y] = fmaf(Lh[y], al, p);
+          float ps = 0.f, add = 0.f;
+#pragma unroll
+          for (int tt = 0; tt < kTok; ++tt) {
+            if (tt < n_tok) {
+              const float p = ptx::ex2(lgt[tt][y] - mn);
+              ps += p;
+              add = fmaf(p, vv[tt], add);
+            }
+          }
+          Ah[y] = fmaf(Ah[y], al, add);
+          Lh[y] = fmaf(Lh[y], al, ps);
           Mh[y] = mn;
+        }
+      }
+      if (a.step == 1 && grp == 0) {  // the token joins the tail at row nr
+        copy_elem(a.kt, b * a.kts_b + h * a.kts_h + int64_t(a.nr) * kD + t, a.kn,
+                  b * a.kns_b + h * a.kns_h + t, a.t_dtype);
+        copy_elem(a.vt, b * a.vts_b + h * a.vts_h + int64_t(a.nr) * kD + t, a.vn,
+                  b * a.vns_b + h * a.vns_h + t, a.t_dtype);
+      }
+      if (a.step == 2) {
+        // the new block in the coefficient domain, as a tile row set would be:
+        // s_j = scale_k,j C_k[j] . q, logits = A s, p, w = p A, acc += w scale_v C_v
+        const StreamOut& ko = a.kout;
+        const StreamOut& vo = a.vout;
+        // (written by this CTA before the barrier above: read through L2)
+        const signed char* kc = static_cast<const signed char*>(ko.coeffs) + b * ko.cs_b + h * ko.cs_h + a.new_slot * S * kD;
+        const signed char* vc = static_cast<const signed char*>(vo.coeffs) + b * vo.cs_b + h * vo.cs_h + a.new_slot * S * kD;
+        const float* ksp = ko.scales + b * ko.ss_b + h * ko.ss_h + a.new_slot * S;
+        const float* vsp = vo.scales + b * vo.ss_b + h * vo.ss_h + a.new_slot * S;
+        float ksc[S], vsc[S];
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+          ksc[j] = __ldcg(ksp + j);
+          vsc[j] = __ldcg(vsp + j);
+        }
+        float sj[S * HPG];
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+          const float kv = float(__ldcg(kc + j * kD + t));
+#pragma unroll
+          for (int y = 0; y < HPG; ++y) sj[j * HPG + y] = kv * qh[y];
+        }
+        group_sum<S * HPG>(sj, red2, w, lane, 1 + grp);
+        float vcode[S];
+#pragma unroll
+        for (int j = 0; j < S; ++j) vcode[j] = float(__ldcg(vc + j * kD + t));
+#pragma unroll
+        for (int y = 0; y < HPG; ++y) {
+          float lg[S * TPT];
+          float mx = Mh[y];
+#pragma unroll
+          for (int tk = 0; tk < S * TPT; ++tk) {
+            float v = 0.f;
+#pragma unroll
+            for (int j = 0; j < S; ++j) v = fmaf(basis.m[j][tk], sj[j * HPG + y] * ksc[j], v);
+            lg[tk] = v;
+            mx = fmaxf(mx, v);
+          }
+          const float al = ptx::ex2(Mh[y] - mx);
+          float ps = 0.f, wv[S];
+#pragma unroll
+          for (int j = 0; j < S; ++j) wv[j] = 0.f;
+#pragma unroll
+          for (int tk = 0; tk < S * TPT; ++tk) {
+            const float p = ptx::ex2(lg[tk] - mx);
+            ps += p;
+#pragma unroll
+            for (int j = 0; j < S; ++j) wv[j] = fmaf(p, basis.m[j][tk], wv[j]);
+          }
+          float add = 0.f;
+#pragma unroll
+          for (int j = 0; j < S; ++j) add = fmaf(wv[j] * vsc[j], vcode[j], add);
+          Ah[y] = fmaf(Ah[y], al, add);
+          Lh[y] = fmaf(Lh[y], al, ps);
+          Mh[y] = mx;
         }
       }
     }
@@ -855,7 +1033,14 @@ bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
 }
 
 template <int G, int S, int TPT>
-int launch(const TcArgs& ta, const Basis& basis, const CUtensorMap* maps, cudaStream_t stream) {
+int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CUtensorMap* maps,
+           cudaStream_t stream) {
+  TcBasis<S, S * TPT> basis;
+  for (int j = 0; j < S; ++j)
+    for (int t = 0; t < S * TPT; ++t) {
+      basis.m[j][t] = full.m[j][t];
+      basis.m64[j][t] = full64.m[j][t];
+    }
   using C = Cfg<G, S, TPT>;
   const size_t smem = C::alloc;
   auto kern = decode_tc_kernel<G, S, TPT>;
@@ -896,6 +1081,8 @@ int tc_tiles_per_head(int64_t nb, int S) { return int((nb + (tc::kRows / S) - 1)
 
 int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive* va, const Basis& basis,
                      cudaStream_t stream) {
+  BasisF64 basis64;
+  make_basis_f64(d.R, d.S, &basis64);
   tc::TcArgs ta;
   ta.d = d;
   ta.tiles_per_head = tc_tiles_per_head(d.nb, d.S);
@@ -908,7 +1095,7 @@ int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive
   const int key = d.G * 10000 + d.S * 100 + d.R / d.S;
   switch (key) {
 #define FC_TC_CASE(G, S, T) \
-  case G * 10000 + S * 100 + T: return tc::launch<G, S, T>(ta, basis, maps, stream);
+  case G * 10000 + S * 100 + T: return tc::launch<G, S, T>(ta, basis, basis64, maps, stream);
     FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
     FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
     FC_TC_CASE(1, 2, 4) FC_TC_CASE(2, 2, 4) FC_TC_CASE(4, 2, 4) FC_TC_CASE(8, 2, 4)

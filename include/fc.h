@@ -253,6 +253,37 @@ int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t* q_strides
                         const int64_t* out_strides, fc_stream stream);
 
 /*
+ * fc_decode_step -- one decode step: fc_append_step(k_new, v_new, ...)
+ * followed by fc_decode_attention(q, ...) over the updated streams, with the
+ * same results (the archive bitwise; `out` up to the rounding of the new
+ * token's or block's softmax terms) in one kernel launch where the
+ * tensor-core kernel applies (flashcodec/cache.py, _CodecStream.append, then
+ * flashcodec/triton_attention.py, the split kernel: the pages run these as
+ * separate calls; fusing them is this library's). In the fused launch the
+ * last chunk's CTA of each (b, kv head) folds the new token into the softmax
+ * as a raw token and stores it at tail row len, or, when the token completes
+ * a block, encodes that block (tail rows 0..R-2 and the token) into archive
+ * slot n_blocks with the codec's own device code and folds it in the
+ * coefficient domain. Elsewhere (portable flag, no archived block yet, other
+ * dtypes) it issues the two calls.
+ *   k_new, v_new, new_dtype, k_strides, v_strides: as in fc_append_step;
+ *              new_dtype must equal the tails' dtype.
+ *   ka, va, kt, vt: as in fc_append_step (tails required); on success the
+ *              host descriptors are updated as fc_append_step does.
+ *   other arguments: as in fc_decode_attention; FC_DECODE_OVERLAP also
+ *              covers k_new and v_new (read after the dependency wait).
+ * Errors as fc_append_step (FC_ERR_CAPACITY leaves everything unchanged) and
+ * fc_decode_attention.
+ */
+int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int64_t Hq,
+                   const void* k_new, const void* v_new, int32_t new_dtype,
+                   const int64_t* k_strides, const int64_t* v_strides, fc_archive* ka,
+                   fc_archive* va, fc_tail* kt, fc_tail* vt, float softmax_scale,
+                   int32_t num_splits, int32_t flags, void* workspace,
+                   size_t workspace_bytes, void* out, int32_t out_dtype,
+                   const int64_t* out_strides, fc_stream stream);
+
+/*
  * fc_combine -- merge split-K partials left in `workspace` by
  * fc_decode_attention without FC_DECODE_FUSE_COMBINE (flashcodec/triton_attention.py,
  * combine kernel): M = max_c m_c, L = sum_c l_c e^(m_c - M),

@@ -30,7 +30,7 @@ def declared_functions():
 def test_library_exports_every_declared_symbol():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 11, names
+    assert len(names) == 12, names
     assert sorted(names) == sorted(_lib.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
@@ -145,6 +145,30 @@ def test_validation_rejects_bad_arguments_without_launching():
     out_str = (ctypes.c_int64 * 4)(8 * 64, 64, 64, 1)
     assert lib.fc_combine(FAKE, 16, 1, 8, 64, 4, FAKE, _lib.FC_DTYPE_F32,
                           out_str, None) == _lib.FC_ERR_INVALID
+
+
+def test_decode_step_validates_without_launching():
+    """fc_decode_step checks the append and the attention arguments on the
+    host: missing token or tails, capacity (nothing written), bad flags."""
+    s4 = lambda *x: (ctypes.c_int64 * 4)(*x)
+    q_str = s4(8 * 64, 64, 64, 1)
+    tok = s4(2 * 64, 64, 64, 1)
+    ka, va = _arc(H=2, cap=2, nb=2), _arc(H=2, cap=2, nb=2)
+    kt, vt = _tail(ka, 7), _tail(va, 7)
+
+    def step(k_new=FAKE, flags=1, kt_=kt, vt_=vt):
+        return _lib.load().fc_decode_step(
+            FAKE, _lib.FC_DTYPE_BF16, q_str, 8, k_new, FAKE, _lib.FC_DTYPE_BF16,
+            tok, tok, ctypes.byref(ka), ctypes.byref(va),
+            None if kt_ is None else ctypes.byref(kt_),
+            None if vt_ is None else ctypes.byref(vt_), 0.0, 0, flags,
+            FAKE, 1 << 30, FAKE, _lib.FC_DTYPE_F32, q_str, None)
+
+    assert step(k_new=None) == _lib.FC_ERR_INVALID
+    assert step(kt_=None) == _lib.FC_ERR_INVALID
+    assert step(flags=1 << 8) == _lib.FC_ERR_INVALID
+    assert step() == _lib.FC_ERR_CAPACITY        # the token completes block 3
+    assert (ka.n_blocks, kt.len, vt.len) == (2, 7, 7)
 
 
 def test_append_capacity_error_leaves_state():

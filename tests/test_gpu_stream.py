@@ -59,3 +59,90 @@ def test_stream_full_size():
     assert cache.k.n_blocks == (w.T + w.steps) // w.R
     for s, (got, ref, nb, nr) in outs.items():
         check_out(got, ref, "step %d" % s)
+
+
+def _twin_caches(w, data):
+    caches = []
+    for _ in range(2):
+        c = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV)
+        c.prefill(data["k"][:, :, :w.T].to(DEV), data["v"][:, :, :w.T].to(DEV))
+        caches.append(c)
+    return caches
+
+
+def _same_stream(a, b):
+    assert (a.k.n_blocks, a.k.tail_len) == (b.k.n_blocks, b.k.tail_len)
+    for sa, sb in ((a.k, b.k), (a.v, b.v)):
+        assert torch.equal(sa.live_coeffs(), sb.live_coeffs())
+        assert torch.equal(sa.live_scales(), sb.live_scales())
+        assert torch.equal(sa.live_tail(), sb.live_tail())
+
+
+@pytest.mark.parametrize("name,S,R,G", [("gqa-like", 2, 8, 4),
+                                       ("long-like", 4, 16, 4),
+                                       ("S8", 8, 16, 2)])
+def test_fused_step_equals_append_then_attention(name, S, R, G):
+    """fc_decode_step (one launch: append + attention) against fc_append_step
+    followed by fc_decode_attention: the archive and tail bitwise, the
+    outputs within rounding, across two block completions; every output
+    against the oracle on the GPU's own archive."""
+    w = synth.Workload("fstep", B=2, Hq=2 * G, Hk=2, D=128, T=R * 40 + R - 3,
+                       R=R, S=S, seed=R + S, steps=2 * R + 1)
+    data = synth.generate(w, q_steps=w.steps)
+    k, v, q = data["k"].to(DEV), data["v"].to(DEV), data["q"].to(DEV)
+    two, one = _twin_caches(w, data)
+    for s in range(w.steps):
+        t = w.T + s
+        two.append(k[:, :, t:t + 1], v[:, :, t:t + 1])
+        o2 = two.attention(q[s])
+        o1 = one.step(q[s], k[:, :, t:t + 1], v[:, :, t:t + 1],
+                      overlap=s % 3 == 1, q_final=s % 3 == 2)
+        torch.cuda.synchronize()
+        _same_stream(two, one)
+        # the fused launch folds the new token or block on the CUDA cores in
+        # fp32, the two-launch path through the tensor-core limbs: rounding
+        # apart, the same value (the oracle check below is the bar)
+        diff = (o1 - o2).abs().max().item()
+        assert diff <= 2e-4, (s, diff)
+        check_out(f64(o1), oracle_on_gpu_archive(one, q[s]), "step %d" % s)
+
+
+def test_fused_step_in_a_graph_and_portable_path():
+    """Steps captured in a CUDA graph give what eager steps give; the
+    portable flag (two launches) matches too, as does a stream that starts
+    with no archived block (two launches until the first block exists)."""
+    w = synth.Workload("fstep", B=1, Hq=8, Hk=2, D=128, T=8 * 30 + 2, R=8, S=2,
+                       seed=5, steps=20)
+    data = synth.generate(w, q_steps=w.steps)
+    k, v, q = data["k"].to(DEV), data["v"].to(DEV), data["q"].to(DEV)
+    eager, graphed = _twin_caches(w, data)
+    cap = (w.T + w.steps) // w.R + 1
+    eager._grow_to(cap)
+    graphed._grow_to(cap)
+    outs_e = [eager.step(q[s], k[:, :, w.T + s:w.T + s + 1],
+                         v[:, :, w.T + s:w.T + s + 1]) for s in range(w.steps)]
+    outs_g = [torch.empty_like(outs_e[0]) for _ in range(w.steps)]
+    graphed.workspace(w.Hq, graphed.num_splits(w.Hq))
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for s in range(w.steps):
+            graphed.step(q[s], k[:, :, w.T + s:w.T + s + 1],
+                         v[:, :, w.T + s:w.T + s + 1], out=outs_g[s],
+                         overlap=True, q_final=True)
+    g.replay()
+    torch.cuda.synchronize()
+    _same_stream(eager, graphed)
+    for a, b in zip(outs_e, outs_g):
+        assert torch.equal(a, b)
+    # portable (append + CUDA-core attention) from an empty cache
+    port = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV)
+    ref = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV)
+    for s in range(2 * w.R + 3):
+        kt, vt = k[:, :, s:s + 1], v[:, :, s:s + 1]
+        o_port = port.step(q[s % w.steps], kt, vt, portable=True)
+        ref.append(kt, vt)
+        o_ref = ref.attention(q[s % w.steps], portable=True)
+        torch.cuda.synchronize()
+        assert torch.equal(o_port, o_ref)
+    _same_stream(port, ref)
