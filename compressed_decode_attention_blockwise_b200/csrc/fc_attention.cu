@@ -8,10 +8,11 @@
 namespace fc {
 namespace {
 
-// Split count. The tensor-core kernel runs one CTA per SM (a six-stage ring
-// of 128-row tiles fills its shared memory): split each kv head into
-// tile-aligned chunks so that all chunks of all kv heads fit in one wave. The
-// portable kernel aims at four CTAs per SM with chunks of at least 16 blocks.
+// Split count. The tensor-core kernel runs one CTA per SM (its two rings of
+// 128-row tiles fill the shared memory): split each kv head into tile-aligned
+// chunks so that all chunks of all kv heads fit in one wave. The portable
+// kernel fits four CTAs per SM (registers) and aims at one wave of them, with
+// chunks of at least 16 blocks.
 // Results do not depend on the split beyond rounding.
 int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   if (nb <= 0) return 1;
@@ -23,7 +24,8 @@ int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
     const int64_t t = tc_tiles_per_head(nb, S);
     if (ns > t) ns = t;
   } else {
-    ns = (int64_t(sm_count()) * 4 + units - 1) / units;
+    // rounded down: a partial second wave of CTAs would double the time
+    ns = int64_t(sm_count()) * 4 / units;
     const int64_t by_len = nb / 16 > 0 ? nb / 16 : 1;
     if (ns > by_len) ns = by_len;
   }
