@@ -250,6 +250,36 @@ __device__ __forceinline__ constexpr bool is_i8() {
   return std::is_same_v<T, int8_t>;
 }
 
+// Warp sums of N values at once (N a power of two <= 16): at each of the
+// first log2(N) butterfly levels a lane keeps half of its values and trades
+// the other half, so 31 / 32 shuffles do the work of N full reductions. Lane l
+// returns the sum of value l / (32 / N); the additions pair the same lanes in
+// the same order as a per-value xor butterfly, so the sums are bitwise those.
+template <int N>
+__device__ __forceinline__ float warp_reduce_scatter(float (&v)[N], int lane) {
+#pragma unroll
+  for (int n = N, off = 16; n > 1; n >>= 1, off >>= 1) {
+    const bool up = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float send = up ? v[i] : v[i + n / 2];
+      const float keep = up ? v[i + n / 2] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int off = 16 / N; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// 2^x on the special-function unit (ex2.approx.ftz: 2^-inf = +0)
+__device__ __forceinline__ float fast_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int VEC, int G, typename KT, typename VT>
 __global__ void __launch_bounds__(kGenericWarps * 32)
     decode_generic_kernel(DecodeArgs a, Basis basis) {
@@ -258,12 +288,17 @@ __global__ void __launch_bounds__(kGenericWarps * 32)
   __shared__ float s_sm[NW][kMaxS * G];
   __shared__ float p_sm[NW][kMaxR * G];
   __shared__ float w_sm[NW][kMaxS * G];
+  __shared__ float mx_sm[NW][G], ps_sm[NW][G];  // per-head block maxima and sums
   __shared__ float mrg_m[NW * G], mrg_l[NW * G];
   extern __shared__ float dyn[];  // NW * G * D merge buffer, reused for combine weights
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int R = a.R, S = a.S, D = a.D;
+  int RS = 1;  // softmax segment: the power of two >= R
+  while (RS < R) RS <<= 1;
+  const int HP = 32 / RS;  // heads per logits pass
+  const int tok = lane & (RS - 1), hp = lane / RS;
   for (int i = tid; i < R * S; i += blockDim.x) {
     const int t = i / S, j = i - (i / S) * S;
     A_sm[i] = basis.m[j][t];
@@ -291,40 +326,91 @@ __global__ void __launch_bounds__(kGenericWarps * 32)
   const VT* vbase = static_cast<const VT*>(a.vc) + b * a.vcs_b + h * a.vcs_h + lane * VEC;
   const float* ksb = a.ks ? a.ks + b * a.kss_b + h * a.kss_h : nullptr;
   const float* vsb = a.vs ? a.vs + b * a.vss_b + h * a.vss_h : nullptr;
+  // a block of at most kPre rows (and lanes of at most 4 channels) has all its
+  // K and V rows and scales requested at once: one memory round trip per block
+  constexpr int kPre = 4;
+  const bool pre = VEC <= 4 && S <= kPre;
   for (int64_t n = n0 + warp; n < n1; n += NW) {
-    // s_j = scale_kj * (C_k[j] . q) for every kept frequency j
     const KT* krow = kbase + n * S * D;
-    for (int j = 0; j < S; ++j) {
-      float kf[VEC];
-      load_vec<KT, VEC>(krow + int64_t(j) * D, kf);
-      float ksc = 1.f;
-      if constexpr (is_i8<KT>()) ksc = __ldg(ksb + n * S + j);
+    const VT* vrow = vbase + n * S * D;
+    float kb[kPre][VEC], vb[kPre][VEC], kscb[kPre];
+    float vs_mine = 1.f;  // V scale of row lane / G (the lane's first w_j)
+    if (pre) {
+#pragma unroll
+      for (int j = 0; j < kPre; ++j) {
+        if (j < S) {
+          load_vec<KT, VEC>(krow + int64_t(j) * D, kb[j]);
+          load_vec<VT, VEC>(vrow + int64_t(j) * D, vb[j]);
+          kscb[j] = 1.f;
+          if constexpr (is_i8<KT>()) kscb[j] = __ldg(ksb + n * S + j);
+        }
+      }
+      if constexpr (is_i8<VT>()) {
+        if (lane < S * G) vs_mine = __ldg(vsb + n * S + lane / G);
+      }
+    }
+    // s_j = scale_kj * (C_k[j] . q) for every kept frequency j
+    auto k_row = [&](int j, const float (&kf)[VEC], float ksc) {
+      float part[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float part = 0.f;
+        float x = 0.f;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) part = fmaf(kf[v], qv[g][v], part);
-        part = warp_sum(part);
-        if (lane == 0) s_sm[warp][j * G + g] = part * ksc;
+        for (int v = 0; v < VEC; ++v) x = fmaf(kf[v], qv[g][v], x);
+        part[g] = x;
+      }
+      const float tot = warp_reduce_scatter<G>(part, lane);  // head lane / (32 / G)
+      if ((lane & (32 / G - 1)) == 0) s_sm[warp][j * G + lane / (32 / G)] = tot * ksc;
+    };
+    if (pre) {
+#pragma unroll
+      for (int j = 0; j < kPre; ++j)
+        if (j < S) k_row(j, kb[j], kscb[j]);
+    } else {
+      for (int j = 0; j < S; ++j) {
+        float kf[VEC];
+        load_vec<KT, VEC>(krow + int64_t(j) * D, kf);
+        float ksc = 1.f;
+        if constexpr (is_i8<KT>()) ksc = __ldg(ksb + n * S + j);
+        k_row(j, kf, ksc);
       }
     }
     __syncwarp();
-    // logits for token t = lane, online-softmax update per query head
+    // logits: lane = (token t, head slot hp) in segments of RS >= R lanes, HP
+    // heads per pass; per-segment max and sum, then every lane takes the new
+    // maxima and sums of all heads from shared memory
+    for (int g0 = 0; g0 < G; g0 += HP) {
+      const int g = g0 + hp;
+      const bool live = tok < R && g < G;
+      float lg = -INFINITY;
+      if (live) {
+        lg = 0.f;
+        for (int j = 0; j < S; ++j) lg = fmaf(A_sm[tok * S + j], s_sm[warp][j * G + g], lg);
+      }
+      float mo = m[0];
+#pragma unroll
+      for (int gg = 1; gg < G; ++gg) mo = (gg == g) ? m[gg] : mo;
+      float mx = lg;
+      for (int off = RS / 2; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      const float mn = fmaxf(mo, mx);
+      const float p = live ? fast_ex2(lg - mn) : 0.f;
+      float ps = p;
+      for (int off = RS / 2; off > 0; off >>= 1) ps += __shfl_xor_sync(0xffffffffu, ps, off);
+      if (live) p_sm[warp][tok * G + g] = p;
+      if (tok == 0 && g < G) {
+        mx_sm[warp][g] = mn;
+        ps_sm[warp][g] = ps;
+      }
+    }
+    __syncwarp();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      float lg = -INFINITY;
-      if (lane < R) {
-        lg = 0.f;
-        for (int j = 0; j < S; ++j) lg = fmaf(A_sm[lane * S + j], s_sm[warp][j * G + g], lg);
-      }
-      const float mn = fmaxf(m[g], warp_max(lg));
-      const float p = lane < R ? exp2f(lg - mn) : 0.f;
-      const float alpha = exp2f(m[g] - mn);
-      l[g] = fmaf(l[g], alpha, warp_sum(p));
+      const float mn = mx_sm[warp][g];
+      const float alpha = fast_ex2(m[g] - mn);
+      l[g] = fmaf(l[g], alpha, ps_sm[warp][g]);
       m[g] = mn;
 #pragma unroll
       for (int v = 0; v < VEC; ++v) acc[g][v] *= alpha;
-      if (lane < R) p_sm[warp][lane * G + g] = p;
     }
     __syncwarp();
     // w_j = scale_vj * sum_t p_t A[t][j]
@@ -332,20 +418,28 @@ __global__ void __launch_bounds__(kGenericWarps * 32)
       const int j = i / G, g = i - (i / G) * G;
       float x = 0.f;
       for (int t = 0; t < R; ++t) x = fmaf(p_sm[warp][t * G + g], A_sm[t * S + j], x);
-      if constexpr (is_i8<VT>()) x *= __ldg(vsb + n * S + j);
+      if constexpr (is_i8<VT>()) x *= (pre && i == lane) ? vs_mine : __ldg(vsb + n * S + j);
       w_sm[warp][i] = x;
     }
     __syncwarp();
     // acc += w C_v
-    const VT* vrow = vbase + n * S * D;
-    for (int j = 0; j < S; ++j) {
-      float vf[VEC];
-      load_vec<VT, VEC>(vrow + int64_t(j) * D, vf);
+    auto v_row = [&](int j, const float (&vf)[VEC]) {
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         const float wg = w_sm[warp][j * G + g];
 #pragma unroll
         for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wg, vf[v], acc[g][v]);
+      }
+    };
+    if (pre) {
+#pragma unroll
+      for (int j = 0; j < kPre; ++j)
+        if (j < S) v_row(j, vb[j]);
+    } else {
+      for (int j = 0; j < S; ++j) {
+        float vf[VEC];
+        load_vec<VT, VEC>(vrow + int64_t(j) * D, vf);
+        v_row(j, vf);
       }
     }
     __syncwarp();
