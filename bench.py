@@ -161,6 +161,7 @@ class ClockSampler:
 # the files the tensor-core decode-attention kernel is compiled from
 DECODE_SOURCES = ("include/fc.h",
                   "compressed_decode_attention_blockwise_b200/csrc/fc_internal.cuh",
+                  "compressed_decode_attention_blockwise_b200/csrc/fc_encode.cuh",
                   "compressed_decode_attention_blockwise_b200/csrc/fc_decode.cuh",
                   "compressed_decode_attention_blockwise_b200/csrc/fc_tc_ptx.cuh",
                   "compressed_decode_attention_blockwise_b200/csrc/fc_decode_tc.cu")
