@@ -136,32 +136,60 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) compress_stream_kernel(C
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t nw = int64_t(gridDim.x) * kStreamWarps;
   const int64_t w0 = int64_t(blockIdx.x) * kStreamWarps + warp;
-  const int64_t items = int64_t(a.B) * a.H * a.n_full;
   const int64_t stage_bytes = int64_t(a.R) * a.D * int64_t(sizeof(TIn));
   uint8_t* ring = csm + warp * NST * stage_bytes;
   const TIn* x = static_cast<const TIn*>(a.x);
 
-  auto issue = [&](int64_t it, int st) {
-    if (it < items) {
-      const int64_t n = it % a.n_full, bh = it / a.n_full;
-      const int h = int(bh % a.H), b = int(bh / a.H);
-      const TIn* src = x + b * a.xs_b + h * a.xs_h + n * a.R * a.xs_t + lane * VEC;
+  // walks this warp's items it = w0, w0 + nw, ... as (block n, stream bh)
+  // cursors advanced without 64-bit divisions (one up front)
+  struct Cursor {
+    int64_t n, bh;
+  };
+  const int64_t step_bh = nw / a.n_full, step_n = nw - step_bh * a.n_full;
+  auto advance = [&](Cursor& cur) {
+    cur.n += step_n;
+    cur.bh += step_bh;
+    if (cur.n >= a.n_full) {
+      cur.n -= a.n_full;
+      ++cur.bh;
+    }
+  };
+  Cursor ci{w0 % a.n_full, w0 / a.n_full};  // next block to issue
+  Cursor cc = ci;                           // next block to encode
+  const int64_t n_bh = int64_t(a.B) * a.H;
+  // (b, h) of a stream index, in 32 bits whenever the index fits
+  const bool narrow = n_bh <= int64_t(0xffffffffLL);
+  auto split_bh = [&](int64_t bh, int64_t& b, int64_t& h) {
+    if (narrow) {
+      const uint32_t u = uint32_t(bh), hh = uint32_t(a.H);
+      h = u % hh;
+      b = u / hh;
+    } else {
+      h = bh % a.H;
+      b = bh / a.H;
+    }
+  };
+  auto issue = [&](int st) {
+    if (ci.bh < n_bh) {
+      int64_t b, h;
+      split_bh(ci.bh, b, h);
+      const TIn* src = x + b * a.xs_b + h * a.xs_h + ci.n * a.R * a.xs_t + lane * VEC;
       uint8_t* dst = ring + st * stage_bytes + lane * kLaneBytes;
       for (int t = 0; t < a.R; ++t)
         cp_async_row<kLaneBytes>(dst + int64_t(t) * a.D * int64_t(sizeof(TIn)), src + t * a.xs_t);
     }
     cp_async_commit();  // possibly empty: keeps one group per ring slot
+    advance(ci);
   };
 
 #pragma unroll
-  for (int s = 0; s < NST - 1; ++s) issue(w0 + s * nw, s);
-  for (int64_t k = 0;; ++k) {
-    const int64_t it = w0 + k * nw;
-    if (it >= items) break;
-    issue(w0 + (k + NST - 1) * nw, int((k + NST - 1) % NST));
+  for (int s = 0; s < NST - 1; ++s) issue(s);
+  for (int64_t k = 0; cc.bh < n_bh; ++k) {
+    issue(int((k + NST - 1) % NST));
     cp_async_wait<NST - 1>();
-    const int64_t n = it % a.n_full, bh = it / a.n_full;
-    const int h = int(bh % a.H), b = int(bh / a.H);
+    int64_t b, h;
+    split_bh(cc.bh, b, h);
+    const int64_t n = cc.n;
     const TIn* rows = reinterpret_cast<const TIn*>(ring + (k % NST) * stage_bytes) + lane * VEC;
     TOut* blk = static_cast<TOut*>(a.out.coeffs) + b * a.out.cs_b + h * a.out.cs_h +
                 (a.slot0 + n) * a.S * a.D;
@@ -169,6 +197,7 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) compress_stream_kernel(C
                               : nullptr;
     encode_block<TOut, VEC>([&](int t, float (&xf)[VEC]) { load_vec_plain<TIn, VEC>(rows + t * a.D, xf); },
                             a.R, a.S, a.D, lane, basis, blk, scl);
+    advance(cc);
   }
   cp_async_wait<0>();
   if (a.tail != nullptr && w0 < int64_t(a.B) * a.H) {
