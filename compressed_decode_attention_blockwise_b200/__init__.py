@@ -9,7 +9,8 @@ layer's compressed K/V streams (raw tail, capacity-doubling archive).
 from . import _lib
 from ._lib import (FcArchive, FcError, FcTail, fc_append_step,
                    fc_archive_copy_prefix, fc_combine, fc_compress_blocks,
-                   fc_decode_attention, fc_decode_plan,
+                   fc_decode_attention, fc_decode_attention_noalloc,
+                   fc_decode_plan, fc_decode_step,
                    fc_decode_workspace_bytes, fc_status_string,
                    fc_storage_bytes, fc_workspace_status)
 from .archive import CodecKVCache, CodecStream, grown_capacity
@@ -18,6 +19,7 @@ __all__ = [
     "CodecKVCache", "CodecStream", "grown_capacity", "FcArchive", "FcTail",
     "FcError", "fc_compress_blocks", "fc_append_step",
     "fc_archive_copy_prefix", "fc_decode_plan", "fc_decode_workspace_bytes",
-    "fc_decode_attention", "fc_combine", "fc_workspace_status",
-    "fc_storage_bytes", "fc_status_string",
+    "fc_decode_attention", "fc_decode_attention_noalloc", "fc_decode_step",
+    "fc_combine", "fc_workspace_status", "fc_storage_bytes",
+    "fc_status_string",
 ]

@@ -1,7 +1,7 @@
 """Shared helpers of the test suite: build a device cache from synthetic
 inputs, bring its archive back for the fp64 oracle, and the tolerance checks.
 
-Tolerances (spec parity bar):
+Tolerances (the parity bar of this hot path):
 * int8 codes bit-exact, except +-1 where the oracle's pre-rounding value lies
   within 1e-5 of a half-integer;
 * scales within 1e-6 relative;
