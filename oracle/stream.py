@@ -11,13 +11,22 @@ Follows ``flashcodec/cache.py`` ``_CodecStream``:
   need; growing copies the live prefix verbatim (``_grow``).
 * ``storage_bytes`` counts the live archive region plus the raw tail, not the
   idle capacity.
+* ``read`` is the reconstructed view: every archived block decompressed
+  (X_hat = M^T C_hat) and restored to the stream input dtype, followed by the
+  raw tail (``_CodecStream.read`` and ``_decode_pending``).
+* ``crop`` removes trailing tokens exactly: archived blocks below the new
+  boundary are kept verbatim and the partial block at the boundary comes back
+  as raw tail tokens taken from the reconstruction (``_CodecStream.crop``).
+* ``select_batch`` gathers the batch axis of the archive and the raw tail
+  (``_CodecStream.select_batch``; beam reorder, repeat and selection of rows);
+  ``reset`` empties the stream and keeps its capacity (``_CodecStream.reset``).
 """
 
 from __future__ import annotations
 
 import numpy as np
 
-from .codec import compress, quantize, round_to_dtype, dequantize
+from .codec import compress, quantize, round_to_dtype, dequantize, decompress
 
 INITIAL_BLOCKS = 16
 
@@ -137,3 +146,66 @@ class CodecStreamOracle:
         if self.raw is not None:
             total += self.raw.size * elem[self.in_dtype]
         return total
+
+    # -- structural operations -----------------------------------------------
+    def read(self) -> np.ndarray:
+        """Reconstructed (B, H, seq_len, D) view as float64 values of the input
+        dtype: the archived blocks decompressed and rounded to ``in_dtype``,
+        then the raw tail as stored. ``None`` for an empty stream."""
+        parts = []
+        if self.n_blocks:
+            parts.append(round_to_dtype(decompress(self.C_hat(), self.R),
+                                        self.in_dtype))
+        if self.raw is not None:
+            parts.append(self.raw)
+        if not parts:
+            return None
+        return np.concatenate(parts, axis=-2) if len(parts) > 1 else \
+            parts[0].copy()
+
+    def crop(self, tokens_to_remove: int) -> None:
+        """Drop the last ``-tokens_to_remove`` tokens (the pages' convention:
+        a negative count; a positive one is an error, zero does nothing)."""
+        if tokens_to_remove > 0:
+            raise ValueError("crop takes a negative count of tokens to remove")
+        if tokens_to_remove == 0:
+            return
+        keep = max(0, self.seq_len - abs(int(tokens_to_remove)))
+        keep_blocks, rest = divmod(keep, self.R)
+        if keep_blocks < self.n_blocks:
+            # the boundary block's first `rest` tokens, as the view holds them
+            view = self.read()
+            self.n_blocks = keep_blocks
+            self.raw = view[:, :, keep_blocks * self.R:keep].copy() \
+                if rest else None
+        elif rest == 0:
+            self.raw = None
+        else:
+            self.raw = self.raw[:, :, :rest].copy()
+
+    def select_batch(self, idx) -> None:
+        """Batch row i of the result is row ``idx[i]`` of the current stream
+        (the live archive region and the raw tail); indices may repeat and
+        their count may differ from B. The capacity is kept."""
+        idx = np.asarray(idx, dtype=np.int64).reshape(-1)
+        nb = self.n_blocks
+
+        def gather(a):
+            if a is None:
+                return None
+            out = np.zeros((idx.size,) + a.shape[1:], dtype=a.dtype)
+            if nb:
+                out[:, :, :nb] = a[idx][:, :, :nb]
+            return out
+
+        self.codes = gather(self.codes)
+        self.scales = gather(self.scales)
+        self.pre_round = gather(self.pre_round)
+        self.coeffs = gather(self.coeffs)
+        if self.raw is not None:
+            self.raw = self.raw[idx].copy()
+
+    def reset(self) -> None:
+        """Empty the stream; the archive keeps its capacity."""
+        self.raw = None
+        self.n_blocks = 0
