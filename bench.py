@@ -262,6 +262,29 @@ def run_fc(args, world, rank, local):
     comp_bytes = 2 * w.B * w.Hk * w.T * w.D * esz + arc_bytes
     del scratch
 
+    # ---------------- reconstructed view: every archived block of K and V
+    # decoded to the token dtype plus the raw tails (fc_read_view)
+    views = [torch.empty((w.B, w.Hk, w.T, w.D), dtype=tok_dt, device=dev)
+             for _ in range(2)]
+
+    def view_once():
+        for st, o in zip((caches[0].k, caches[0].v), views):
+            _lib.fc_read_view(st.arc, st.tail_desc, 0, o)
+
+    n_view = max(3, min(K, 30))
+    for _ in range(max(W, 3)):
+        view_once()
+    torch.cuda.synchronize()
+    barrier(world)
+    ev0.record()
+    for _ in range(n_view):
+        view_once()
+    ev1.record()
+    torch.cuda.synchronize()
+    view_s = max_over_ranks(ev0.elapsed_time(ev1) / 1e3 / n_view, world)
+    view_bytes = arc_bytes + 2 * w.B * w.Hk * w.D * esz * (w.T + w.n_tail)
+    del views
+
     Hq = w.Hq
     out_bufs = [torch.empty((w.B, Hq, 1, w.D), dtype=torch.float32,
                             device=dev) for _ in range(copies)]
@@ -440,6 +463,17 @@ def run_fc(args, world, rank, local):
             "GB_per_s": round(comp_bytes / comp_s / 1e9, 2),
             "us_per_prefill": round(comp_s * 1e6, 2),
             "frac_of_peak": round(comp_bytes / comp_s / 1e9 / peak, 4),
+        },
+        "read_view": {
+            "kernel": "fc_read_view: every archived block of K and V decoded "
+                      "to the token dtype, plus the raw tails",
+            "us": round(view_s * 1e6, 2),
+            "GB_per_s": round(view_bytes / view_s / 1e9, 2),
+            "frac_of_peak": round(view_bytes / view_s / 1e9 / peak, 4),
+            "bytes": int(view_bytes),
+            "l2": "each pass writes %.0f MB (> L2), evicting the archive "
+                  "before the next pass" % (2 * w.B * w.Hk * w.T * w.D * esz
+                                            / 1e6),
         },
         "us_per_layer": round(step_s * 1e6, 3),
         "e2e": {"value": round(whole_job_gbs(e2e_bytes, world, e2e_s), 2),

@@ -1,4 +1,4 @@
-"""Thin ctypes binding of libfc (``include/fc.h``).
+"""Thin ctypes binding of libfc (``include/fc.h``, ``include/fc_view.h``).
 
 Argument marshalling only: tensors become device pointers, element strides
 and the current CUDA stream; every computation runs in libfc's kernels. A
@@ -30,6 +30,8 @@ FC_DECODE_PORTABLE = 2
 FC_DECODE_OVERLAP = 4
 FC_DECODE_Q_FINAL = 8
 
+FC_SELECT_MAX_BATCH = 1024
+
 FC_DTYPE_F32 = 0
 FC_DTYPE_BF16 = 1
 FC_DTYPE_I8 = 2
@@ -37,12 +39,13 @@ FC_DTYPE_I8 = 2
 _DTYPE_CODE = {torch.float32: FC_DTYPE_F32, torch.bfloat16: FC_DTYPE_BF16,
                torch.int8: FC_DTYPE_I8}
 
-# Every symbol include/fc.h declares.
+# Every symbol include/fc.h and include/fc_view.h declare.
 EXPORTS = (
     "fc_compress_blocks", "fc_append_step", "fc_archive_copy_prefix",
     "fc_decode_plan", "fc_decode_workspace_bytes", "fc_decode_attention",
     "fc_combine", "fc_decode_attention_noalloc", "fc_workspace_status",
     "fc_storage_bytes", "fc_status_string", "fc_decode_step",
+    "fc_read_view", "fc_crop", "fc_select_batch",
 )
 
 
@@ -119,6 +122,9 @@ def load() -> ctypes.CDLL:
                                                P]),
         "fc_storage_bytes": (ctypes.c_int64, [PA, PT]),
         "fc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "fc_read_view": (ctypes.c_int, [PA, PT, I64, P, I32, PI64, I64, P]),
+        "fc_crop": (ctypes.c_int, [PA, PT, I64, P]),
+        "fc_select_batch": (ctypes.c_int, [PA, PT, PI64, I64, PA, PT, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -302,3 +308,41 @@ def fc_storage_bytes(arc: FcArchive, tail: Optional[FcTail] = None) -> int:
     if n < 0:
         raise FcError(FC_ERR_INVALID, "fc_storage_bytes")
     return n
+
+
+# --------------------------------------------------- stream structure (view)
+
+def fc_read_view(arc: FcArchive, tail: Optional[FcTail], first_block: int,
+                 out: torch.Tensor, stream=None) -> None:
+    """Decode archived blocks [first_block, n_blocks) and copy the live tail
+    rows into ``out`` (B, H, T_out, D) at their token positions."""
+    st = load().fc_read_view(ctypes.byref(arc), _ref(tail), int(first_block),
+                             _ptr(out), dtype_code(out.dtype),
+                             _strides4(out), int(out.shape[2]),
+                             _stream(stream, out))
+    _check(st, "fc_read_view")
+
+
+def fc_crop(arc: FcArchive, tail: FcTail, tokens_to_remove: int,
+            stream=None, device=None) -> None:
+    """Remove the last ``-tokens_to_remove`` tokens (a negative count)."""
+    s = _stream(stream) if stream is not None or device is None else \
+        ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = load().fc_crop(ctypes.byref(arc), ctypes.byref(tail),
+                        int(tokens_to_remove), s)
+    _check(st, "fc_crop")
+
+
+def fc_select_batch(src: FcArchive, src_tail: Optional[FcTail], idx,
+                    dst: FcArchive, dst_tail: Optional[FcTail],
+                    stream=None, device=None) -> None:
+    """Batch row i of ``dst`` := batch row ``idx[i]`` of ``src`` (archive
+    live blocks and tail rows). ``idx`` is a host sequence of ints."""
+    idx = [int(i) for i in idx]
+    arr = (ctypes.c_int64 * max(1, len(idx)))(*idx)
+    s = _stream(stream) if stream is not None or device is None else \
+        ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = load().fc_select_batch(ctypes.byref(src), _ref(src_tail), arr,
+                                len(idx), ctypes.byref(dst), _ref(dst_tail),
+                                s)
+    _check(st, "fc_select_batch")

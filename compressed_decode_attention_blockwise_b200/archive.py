@@ -4,6 +4,9 @@ Host bookkeeping around libfc (flashcodec/cache.py, ``_CodecStream`` and
 ``CodecKVCache``): each stream keeps a raw tail of at most R-1 tokens at the
 input precision and a compressed archive whose capacity starts at 16 blocks
 and doubles when full, the live prefix being copied by libfc's copy kernel.
+The structural operations of the pages' cache are here too: the memoised
+reconstructed view (``read``), exact ``crop``, batch gather
+(``select_batch`` / ``reorder_cache``) and ``reset``.
 Device memory comes from torch; every byte of codec and attention arithmetic
 runs in libfc's kernels.
 """
@@ -56,18 +59,22 @@ class CodecStream:
         self.tail_desc.len = 0
         self.tail_desc.stride_b, self.tail_desc.stride_h = \
             self.tail.stride(0), self.tail.stride(1)
+        self._rec: Optional[torch.Tensor] = None   # reconstructed view
+        self._rec_blocks = 0                       # blocks decoded into it
         self._alloc(grown_capacity(0, max(capacity, 1)))
 
     # -- storage -----------------------------------------------------------
-    def _alloc(self, cap: int):
-        coeffs = torch.empty((self.B, self.H, cap, self.S, self.D),
+    def _storage(self, B: int, cap: int):
+        """Fresh (coeffs, scales, descriptor with n_blocks = 0) for B rows."""
+        coeffs = torch.empty((B, self.H, cap, self.S, self.D),
                              dtype=_COEFF[self.coeff], device=self.device)
         scales = None
         if self.coeff == "i8":
-            scales = torch.empty((self.B, self.H, cap, self.S),
+            scales = torch.empty((B, self.H, cap, self.S),
                                  dtype=torch.float32, device=self.device)
         new = _lib.FcArchive()
         ctypes_copy(new, self.arc)
+        new.B = B
         new.coeffs = coeffs.data_ptr()
         new.scales = None if scales is None else scales.data_ptr()
         new.capacity = cap
@@ -79,6 +86,10 @@ class CodecStream:
                 scales.stride(1)
         else:
             new.scale_stride_b = new.scale_stride_h = 0
+        return coeffs, scales, new
+
+    def _alloc(self, cap: int):
+        coeffs, scales, new = self._storage(self.B, cap)
         if self.coeffs is not None and self.arc.n_blocks:
             _lib.fc_archive_copy_prefix(self.arc, new, device=self.device)
         else:
@@ -119,6 +130,80 @@ class CodecStream:
 
     def storage_bytes(self) -> int:
         return _lib.fc_storage_bytes(self.arc, self.tail_desc)
+
+    # -- structure (flashcodec/cache.py, _CodecStream) -------------------------
+    def read(self) -> Optional[torch.Tensor]:
+        """Reconstructed (B, H, seq_len, D) view in the token dtype
+        (``_CodecStream.read``): archived blocks decompressed by libfc, then
+        the raw tail. Each archived block is decoded once into a persistent
+        buffer (append-only memoisation); ``None`` for an empty stream, the
+        tail itself when nothing is archived. The returned tensor aliases
+        that buffer: rows below ``n_blocks * R`` keep their values until a
+        crop, batch gather or reset, while the raw-tail rows after them are
+        rewritten by the next read (with the decoded block once it is
+        archived)."""
+        T = self.seq_len
+        if T == 0:
+            return None
+        if self.n_blocks == 0:
+            return self.live_tail()
+        need = -(-T // self.R) * self.R
+        if self._rec is None or self._rec.shape[2] < need:
+            old = 0 if self._rec is None else self._rec.shape[2]
+            rows = max(need, 2 * old, INITIAL_BLOCKS * self.R)
+            self._rec = torch.empty((self.B, self.H, rows, self.D),
+                                    dtype=self.token_dtype,
+                                    device=self.device)
+            self._rec_blocks = 0   # a new buffer is decoded from block 0
+        _lib.fc_read_view(self.arc, self.tail_desc, self._rec_blocks,
+                          self._rec)
+        self._rec_blocks = self.n_blocks
+        return self._rec[:, :, :T]
+
+    def discard_view(self):
+        """Free the reconstructed view (rebuilt by the next ``read``)."""
+        self._rec = None
+        self._rec_blocks = 0
+
+    def crop(self, tokens_to_remove: int):
+        """Remove the last ``-tokens_to_remove`` tokens exactly: archived
+        blocks below the new end stay verbatim, a partial boundary block
+        returns to the raw tail from its reconstruction
+        (``_CodecStream.crop``; a negative count, zero does nothing)."""
+        if tokens_to_remove > 0:
+            raise ValueError("crop takes a negative count of tokens to remove")
+        _lib.fc_crop(self.arc, self.tail_desc, int(tokens_to_remove),
+                     device=self.device)
+        self._rec_blocks = min(self._rec_blocks, self.n_blocks)
+
+    def select_batch(self, idx):
+        """Batch row i becomes row ``idx[i]`` (``_CodecStream.select_batch``):
+        the archive and the raw tail are gathered by libfc into new storage
+        of the same capacity; the view is rebuilt by the next ``read``."""
+        if isinstance(idx, torch.Tensor):
+            idx = idx.tolist()
+        idx = [int(i) for i in idx]
+        coeffs, scales, arc = self._storage(len(idx), self.capacity)
+        tail = torch.zeros((len(idx), self.H, self.R, self.D),
+                           dtype=self.token_dtype, device=self.device)
+        td = _lib.FcTail()
+        ctypes_copy(td, self.tail_desc)
+        td.data = tail.data_ptr()
+        td.len = 0
+        td.stride_b, td.stride_h = tail.stride(0), tail.stride(1)
+        _lib.fc_select_batch(self.arc, self.tail_desc, idx, arc, td,
+                             device=self.device)
+        self.B = len(idx)
+        self.coeffs, self.scales, self.arc = coeffs, scales, arc
+        self.tail, self.tail_desc = tail, td
+        self.discard_view()
+
+    def reset(self):
+        """Empty the stream; capacity and buffers are kept
+        (``_CodecStream.reset``)."""
+        self.arc.n_blocks = 0
+        self.tail_desc.len = 0
+        self._rec_blocks = 0
 
 
 def ctypes_copy(dst, src):
@@ -259,6 +344,53 @@ class CodecKVCache:
 
     def storage_bytes(self) -> int:
         return self.k.storage_bytes() + self.v.storage_bytes()
+
+    # -- the pages' cache interface (flashcodec/cache.py, CodecKVCache) --------
+    def update(self, k_states: torch.Tensor, v_states: torch.Tensor):
+        """Append (B, Hk, m, D) tokens to both streams, archiving across block
+        boundaries, and return the reconstructed (key_view, value_view)."""
+        self.prefill(k_states, v_states)
+        return self.read()
+
+    def read(self):
+        """(key_view, value_view): each stream's reconstructed view."""
+        return self.k.read(), self.v.read()
+
+    def get_seq_length(self) -> int:
+        return self.seq_len
+
+    def crop(self, tokens_to_remove: int):
+        """Exact removal of trailing tokens from both streams (negative count,
+        e.g. rejected speculative tokens)."""
+        self.k.crop(tokens_to_remove)
+        self.v.crop(tokens_to_remove)
+
+    def select_batch(self, idx):
+        """Gather batch rows of both streams (archives and raw tails)."""
+        self.k.select_batch(idx)
+        self.v.select_batch(idx)
+        self.B = self.k.B
+        self._plans.clear()
+        self._ws_need.clear()
+
+    reorder_cache = select_batch   # beam search
+
+    def batch_repeat_interleave(self, repeats: int):
+        """Replicate every batch row ``repeats`` times (contrastive search)."""
+        self.select_batch([b for b in range(self.B) for _ in range(repeats)])
+
+    def batch_select_indices(self, indices):
+        """Keep only the given batch rows."""
+        self.select_batch(indices)
+
+    def discard_view(self):
+        self.k.discard_view()
+        self.v.discard_view()
+
+    def reset(self):
+        """Empty both streams, keeping their capacity."""
+        self.k.reset()
+        self.v.reset()
 
 
 def default_scale(D: int) -> float:

@@ -15,22 +15,27 @@ from compressed_decode_attention_blockwise_b200.archive import grown_capacity
 from oracle.stream import grown_capacity as oracle_grown_capacity
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "fc.h")
+INCLUDE = os.path.join(ROOT, "include")
 FAKE = 0x10000  # aligned non-null address; never dereferenced here
 
 
 def declared_functions():
-    src = open(HEADER).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(
-        r"^\s*(?:const\s+)?[A-Za-z_0-9]+\s*\*?\s+(fc_[a-z_0-9]+)\s*\(", src,
-        flags=re.M)))
+    names = set()
+    for fn in sorted(os.listdir(INCLUDE)):
+        if not fn.endswith(".h"):
+            continue
+        src = open(os.path.join(INCLUDE, fn)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names.update(re.findall(
+            r"^\s*(?:const\s+)?[A-Za-z_0-9]+\s*\*?\s+(fc_[a-z_0-9]+)\s*\(",
+            src, flags=re.M))
+    return sorted(names)
 
 
 def test_library_exports_every_declared_symbol():
     lib = _lib.load()
     names = declared_functions()
-    assert len(names) == 12, names
+    assert len(names) == 15, names
     assert sorted(names) == sorted(_lib.EXPORTS)
     for n in names:
         assert hasattr(lib, n), n
@@ -221,3 +226,84 @@ def test_split_planner():
     assert plan(64, 8, 64, 8, 3, 1024, 64) == 1        # 512 pairs > 148 * 4 / 2
     assert plan(16, 8, 64, 8, 3, 1024, 64) == 4        # floor(592 / 128)
     assert plan(1, 4, 64, 8, 2, 32, 4, _lib.FC_DTYPE_F32) == 2  # nb / 16
+
+
+def test_view_crop_and_gather_validate_without_launching():
+    """fc_read_view, fc_crop and fc_select_batch check their arguments on
+    the host; the cases below either fail validation or need no launch."""
+    lib = _lib.load()
+    s4 = lambda *x: (ctypes.c_int64 * 4)(*x)
+    a = _arc(H=2, cap=4, nb=3)
+    t = _tail(a, 5)
+    rows = 3 * 8 + 5
+    out_str = s4(2 * 32 * 64, 32 * 64, 64, 1)
+
+    def view(first=0, out=FAKE, dt=_lib.FC_DTYPE_BF16, strides=out_str,
+             tokens=32, tail=t):
+        return lib.fc_read_view(ctypes.byref(a), _ref(tail), first, out, dt,
+                                strides, tokens, None)
+
+    _ref = lambda x: None if x is None else ctypes.byref(x)
+    assert view(first=-1) == _lib.FC_ERR_INVALID
+    assert view(first=4) == _lib.FC_ERR_INVALID            # > n_blocks
+    assert view(out=None) == _lib.FC_ERR_INVALID
+    assert view(out=FAKE + 8) == _lib.FC_ERR_INVALID       # misaligned
+    assert view(dt=_lib.FC_DTYPE_I8) == _lib.FC_ERR_INVALID
+    assert view(tokens=rows - 1) == _lib.FC_ERR_INVALID    # too few rows
+    assert view(strides=s4(2 * 32 * 64, 32 * 64, 64, 2)) == \
+        _lib.FC_ERR_INVALID                                # inner stride
+    assert view(strides=s4(2 * 32 * 64, 32 * 64, 60, 1)) == \
+        _lib.FC_ERR_INVALID                                # rows overlap
+    # nothing to write: every block already decoded, empty tail
+    assert view(first=3, tail=None) == _lib.FC_OK
+
+    # crop: sign convention, missing tail, host-only cases
+    c = _arc(H=2, cap=4, nb=3)
+    ct = _tail(c, 5)
+    assert lib.fc_crop(ctypes.byref(c), ctypes.byref(ct), 2, None) == \
+        _lib.FC_ERR_INVALID
+    assert lib.fc_crop(ctypes.byref(c), None, -2, None) == \
+        _lib.FC_ERR_INVALID
+    assert lib.fc_crop(ctypes.byref(c), ctypes.byref(ct), 0, None) == \
+        _lib.FC_OK
+    assert (c.n_blocks, ct.len) == (3, 5)
+    assert lib.fc_crop(ctypes.byref(c), ctypes.byref(ct), -2, None) == \
+        _lib.FC_OK                                         # tail only
+    assert (c.n_blocks, ct.len) == (3, 3)
+    assert lib.fc_crop(ctypes.byref(c), ctypes.byref(ct), -11, None) == \
+        _lib.FC_OK                                         # to a boundary
+    assert (c.n_blocks, ct.len) == (2, 0)
+    assert lib.fc_crop(ctypes.byref(c), ctypes.byref(ct), -1000, None) == \
+        _lib.FC_OK                                         # everything
+    assert (c.n_blocks, ct.len) == (0, 0)
+
+    # select_batch: index range, batch size, overlap, capacity, tails
+    src = _arc(B=3, H=2, cap=4, nb=3)
+    dst = _arc(B=2, H=2, cap=4)
+    dst.coeffs = FAKE + (1 << 24)
+    dst.scales = FAKE + (2 << 24)
+    src.scales = FAKE + (3 << 24)
+
+    def gather(idx, d=dst, st=None, dt=None):
+        arr = (ctypes.c_int64 * len(idx))(*idx)
+        return lib.fc_select_batch(ctypes.byref(src), _ref(st), arr, len(idx),
+                                   ctypes.byref(d), _ref(dt), None)
+
+    assert gather([0, 3]) == _lib.FC_ERR_INVALID           # index >= B
+    assert gather([0, -1]) == _lib.FC_ERR_INVALID
+    assert gather([0, 1, 2]) == _lib.FC_ERR_INVALID        # dst.B != n_idx
+    same = _arc(B=2, H=2, cap=4)                           # overlaps src
+    same.scales = FAKE + (2 << 24)
+    assert gather([0, 1], d=same) == _lib.FC_ERR_INVALID
+    small = _arc(B=2, H=2, cap=2)
+    small.coeffs, small.scales = dst.coeffs, dst.scales
+    assert gather([0, 1], d=small) == _lib.FC_ERR_CAPACITY
+    assert gather([0, 1], st=_tail(src, 2)) == _lib.FC_ERR_INVALID  # one tail
+    assert dst.n_blocks == 0
+    assert lib.fc_select_batch(ctypes.byref(src), None, None, 2,
+                               ctypes.byref(dst), None, None) == \
+        _lib.FC_ERR_INVALID
+    big = (ctypes.c_int64 * 1025)(*([0] * 1025))
+    assert lib.fc_select_batch(ctypes.byref(src), None, big, 1025,
+                               ctypes.byref(dst), None, None) == \
+        _lib.FC_ERR_UNSUPPORTED
