@@ -44,7 +44,8 @@ struct ViewArgs {
   int64_t tail_items;   // B * H when tail rows are copied, else 0
 };
 
-// VEC consecutive outputs of one lane, rounded to the out dtype.
+// VEC consecutive outputs of one lane, rounded to the out dtype (bf16: round
+// to nearest even, two values per conversion).
 template <typename TO, int VEC>
 __device__ __forceinline__ void store_out(TO* p, const float (&v)[VEC]) {
   if constexpr (std::is_same<TO, float>::value) {
@@ -57,17 +58,16 @@ __device__ __forceinline__ void store_out(TO* p, const float (&v)[VEC]) {
       for (int c = 0; c < VEC / 4; ++c)
         reinterpret_cast<float4*>(p)[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
     }
+  } else if constexpr (VEC == 1) {
+    *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(v[0]);
   } else {
-    uint32_t w[(VEC + 1) / 2];
+    uint32_t w[VEC / 2];
 #pragma unroll
-    for (int i = 0; i < VEC; i += 2) {
-      const uint32_t lo = __bfloat16_as_ushort(__float2bfloat16_rn(v[i]));
-      const uint32_t hi = (i + 1 < VEC) ? __bfloat16_as_ushort(__float2bfloat16_rn(v[i + 1])) : 0u;
-      w[i / 2] = lo | (hi << 16);
+    for (int i = 0; i < VEC / 2; ++i) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+      w[i] = *reinterpret_cast<const uint32_t*>(&h);
     }
-    if constexpr (VEC == 1) {
-      *reinterpret_cast<unsigned short*>(p) = static_cast<unsigned short>(w[0]);
-    } else if constexpr (VEC == 2) {
+    if constexpr (VEC == 2) {
       *reinterpret_cast<uint32_t*>(p) = w[0];
     } else if constexpr (VEC == 4) {
       *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
@@ -77,18 +77,72 @@ __device__ __forceinline__ void store_out(TO* p, const float (&v)[VEC]) {
   }
 }
 
-// Resident CTAs per SM the view kernel is compiled for (64 registers per
-// thread with up to 8 coefficient rows, 128 with up to 16).
-template <int MAXS>
+// The raw bytes of one lane's VEC consecutive coefficients of one frequency
+// row, loaded ahead of their use and converted afterwards.
+template <typename TC, int VEC>
+struct RawRow {
+  static constexpr int kBytes = VEC * int(sizeof(TC));
+  static constexpr int kWords = kBytes >= 4 ? kBytes / 4 : 1;
+  uint32_t w[kWords];
+
+  __device__ __forceinline__ void load(const TC* p) {
+    if constexpr (kBytes >= 16) {
+#pragma unroll
+      for (int c = 0; c < kBytes / 16; ++c) {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(p) + c);
+        w[4 * c] = u.x;
+        w[4 * c + 1] = u.y;
+        w[4 * c + 2] = u.z;
+        w[4 * c + 3] = u.w;
+      }
+    } else if constexpr (kBytes == 8) {
+      const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+      w[0] = u.x;
+      w[1] = u.y;
+    } else if constexpr (kBytes == 4) {
+      w[0] = __ldg(reinterpret_cast<const unsigned int*>(p));
+    } else if constexpr (kBytes == 2) {
+      w[0] = __ldg(reinterpret_cast<const unsigned short*>(p));
+    } else {
+      w[0] = static_cast<uint8_t>(__ldg(reinterpret_cast<const signed char*>(p)));
+    }
+  }
+
+  // int8: exact, without a conversion instruction: the biased byte b + 128
+  // becomes the low mantissa bits of 2^23, and 2^23 + 128 is subtracted.
+  __device__ __forceinline__ void to_float(float (&out)[VEC]) const {
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) {
+      if constexpr (std::is_same<TC, int8_t>::value) {
+        const uint32_t u = w[i / 4] ^ 0x80808080u;
+        out[i] = __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7440u | uint32_t(i % 4))) - 8388736.0f;
+      } else if constexpr (std::is_same<TC, __nv_bfloat16>::value) {
+        const uint32_t x = w[i / 2];
+        out[i] = __uint_as_float((i % 2) ? (x & 0xffff0000u) : (x << 16));
+      } else {
+        out[i] = __uint_as_float(w[i]);
+      }
+    }
+  }
+};
+
+// Resident CTAs per SM the view kernel is compiled for, from the registers
+// a lane holds: MAXS >= S coefficient rows of VEC values (and their raw
+// prefetched words, twice as many for fp32 storage).
+template <typename TC, int VEC, int MAXS>
 constexpr int view_ctas_per_sm() {
-  return MAXS <= 8 ? 4 : 2;
+  constexpr int held = MAXS * VEC * (sizeof(TC) == 4 ? 2 : 1);
+  return held <= 16 ? 5 : held <= 32 ? 3 : held <= 64 ? 2 : 1;
 }
 
-// TC: stored coefficient type; TO: view dtype; VEC = D / 32; MAXS >= S bounds
-// the register-resident coefficient rows (loops over j are unrolled to MAXS
-// and guarded by j < S, so the rows are never indexed dynamically).
+// TC: stored coefficient type; TO: view dtype; VEC = D / 32. Loops over the
+// frequencies j are unrolled to MAXS and guarded by j < S, so the rows are
+// never indexed dynamically. Each warp walks its items with a stride of the
+// grid's warp count and loads the next item's codes and scales before it
+// writes the current item's R rows. Item counts fit in 31 bits (checked on
+// the host).
 template <typename TC, typename TO, int VEC, int MAXS>
-__global__ void __launch_bounds__(kViewThreads, view_ctas_per_sm<MAXS>())
+__global__ void __launch_bounds__(kViewThreads, view_ctas_per_sm<TC, VEC, MAXS>())
     read_view_kernel(ViewArgs a, Basis basis) {
   __shared__ float m_s[kMaxS * kMaxR];  // m_s[j * R + t] = M[j][t]
   for (int i = threadIdx.x; i < a.S * a.R; i += kViewThreads) {
@@ -98,29 +152,51 @@ __global__ void __launch_bounds__(kViewThreads, view_ctas_per_sm<MAXS>())
   __syncthreads();
 
   constexpr int D = VEC * 32;
+  constexpr bool kQuant = std::is_same<TC, int8_t>::value;
   const int lane = threadIdx.x & 31;
-  const int64_t warps = int64_t(gridDim.x) * kViewWarps;
-  const int64_t total = a.block_items + a.tail_items;
-  for (int64_t item = int64_t(blockIdx.x) * kViewWarps + (threadIdx.x >> 5); item < total; item += warps) {
-    if (item < a.block_items) {
-      const int64_t bh = item / a.count;
-      const int64_t n = a.first + (item - bh * a.count);
-      const int64_t b = bh / a.H, h = bh - b * a.H;
-      const TC* cp = static_cast<const TC*>(a.coeffs) + b * a.cs_b + h * a.cs_h + n * a.S * D + lane * VEC;
+  const uint32_t warps = gridDim.x * kViewWarps;
+  const uint32_t block_items = uint32_t(a.block_items);
+  const uint32_t total = block_items + uint32_t(a.tail_items);
+  const uint32_t count = uint32_t(a.count), H = uint32_t(a.H);
+
+  RawRow<TC, VEC> raw[MAXS];
+  float sc[MAXS];
+  auto fetch = [&](uint32_t item) {
+    const uint32_t bh = item / count;
+    const int64_t n = a.first + (item - bh * count);
+    const uint32_t b = bh / H, h = bh - b * H;
+    const TC* cp = static_cast<const TC*>(a.coeffs) + b * a.cs_b + h * a.cs_h + n * a.S * D + lane * VEC;
+    const float* sp = kQuant ? a.scales + b * a.ss_b + h * a.ss_h + n * a.S : nullptr;
+#pragma unroll
+    for (int j = 0; j < MAXS; ++j) {
+      if (j < a.S) {
+        raw[j].load(cp + j * D);
+        if constexpr (kQuant) sc[j] = __ldg(sp + j);
+      }
+    }
+  };
+
+  uint32_t item = blockIdx.x * kViewWarps + (threadIdx.x >> 5);
+  if (item < block_items) fetch(item);
+  for (; item < total; item += warps) {
+    if (item < block_items) {
       float c[MAXS][VEC];
 #pragma unroll
       for (int j = 0; j < MAXS; ++j) {
         if (j < a.S) {
-          load_vec<TC, VEC>(cp + j * D, c[j]);
-          if constexpr (std::is_same<TC, int8_t>::value) {
-            const float s = __ldg(a.scales + b * a.ss_b + h * a.ss_h + n * a.S + j);
+          raw[j].to_float(c[j]);
+          if constexpr (kQuant) {
 #pragma unroll
-            for (int v = 0; v < VEC; ++v) c[j][v] *= s;
+            for (int v = 0; v < VEC; ++v) c[j][v] *= sc[j];
           }
         }
       }
-      TO* op = static_cast<TO*>(a.out) + b * a.os_b + h * a.os_h +
-               (a.out_row0 + (n - a.first) * a.R) * a.os_t + lane * VEC;
+      const uint32_t bh = item / count;
+      const int64_t nr = item - bh * count;  // block index relative to `first`
+      const uint32_t b = bh / H, h = bh - b * H;
+      if (item + warps < block_items) fetch(item + warps);
+      TO* op = static_cast<TO*>(a.out) + b * a.os_b + h * a.os_h + (a.out_row0 + nr * a.R) * a.os_t +
+               lane * VEC;
       for (int t = 0; t < a.rows; ++t) {
         float x[VEC];
 #pragma unroll
@@ -137,8 +213,8 @@ __global__ void __launch_bounds__(kViewThreads, view_ctas_per_sm<MAXS>())
       }
     } else {
       // raw tail rows, converted to the view dtype
-      const int64_t bh = item - a.block_items;
-      const int64_t b = bh / a.H, h = bh - b * a.H;
+      const uint32_t bh = item - block_items;
+      const uint32_t b = bh / H, h = bh - b * H;
       TO* op = static_cast<TO*>(a.out) + b * a.os_b + h * a.os_h + a.tail_row0 * a.os_t + lane * VEC;
       const int64_t tbase = b * a.ts_b + h * a.ts_h + lane * VEC;
       for (int r = 0; r < a.tail_len; ++r) {
@@ -228,15 +304,22 @@ int dispatch_d(int64_t D, F&& f) {
   }
 }
 
+template <typename TC, typename TO, int VEC, int MAXS>
+int launch_view_as(const ViewArgs& a, const Basis& basis, int64_t total, fc_stream stream) {
+  int64_t grid = (total + kViewWarps - 1) / kViewWarps;
+  const int64_t cap = int64_t(sm_count()) * view_ctas_per_sm<TC, VEC, MAXS>();
+  if (grid > cap) grid = cap;
+  read_view_kernel<TC, TO, VEC, MAXS><<<unsigned(grid), kViewThreads, 0, stream>>>(a, basis);
+  return cuda_status(cudaGetLastError());
+}
+
 // Launches the view kernel for `a` (items already counted). Grid: enough
 // warps for every item, at most one wave of resident CTAs (a grid-stride
 // loop covers the rest).
 int launch_view(const ViewArgs& a, int coeff_dtype, int out_dtype, int64_t D, fc_stream stream) {
   const int64_t total = a.block_items + a.tail_items;
   if (total == 0) return FC_OK;
-  int64_t grid = (total + kViewWarps - 1) / kViewWarps;
-  const int64_t cap = int64_t(sm_count()) * (a.S <= 8 ? view_ctas_per_sm<8>() : view_ctas_per_sm<kMaxS>());
-  if (grid > cap) grid = cap;
+  if (total >= (int64_t(1) << 31)) return FC_ERR_UNSUPPORTED;
   Basis basis;
   make_basis(a.R, a.S, &basis);
   return dispatch_coeff(coeff_dtype, [&](auto tc) {
@@ -245,11 +328,10 @@ int launch_view(const ViewArgs& a, int coeff_dtype, int out_dtype, int64_t D, fc
       using TO = decltype(to);
       return dispatch_d(D, [&](auto vec) {
         constexpr int VEC = decltype(vec)::value;
-        if (a.S <= 8)
-          read_view_kernel<TC, TO, VEC, 8><<<unsigned(grid), kViewThreads, 0, stream>>>(a, basis);
-        else
-          read_view_kernel<TC, TO, VEC, kMaxS><<<unsigned(grid), kViewThreads, 0, stream>>>(a, basis);
-        return cuda_status(cudaGetLastError());
+        if (a.S <= 2) return launch_view_as<TC, TO, VEC, 2>(a, basis, total, stream);
+        if (a.S <= 4) return launch_view_as<TC, TO, VEC, 4>(a, basis, total, stream);
+        if (a.S <= 8) return launch_view_as<TC, TO, VEC, 8>(a, basis, total, stream);
+        return launch_view_as<TC, TO, VEC, kMaxS>(a, basis, total, stream);
       });
     });
   });
