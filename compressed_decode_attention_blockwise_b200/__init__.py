@@ -1,9 +1,10 @@
 """Block-DCT int8 KV-cache codec and coefficient-domain decode attention for
 NVIDIA B200 (sm_100a).
 
-The compute lives in ``libfc.so`` (C ABI declared in ``include/fc.h``);
-``_lib`` is its ctypes binding and ``archive`` the host bookkeeping of one
-layer's compressed K/V streams (raw tail, capacity-doubling archive).
+The compute lives in ``libfc.so`` (C ABI declared in ``include/fc.h`` and
+``include/fc_view.h``); ``_lib`` is its ctypes binding and ``archive`` the
+host bookkeeping of one layer's compressed K/V streams (raw tail,
+capacity-doubling archive, reconstructed view, crop, batch gather, reset).
 """
 
 from . import _lib
@@ -12,7 +13,8 @@ from ._lib import (FcArchive, FcError, FcTail, fc_append_step,
                    fc_decode_attention, fc_decode_attention_noalloc,
                    fc_decode_plan, fc_decode_step,
                    fc_decode_workspace_bytes, fc_status_string,
-                   fc_storage_bytes, fc_workspace_status)
+                   fc_storage_bytes, fc_workspace_status, fc_read_view,
+                   fc_crop, fc_select_batch)
 from .archive import CodecKVCache, CodecStream, grown_capacity
 
 __all__ = [
@@ -21,5 +23,5 @@ __all__ = [
     "fc_archive_copy_prefix", "fc_decode_plan", "fc_decode_workspace_bytes",
     "fc_decode_attention", "fc_decode_attention_noalloc", "fc_decode_step",
     "fc_combine", "fc_workspace_status", "fc_storage_bytes",
-    "fc_status_string",
+    "fc_status_string", "fc_read_view", "fc_crop", "fc_select_batch",
 ]
