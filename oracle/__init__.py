@@ -19,8 +19,12 @@ flashcodec-kv 1.0.0 pages:
                    softmax (README "Materialization-free decode attention";
                    ``flashcodec/triton_attention.py`` module docstring), and its
                    split-K partials plus combine.
-* ``stream``    -- the raw-tail / capacity-doubling archive with append
+* ``stream``    -- the raw-tail / capacity-doubling archive with append,
+                   the reconstructed view, crop, batch gather and reset
                    (``flashcodec/cache.py`` ``_CodecStream``).
+* ``png``       -- the PNG-style lossless tier: per-block anchor and fp32
+                   first differences, cumulative-sum reconstruction, storage,
+                   and decode attention on the stored rows (README "Math").
 
 Every function is pinned by a ``-m "not gpu"`` test against something other
 than itself (library DCT, closed forms, brute force, the pages' printed
@@ -36,6 +40,9 @@ from .attention import (decode_attention_reference, coeff_decode_attention,
                         split_partials, combine_partials,
                         splitk_decode_attention, attend_archive)
 from .stream import CodecStreamOracle
+from .png import (png_filter, png_store, png_reconstruct, png_synthesis,
+                  png_rows, png_storage_bytes, png_decode_attention_reference,
+                  png_coeff_decode_attention, png_splitk_decode_attention)
 
 __all__ = [
     "dct_basis", "synthesis_basis", "split_blocks", "compress", "quantize",
@@ -44,4 +51,7 @@ __all__ = [
     "decode_attention_reference", "coeff_decode_attention", "split_partials",
     "combine_partials", "splitk_decode_attention", "attend_archive",
     "CodecStreamOracle",
+    "png_filter", "png_store", "png_reconstruct", "png_synthesis", "png_rows",
+    "png_storage_bytes", "png_decode_attention_reference",
+    "png_coeff_decode_attention", "png_splitk_decode_attention",
 ]
