@@ -1,0 +1,164 @@
+"""Host bookkeeping of the device cache binding (``archive.py``) on the CPU:
+libfc's launching calls are replaced by host fakes that only advance the
+descriptors as ``include/fc.h`` / ``include/fc_view.h`` document, so the
+memoised view (which blocks each read decodes, buffer growth), crop, batch
+gather (new storage, cleared plans) and reset are checked without a kernel."""
+
+import pytest
+import torch
+
+from compressed_decode_attention_blockwise_b200 import _lib
+from compressed_decode_attention_blockwise_b200.archive import CodecKVCache
+
+
+class FakeLib:
+    """Descriptor-level stand-ins for the calls archive.py makes."""
+
+    def __init__(self):
+        self.reads = []      # (first_block, n_blocks, tail len, out rows, ptr)
+        self.gathers = []
+
+    def fc_compress_blocks(self, x, arc, tail=None, stream=None):
+        T = x.shape[2]
+        if arc.n_blocks + T // arc.R > arc.capacity:
+            raise _lib.FcError(_lib.FC_ERR_CAPACITY, "fc_compress_blocks")
+        arc.n_blocks += T // arc.R
+        if tail is not None:
+            tail.len = T % arc.R
+
+    def fc_append_step(self, k, v, ka, va, kt, vt, stream=None):
+        if kt.len + 1 == ka.R:
+            if ka.n_blocks == ka.capacity:
+                raise _lib.FcError(_lib.FC_ERR_CAPACITY, "fc_append_step")
+            ka.n_blocks += 1
+            va.n_blocks += 1
+            kt.len = vt.len = 0
+        else:
+            kt.len += 1
+            vt.len += 1
+
+    def fc_archive_copy_prefix(self, src, dst, stream=None, device=None):
+        assert dst.capacity >= src.n_blocks
+        dst.n_blocks = src.n_blocks
+
+    def fc_read_view(self, arc, tail, first_block, out, stream=None):
+        assert 0 <= first_block <= arc.n_blocks
+        assert out.shape[2] >= arc.n_blocks * arc.R + tail.len
+        self.reads.append((first_block, arc.n_blocks, tail.len, out.shape[2],
+                           out.data_ptr()))
+
+    def fc_crop(self, arc, tail, tokens_to_remove, stream=None, device=None):
+        assert tokens_to_remove <= 0
+        keep = max(0, arc.n_blocks * arc.R + tail.len + tokens_to_remove)
+        kb, rest = divmod(keep, arc.R)
+        arc.n_blocks = min(arc.n_blocks, kb)
+        tail.len = rest
+
+    def fc_select_batch(self, src, src_tail, idx, dst, dst_tail, stream=None,
+                        device=None):
+        assert all(0 <= i < src.B for i in idx) and dst.B == len(idx)
+        assert dst.capacity >= src.n_blocks
+        self.gathers.append(list(idx))
+        dst.n_blocks = src.n_blocks
+        dst_tail.len = src_tail.len
+
+
+@pytest.fixture
+def fake(monkeypatch):
+    f = FakeLib()
+    for name in ("fc_compress_blocks", "fc_append_step",
+                 "fc_archive_copy_prefix", "fc_read_view", "fc_crop",
+                 "fc_select_batch"):
+        monkeypatch.setattr(_lib, name, getattr(f, name))
+    return f
+
+
+def _cache(B=2, H=2, D=32, R=8):
+    return CodecKVCache(B, H, D, R, 2, device="cpu")
+
+
+def _tokens(c, T):
+    return (torch.zeros((c.B, c.Hk, T, c.D), dtype=torch.bfloat16),
+            torch.zeros((c.B, c.Hk, T, c.D), dtype=torch.bfloat16))
+
+
+def test_view_decodes_each_block_once_and_grows_by_doubling(fake):
+    c = _cache()
+    assert c.read() == (None, None)                 # empty: nothing to read
+    c.prefill(*_tokens(c, 5))
+    kv, vv = c.read()                               # tail only: the tail itself
+    assert kv.shape == (2, 2, 5, 32) and not fake.reads
+    c.prefill(*_tokens(c, 8 * 14 + 6))              # 15 blocks + 3 raw
+    kv, vv = c.read()
+    assert kv.shape[2] == vv.shape[2] == 8 * 15 + 3
+    kv = c.k.read()                                 # nothing new to decode
+    assert fake.reads[-1][:4] == (15, 15, 3, 16 * 8)  # first buffer: 16 blocks
+    assert fake.reads[-3][:4] == (0, 15, 3, 16 * 8)   # K's first read
+    ptr = fake.reads[-1][4]
+    for _ in range(5):                              # completes block 16
+        c.append(*_tokens(c, 1))
+    c.k.read()
+    assert fake.reads[-1][:4] == (15, 16, 0, 128)   # only the new block
+    assert fake.reads[-1][4] == ptr
+    c.append(*_tokens(c, 1))                        # 129 tokens > 128 rows
+    view = c.k.read()
+    assert view.shape[2] == 129
+    assert fake.reads[-1][:4] == (0, 16, 1, 256)    # doubled, decoded afresh
+    assert fake.reads[-1][4] != ptr
+
+
+def test_crop_rewinds_the_memoised_view(fake):
+    c = _cache()
+    c.prefill(*_tokens(c, 8 * 20 + 5))
+    c.read()
+    with pytest.raises(ValueError):
+        c.crop(3)
+    c.crop(-2)                                      # tail only
+    assert (c.k.n_blocks, c.k.tail_len, c.k._rec_blocks) == (20, 3, 20)
+    c.crop(-30)                                     # 133 tokens: 16 blocks + 5
+    assert (c.k.n_blocks, c.k.tail_len, c.v.tail_len) == (16, 5, 5)
+    assert c.k._rec_blocks == 16
+    c.k.read()
+    assert fake.reads[-1][:3] == (16, 16, 5)        # nothing re-decoded
+    c.crop(-1000)
+    assert c.seq_len == 0 and c.read() == (None, None)
+
+
+def test_batch_gather_replaces_storage_and_plans(fake):
+    c = _cache(B=3)
+    c.prefill(*_tokens(c, 8 * 20 + 5))
+    c.read()
+    c._plans[(8, 20)] = 4
+    c._ws_need[(8, 4)] = 1 << 20
+    cap = c.k.capacity
+    old_ptr = c.k.coeffs.data_ptr()
+    c.reorder_cache(torch.tensor([2, 0, 2, 1]))
+    assert fake.gathers[-2:] == [[2, 0, 2, 1], [2, 0, 2, 1]]   # K and V
+    assert c.B == c.k.B == c.v.B == 4
+    assert c.k.coeffs.shape == (4, 2, cap, 2, 32) and c.k.capacity == cap
+    assert c.k.scales.shape == (4, 2, cap, 2)
+    assert c.k.tail.shape == (4, 2, 8, 32)
+    assert c.k.arc.coeffs == c.k.coeffs.data_ptr() != old_ptr
+    assert c.k.tail_desc.data == c.k.tail.data_ptr()
+    assert (c.k.n_blocks, c.k.tail_len) == (20, 5)
+    assert c.k._rec is None and not c._plans and not c._ws_need
+    c.batch_select_indices([3, 0])
+    assert c.B == 2 and fake.gathers[-1] == [3, 0]
+    c.batch_repeat_interleave(3)
+    assert c.B == 6 and fake.gathers[-1] == [0, 0, 0, 1, 1, 1]
+    kv, vv = c.read()
+    assert kv.shape == (6, 2, 165, 32)
+    assert fake.reads[-1][0] == 0                   # rebuilt from block 0
+
+
+def test_reset_keeps_capacity_and_update_returns_the_view(fake):
+    c = _cache()
+    c.prefill(*_tokens(c, 8 * 40 + 1))
+    c.read()
+    cap = c.k.capacity
+    c.reset()
+    assert (c.seq_len, c.k.capacity, c.k._rec_blocks) == (0, cap, 0)
+    kv, vv = c.update(*_tokens(c, 8 * 3 + 2))
+    assert kv.shape == (2, 2, 26, 32) and c.get_seq_length() == 26
+    assert fake.reads[-1][:3] == (0, 3, 2)
+
