@@ -180,9 +180,11 @@ class CodecStream:
         """Batch row i becomes row ``idx[i]`` (``_CodecStream.select_batch``):
         the archive and the raw tail are gathered by libfc into new storage
         of the same capacity; the view is rebuilt by the next ``read``."""
-        if isinstance(idx, torch.Tensor):
-            idx = idx.tolist()
-        idx = [int(i) for i in idx]
+        self._adopt(self._gathered(host_indices(idx)))
+
+    def _gathered(self, idx):
+        """New storage holding batch rows ``idx`` of this stream, filled by
+        libfc; the stream itself is not changed."""
         coeffs, scales, arc = self._storage(len(idx), self.capacity)
         tail = torch.zeros((len(idx), self.H, self.R, self.D),
                            dtype=self.token_dtype, device=self.device)
@@ -193,9 +195,11 @@ class CodecStream:
         td.stride_b, td.stride_h = tail.stride(0), tail.stride(1)
         _lib.fc_select_batch(self.arc, self.tail_desc, idx, arc, td,
                              device=self.device)
-        self.B = len(idx)
-        self.coeffs, self.scales, self.arc = coeffs, scales, arc
-        self.tail, self.tail_desc = tail, td
+        return len(idx), coeffs, scales, arc, tail, td
+
+    def _adopt(self, gathered):
+        (self.B, self.coeffs, self.scales, self.arc, self.tail,
+         self.tail_desc) = gathered
         self.discard_view()
 
     def reset(self):
@@ -204,6 +208,13 @@ class CodecStream:
         self.arc.n_blocks = 0
         self.tail_desc.len = 0
         self._rec_blocks = 0
+
+
+def host_indices(idx):
+    """Batch indices as a list of Python ints (a tensor is read back)."""
+    if isinstance(idx, torch.Tensor):
+        idx = idx.tolist()
+    return [int(i) for i in idx]
 
 
 def ctypes_copy(dst, src):
@@ -366,9 +377,14 @@ class CodecKVCache:
         self.v.crop(tokens_to_remove)
 
     def select_batch(self, idx):
-        """Gather batch rows of both streams (archives and raw tails)."""
-        self.k.select_batch(idx)
-        self.v.select_batch(idx)
+        """Gather batch rows of both streams (archives and raw tails); both
+        are gathered before either is replaced, so a failure leaves the
+        cache as it was."""
+        idx = host_indices(idx)
+        gk = self.k._gathered(idx)
+        gv = self.v._gathered(idx)
+        self.k._adopt(gk)
+        self.v._adopt(gv)
         self.B = self.k.B
         self._plans.clear()
         self._ws_need.clear()

@@ -162,3 +162,24 @@ def test_reset_keeps_capacity_and_update_returns_the_view(fake):
     assert kv.shape == (2, 2, 26, 32) and c.get_seq_length() == 26
     assert fake.reads[-1][:3] == (0, 3, 2)
 
+
+
+def test_failed_gather_leaves_the_cache_unchanged(fake, monkeypatch):
+    c = _cache(B=3)
+    c.prefill(*_tokens(c, 8 * 5 + 2))
+    k_arc, v_arc = c.k.arc, c.v.arc
+    calls = []
+
+    def failing(src, src_tail, idx, dst, dst_tail, stream=None, device=None):
+        calls.append(idx)
+        if len(calls) == 2:                         # the V stream
+            raise _lib.FcError(_lib.FC_ERR_CUDA, "fc_select_batch")
+        dst.n_blocks = src.n_blocks
+        dst_tail.len = src_tail.len
+
+    monkeypatch.setattr(_lib, "fc_select_batch", failing)
+    with pytest.raises(_lib.FcError):
+        c.reorder_cache([1, 0])
+    assert c.B == c.k.B == c.v.B == 3
+    assert c.k.arc is k_arc and c.v.arc is v_arc
+    assert c.k.coeffs.shape[0] == c.v.coeffs.shape[0] == 3
