@@ -20,7 +20,7 @@ Three paths that must agree to rounding:
   (max, sum, acc) partial, merged by the flash-decoding combine
   (``flashcodec/triton_attention.py``, split and combine kernels).
 
-Readings (listed in the design doc): the softmax scale defaults to D**-0.5
+Readings where the pages are silent: the softmax scale defaults to D**-0.5
 (``codec_decode_attention_triton``); a chunk with no blocks and no tail
 contributes (m=-inf, l=0) and the combine skips it instead of producing NaN.
 """

@@ -14,7 +14,7 @@ Sources (flashcodec-kv 1.0.0):
 * ``flashcodec/cache.py``, ``_CodecStream.append``: only complete blocks are
   archived; the remainder stays raw.
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 * c_0 = sqrt(1/R), c_j = sqrt(2/R): the normalisation that makes the rows
   orthonormal, i.e. the standard orthonormal DCT-II.
 * scale = max_d |C| / 127, code = clamp(round_half_even(C / scale), -127, 127);

@@ -17,7 +17,7 @@ Sources (flashcodec-kv 1.0.0):
 * README, mode table and "Cache footprint & latency": the tier is lossless
   at keep_ratio = 1.0 and costs 188 % of bf16 KV (100 % of fp32 KV).
 
-Readings where the pages are silent (each listed in the design doc):
+Readings where the pages are silent:
 * Only the lossless tier (keep_ratio = 1.0) is modelled: the Top-M filter
   used below 1.0 is named on the pages but never defined.
 * The stored delta is the exact difference of the two stored token values,
