@@ -45,7 +45,7 @@ EXPORTS = (
     "fc_decode_plan", "fc_decode_workspace_bytes", "fc_decode_attention",
     "fc_combine", "fc_decode_attention_noalloc", "fc_workspace_status",
     "fc_storage_bytes", "fc_status_string", "fc_decode_step",
-    "fc_read_view", "fc_crop", "fc_select_batch",
+    "fc_read_view", "fc_crop", "fc_select_batch", "fc_noalloc_status",
 )
 
 
@@ -120,6 +120,8 @@ def load() -> ctypes.CDLL:
         "fc_workspace_status": (ctypes.c_int, [P, ctypes.c_size_t,
                                                ctypes.POINTER(ctypes.c_uint32),
                                                P]),
+        "fc_noalloc_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32),
+                                             P]),
         "fc_storage_bytes": (ctypes.c_int64, [PA, PT]),
         "fc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "fc_read_view": (ctypes.c_int, [PA, PT, I64, P, I32, PI64, I64, P]),
@@ -300,6 +302,18 @@ def fc_workspace_status(workspace: torch.Tensor, stream=None) -> int:
         ctypes.byref(v), _stream(stream, workspace))
     if st not in (FC_OK, FC_ERR_DEVICE):
         _check(st, "fc_workspace_status")
+    return int(v.value)
+
+
+def fc_noalloc_status(stream=None, device=None) -> int:
+    """Status word of fc_decode_attention_noalloc's static scratch on the
+    current device (0 = no error reported); reading clears it."""
+    v = ctypes.c_uint32(0)
+    s = _stream(stream) if stream is not None or device is None else \
+        ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = load().fc_noalloc_status(ctypes.byref(v), s)
+    if st not in (FC_OK, FC_ERR_DEVICE):
+        _check(st, "fc_noalloc_status")
     return int(v.value)
 
 

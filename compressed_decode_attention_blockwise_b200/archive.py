@@ -137,17 +137,19 @@ class CodecStream:
         (``_CodecStream.read``): archived blocks decompressed by libfc, then
         the raw tail. Each archived block is decoded once into a persistent
         buffer (append-only memoisation); ``None`` for an empty stream, the
-        tail itself when nothing is archived. The returned tensor aliases
-        that buffer: rows below ``n_blocks * R`` keep their values until a
-        crop, batch gather or reset, while the raw-tail rows after them are
-        rewritten by the next read (with the decoded block once it is
-        archived)."""
+        tail itself when nothing is archived. Without raw tokens the returned
+        tensor aliases that buffer (its rows keep their values until a crop,
+        batch gather or reset); with raw tokens it is a fresh tensor (the
+        decoded prefix copied, the tail rows written by libfc), so a tensor
+        handed out earlier never changes when a later read archives those
+        tail tokens."""
         T = self.seq_len
         if T == 0:
             return None
         if self.n_blocks == 0:
             return self.live_tail()
-        need = -(-T // self.R) * self.R
+        nb = self.n_blocks
+        need = nb * self.R
         if self._rec is None or self._rec.shape[2] < need:
             old = 0 if self._rec is None else self._rec.shape[2]
             rows = max(need, 2 * old, INITIAL_BLOCKS * self.R)
@@ -155,10 +157,16 @@ class CodecStream:
                                     dtype=self.token_dtype,
                                     device=self.device)
             self._rec_blocks = 0   # a new buffer is decoded from block 0
-        _lib.fc_read_view(self.arc, self.tail_desc, self._rec_blocks,
-                          self._rec)
-        self._rec_blocks = self.n_blocks
-        return self._rec[:, :, :T]
+        if self._rec_blocks < nb:
+            _lib.fc_read_view(self.arc, None, self._rec_blocks, self._rec)
+        self._rec_blocks = nb
+        if self.tail_len == 0:
+            return self._rec[:, :, :T]
+        out = torch.empty((self.B, self.H, T, self.D), dtype=self.token_dtype,
+                          device=self.device)
+        out[:, :, :need].copy_(self._rec[:, :, :need])
+        _lib.fc_read_view(self.arc, self.tail_desc, nb, out)
+        return out
 
     def discard_view(self):
         """Free the reconstructed view (rebuilt by the next ``read``)."""
@@ -372,9 +380,24 @@ class CodecKVCache:
 
     def crop(self, tokens_to_remove: int):
         """Exact removal of trailing tokens from both streams (negative count,
-        e.g. rejected speculative tokens)."""
+        e.g. rejected speculative tokens). If the V crop fails, K is put back
+        as it was (descriptors and raw tail rows), so the two streams never
+        disagree on length."""
+        if tokens_to_remove > 0:
+            raise ValueError("crop takes a negative count of tokens to remove")
+        if (self.k.n_blocks, self.k.tail_len) != \
+                (self.v.n_blocks, self.v.tail_len):
+            raise RuntimeError("K and V streams disagree on length")
+        saved = (self.k.arc.n_blocks, self.k.tail_desc.len,
+                 self.k._rec_blocks, self.k.tail.clone())
         self.k.crop(tokens_to_remove)
-        self.v.crop(tokens_to_remove)
+        try:
+            self.v.crop(tokens_to_remove)
+        except Exception:
+            (self.k.arc.n_blocks, self.k.tail_desc.len, self.k._rec_blocks,
+             tail) = saved
+            self.k.tail.copy_(tail)
+            raise
 
     def select_batch(self, idx):
         """Gather batch rows of both streams (archives and raw tails); both

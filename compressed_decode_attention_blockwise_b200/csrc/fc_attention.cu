@@ -345,10 +345,20 @@ extern "C" int fc_decode_attention_noalloc(const void* q, int32_t q_dtype, const
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != FC_OK) return st;
-  // the status word and the tickets must start at zero; the array keeps
-  // whatever the previous call left
-  if (cudaMemsetAsync(scratch, 0, wl.m, stream) != cudaSuccess) return FC_ERR_CUDA;
+  // the tickets must start at zero (the array keeps whatever the previous
+  // call left); the status word is not cleared here, so that an error a
+  // kernel reported stays readable through fc_noalloc_status
+  if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + wl.tickets, 0, wl.m - wl.tickets, stream) != cudaSuccess)
+    return FC_ERR_CUDA;
   return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, ns,
                              FC_DECODE_FUSE_COMBINE, scratch, FC_NOALLOC_SCRATCH_BYTES, out, out_dtype,
                              out_strides, stream);
+}
+
+extern "C" int fc_noalloc_status(uint32_t* device_status, fc_stream stream) {
+  if (!device_status) return FC_ERR_INVALID;
+  void* scratch = nullptr;
+  const int st = noalloc_scratch(&scratch);
+  if (st != FC_OK) return st;
+  return fc_workspace_status(scratch, FC_NOALLOC_SCRATCH_BYTES, device_status, stream);
 }

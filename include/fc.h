@@ -307,10 +307,12 @@ int fc_combine(const void* workspace, size_t workspace_bytes, int64_t B,
  * first call on a device resolves the array's device address with
  * cudaGetSymbolAddress (once per device, with that device current); make that
  * first call before any stream capture. Every call shares the array and
- * clears its status word and tickets on `stream` before the kernel, so calls
- * whose executions overlap on the GPU (other streams, other host threads)
- * race; serialise them. Arguments and results as in fc_decode_attention;
- * returns FC_ERR_SCRATCH_LIMIT, launching nothing, when
+ * clears its tickets on `stream` before the kernel, so calls whose executions
+ * overlap on the GPU (other streams, other host threads) race; serialise
+ * them. The array's status word is not cleared by these calls: a kernel error
+ * (a bounded wait that gave up) stays recorded until fc_noalloc_status reads
+ * and clears it. Arguments and results as in fc_decode_attention; returns
+ * FC_ERR_SCRATCH_LIMIT, launching nothing, when
  * fc_decode_workspace_bytes(B, Hq, D, splits) exceeds the array.
  */
 #define FC_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
@@ -319,6 +321,15 @@ int fc_decode_attention_noalloc(const void* q, int32_t q_dtype, const int64_t* q
                                 const fc_tail* kt, const fc_tail* vt, float softmax_scale,
                                 int32_t num_splits, void* out, int32_t out_dtype,
                                 const int64_t* out_strides, fc_stream stream);
+
+/*
+ * fc_noalloc_status -- fc_workspace_status for the static scratch array of
+ * fc_decode_attention_noalloc on the current device: synchronises `stream`,
+ * stores the status word in *device_status (0 = no fc_decode_attention_noalloc
+ * kernel on this device reported a problem since the last read) and clears
+ * it. Returns FC_ERR_DEVICE when it was nonzero. Allocates nothing.
+ */
+int fc_noalloc_status(uint32_t* device_status, fc_stream stream);
 
 /*
  * fc_workspace_status -- synchronise `stream`, read the workspace status word

@@ -42,10 +42,16 @@ class FakeLib:
         dst.n_blocks = src.n_blocks
 
     def fc_read_view(self, arc, tail, first_block, out, stream=None):
+        n_raw = 0 if tail is None else tail.len
         assert 0 <= first_block <= arc.n_blocks
-        assert out.shape[2] >= arc.n_blocks * arc.R + tail.len
-        self.reads.append((first_block, arc.n_blocks, tail.len, out.shape[2],
+        assert out.shape[2] >= arc.n_blocks * arc.R + n_raw
+        self.reads.append((first_block, arc.n_blocks, n_raw, out.shape[2],
                            out.data_ptr()))
+        # marker values: block n's rows hold n + 1, raw token i holds -(i + 1)
+        for n in range(first_block, arc.n_blocks):
+            out[:, :, n * arc.R:(n + 1) * arc.R] = n + 1
+        for i in range(n_raw):
+            out[:, :, arc.n_blocks * arc.R + i] = -(i + 1)
 
     def fc_crop(self, arc, tail, tokens_to_remove, stream=None, device=None):
         assert tokens_to_remove <= 0
@@ -91,20 +97,42 @@ def test_view_decodes_each_block_once_and_grows_by_doubling(fake):
     c.prefill(*_tokens(c, 8 * 14 + 6))              # 15 blocks + 3 raw
     kv, vv = c.read()
     assert kv.shape[2] == vv.shape[2] == 8 * 15 + 3
+    assert fake.reads[-4][:4] == (0, 15, 0, 16 * 8)   # K's blocks: 16-block buffer
+    assert fake.reads[-3][:4] == (15, 15, 3, 123)     # K's tail: a fresh tensor
+    ptr = fake.reads[-4][4]
     kv = c.k.read()                                 # nothing new to decode
-    assert fake.reads[-1][:4] == (15, 15, 3, 16 * 8)  # first buffer: 16 blocks
-    assert fake.reads[-3][:4] == (0, 15, 3, 16 * 8)   # K's first read
-    ptr = fake.reads[-1][4]
+    assert fake.reads[-1][:4] == (15, 15, 3, 123) and fake.reads[-1][4] != ptr
+    n = len(fake.reads)
     for _ in range(5):                              # completes block 16
         c.append(*_tokens(c, 1))
-    c.k.read()
-    assert fake.reads[-1][:4] == (15, 16, 0, 128)   # only the new block
-    assert fake.reads[-1][4] == ptr
-    c.append(*_tokens(c, 1))                        # 129 tokens > 128 rows
+    view = c.k.read()
+    assert fake.reads[n:] == [(15, 16, 0, 128, ptr)]  # only the new block
+    assert view.data_ptr() == ptr and view.shape[2] == 128
+    c.append(*_tokens(c, 1))                        # 129 tokens: one raw
     view = c.k.read()
     assert view.shape[2] == 129
-    assert fake.reads[-1][:4] == (0, 16, 1, 256)    # doubled, decoded afresh
+    assert fake.reads[-1][:4] == (16, 16, 1, 129)   # tail rows only
+    for _ in range(7):                              # 17 blocks > 16 in the buffer
+        c.append(*_tokens(c, 1))
+    view = c.k.read()
+    assert fake.reads[-1][:4] == (0, 17, 0, 256)    # doubled, decoded afresh
     assert fake.reads[-1][4] != ptr
+
+
+def test_view_handed_out_earlier_keeps_its_tail_rows(fake):
+    """A read with raw tokens returns a fresh tensor: when those tokens are
+    archived later, the earlier tensor still holds the raw rows
+    (flashcodec/cache.py, _CodecStream.read)."""
+    c = _cache()
+    c.prefill(*_tokens(c, 8 * 15 + 3))
+    early = c.k.read()
+    assert early[0, 0, 120:123, 0].tolist() == [-1, -2, -3]
+    for _ in range(5):                              # archives tokens 120..127
+        c.append(*_tokens(c, 1))
+    later = c.k.read()
+    assert later[0, 0, 120:128, 0].tolist() == [16] * 8
+    assert early[0, 0, 120:123, 0].tolist() == [-1, -2, -3]
+    assert early[0, 0, :120, 0].tolist() == later[0, 0, :120, 0].tolist()
 
 
 def test_crop_rewinds_the_memoised_view(fake):
@@ -119,7 +147,7 @@ def test_crop_rewinds_the_memoised_view(fake):
     assert (c.k.n_blocks, c.k.tail_len, c.v.tail_len) == (16, 5, 5)
     assert c.k._rec_blocks == 16
     c.k.read()
-    assert fake.reads[-1][:3] == (16, 16, 5)        # nothing re-decoded
+    assert fake.reads[-1][:3] == (16, 16, 5)        # tail rows only
     c.crop(-1000)
     assert c.seq_len == 0 and c.read() == (None, None)
 
@@ -148,7 +176,7 @@ def test_batch_gather_replaces_storage_and_plans(fake):
     assert c.B == 6 and fake.gathers[-1] == [0, 0, 0, 1, 1, 1]
     kv, vv = c.read()
     assert kv.shape == (6, 2, 165, 32)
-    assert fake.reads[-1][0] == 0                   # rebuilt from block 0
+    assert fake.reads[-4][:2] == (0, 20)            # rebuilt from block 0
 
 
 def test_reset_keeps_capacity_and_update_returns_the_view(fake):
@@ -160,7 +188,8 @@ def test_reset_keeps_capacity_and_update_returns_the_view(fake):
     assert (c.seq_len, c.k.capacity, c.k._rec_blocks) == (0, cap, 0)
     kv, vv = c.update(*_tokens(c, 8 * 3 + 2))
     assert kv.shape == (2, 2, 26, 32) and c.get_seq_length() == 26
-    assert fake.reads[-1][:3] == (0, 3, 2)
+    assert fake.reads[-4][:3] == (0, 3, 0)          # K's blocks from block 0
+    assert fake.reads[-3][:3] == (3, 3, 2)          # then its tail rows
 
 
 
@@ -183,3 +212,25 @@ def test_failed_gather_leaves_the_cache_unchanged(fake, monkeypatch):
     assert c.B == c.k.B == c.v.B == 3
     assert c.k.arc is k_arc and c.v.arc is v_arc
     assert c.k.coeffs.shape[0] == c.v.coeffs.shape[0] == 3
+
+
+def test_failed_crop_leaves_both_streams_as_they_were(fake, monkeypatch):
+    c = _cache()
+    c.prefill(*_tokens(c, 8 * 6 + 5))
+    c.k.tail.fill_(3.0)
+    calls = []
+
+    def failing(arc, tail, tokens_to_remove, stream=None, device=None):
+        calls.append(tokens_to_remove)
+        if len(calls) == 2:                         # the V stream
+            raise _lib.FcError(_lib.FC_ERR_CUDA, "fc_crop")
+        fake.fc_crop(arc, tail, tokens_to_remove)
+        c.k.tail.fill_(7.0)                         # the boundary rows rewritten
+
+    monkeypatch.setattr(_lib, "fc_crop", failing)
+    with pytest.raises(_lib.FcError):
+        c.crop(-9)
+    assert (c.k.n_blocks, c.k.tail_len) == (c.v.n_blocks, c.v.tail_len) == (6, 5)
+    assert torch.all(c.k.tail == 3.0)
+    with pytest.raises(ValueError):
+        c.crop(1)

@@ -5,7 +5,8 @@ workspace (a C host inside a fixed device-memory budget without an allocator,
 or a serving loop that must not call cudaMalloc per step). It must give the
 same result as fc_decode_attention with a caller workspace, call after call
 (the static scratch it shares between calls keeps the previous call's bytes),
-and reject requests larger than its scratch. This file is collected last so
+and reject requests larger than its scratch; the status word of that
+scratch stays readable through fc_noalloc_status. This file is collected last so
 that a run stopping at the first failure has already run every other test.
 """
 
@@ -42,6 +43,9 @@ def test_noalloc_matches_workspace_entry_point(w):
                                          out)
         torch.cuda.synchronize()
         check_out(f64(out), f64(ref), "noalloc vs workspace")
+        # no kernel reported an error in the scratch's status word, which
+        # the calls themselves never clear (reading it does)
+        assert _lib.fc_noalloc_status() == 0
 
 
 def test_noalloc_rejects_requests_beyond_its_scratch():
