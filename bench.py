@@ -199,6 +199,95 @@ def attention_bytes(cache, Hq: int, q_elem: int, out_elem: int) -> int:
     return b + cache.B * Hq * cache.D * (q_elem + out_elem)
 
 
+ROOF_LAUNCHES = 600
+# fc_decode_attention flag modes of the roofline legs: (overlap, q_final)
+MODES = {"isolated": (False, False), "overlap": (True, False),
+         "overlap_q_final": (True, True)}
+
+
+def attention_modes(caches, q_pool, out_bufs, n_launch, W, world,
+                    modes=MODES):
+    """Mean per-launch time of fc_decode_attention in each flag mode: one
+    CUDA graph of ``n_launch`` launches over the archive copies round-robin
+    (each launch reads a different copy than the previous one), timed with
+    CUDA events on the launching stream after W warm-up replays.
+    isolated: no flags, each launch starts after the previous one completed;
+    overlap: FC_DECODE_OVERLAP, the next launch streams its archive while the
+    previous drains (valid in any decode loop); overlap_q_final: also
+    FC_DECODE_Q_FINAL (q final before the previous launch started)."""
+    copies = len(caches)
+    ev0, ev1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    res = {}
+    for name, (ov, qf) in modes.items():
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(n_launch):
+                c = i % copies
+                caches[c].attention(q_pool[i % len(q_pool)], out=out_bufs[c],
+                                    overlap=ov, q_final=qf)
+        for _ in range(max(W, 3)):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        ev0.record()
+        g.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        res[name] = max_over_ranks(ev0.elapsed_time(ev1) / 1e3 / n_launch,
+                                   world)
+        del g
+    return res
+
+
+def bench_workload(name, peak, W, world, dev, l2, budget_s=0.25):
+    """Decode-attention throughput of one more workload at its full size
+    (archive copies round-robin above twice the L2), in the three flag
+    modes; the number of launches per graph keeps each replay near
+    ``budget_s``."""
+    from compressed_decode_attention_blockwise_b200 import CodecKVCache
+    w = synth.WORKLOADS[name]
+    tok_dt = synth.torch_dtype(w.in_dtype)
+    esz = torch.tensor([], dtype=tok_dt).element_size()
+    data = synth.generate(w.replace(steps=0), q_steps=Q_POOL)
+    kd, vd = data["k"].to(dev), data["v"].to(dev)
+    del data["k"], data["v"]
+    arc_bytes = None
+    caches = []
+    while True:
+        c = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, w.k_coeff, w.v_coeff,
+                         token_dtype=tok_dt, device=dev)
+        c.prefill(kd[:, :, :w.T], vd[:, :, :w.T])
+        caches.append(c)
+        arc_bytes = c.storage_bytes()
+        if len(caches) * arc_bytes > 2 * l2:
+            break
+    del kd, vd
+    q_pool = data["q"].to(dev)
+    outs = [torch.empty((w.B, w.Hq, 1, w.D), dtype=torch.float32,
+                        device=dev) for _ in caches]
+    for i, c in enumerate(caches):
+        c.attention(q_pool[0], out=outs[i])
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    caches[0].attention(q_pool[0], out=outs[0])
+    torch.cuda.synchronize()
+    one = max(time.perf_counter() - t0, 1e-6)
+    n = int(max(20, min(ROOF_LAUNCHES, budget_s / one)))
+    modes = attention_modes(caches, q_pool, outs, n, W, world)
+    nbytes = attention_bytes(caches[0], w.Hq, esz, 4)
+    entry = {"bytes_per_launch": int(nbytes), "launches": n,
+             "archive_copies": len(caches),
+             "kernel": "tensor-core" if caches[0].tensor_core_path(w.Hq)
+             else "cuda-core"}
+    for m, t in modes.items():
+        entry[m] = {"us_per_launch": round(t * 1e6, 3),
+                    "GB_per_s": round(nbytes / t / 1e9, 2),
+                    "frac": round(nbytes / t / 1e9 / peak, 4)}
+    del caches, outs
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_fc(args, world, rank, local):
     from compressed_decode_attention_blockwise_b200 import CodecKVCache, _lib
 
@@ -292,45 +381,15 @@ def run_fc(args, world, rank, local):
         c.attention(q_pool[0], out=out_bufs[i])
     torch.cuda.synchronize()
 
-    # ---------------- attention-only graph: per-launch duration (roofline)
+    # ---------------- attention-only graphs: per-launch duration (roofline)
+    # ROOF_LAUNCHES launches whatever --steps is, so that the first launch of
+    # a replay (which cannot overlap the previous replay) weighs little
     att_bytes = [attention_bytes(c, Hq, esz, 4) for c in caches]
-    g_att = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_att):
-        for i in range(K):
-            c = i % copies
-            caches[c].attention(q_pool[i % Q_POOL], out=out_bufs[c],
-                                overlap=True, q_final=True)
-    for _ in range(max(W, 3)):
-        g_att.replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record()
-    g_att.replay()
-    ev1.record()
-    torch.cuda.synchronize()
-    att_launch_s = max_over_ranks(ev0.elapsed_time(ev1) / 1e3 / K, world)
-    att_bytes_mean = sum(att_bytes[i % copies] for i in range(K)) / K
-    del g_att
-
-    # the same launches without the overlap flags: each launch starts after
-    # the previous one has completed (the kernel's own duration, launch gaps
-    # included)
-    K_iso = min(K, 2000)
-    g_iso = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_iso):
-        for i in range(K_iso):
-            c = i % copies
-            caches[c].attention(q_pool[i % Q_POOL], out=out_bufs[c])
-    for _ in range(max(W, 3)):
-        g_iso.replay()
-    torch.cuda.synchronize()
-    barrier(world)
-    ev0.record()
-    g_iso.replay()
-    ev1.record()
-    torch.cuda.synchronize()
-    iso_launch_s = max_over_ranks(ev0.elapsed_time(ev1) / 1e3 / K_iso, world)
-    del g_iso
+    modes = attention_modes(caches, q_pool, out_bufs, ROOF_LAUNCHES, W, world)
+    att_launch_s = modes["overlap_q_final"]
+    iso_launch_s = modes["isolated"]
+    att_bytes_mean = sum(att_bytes[i % copies]
+                         for i in range(ROOF_LAUNCHES)) / ROOF_LAUNCHES
 
     # ---------------- decode steps (append + attention), CUDA graph
     step_bytes = []
@@ -447,16 +506,20 @@ def run_fc(args, world, rank, local):
             "traffic": profiled_traffic("decode_attention_%s.md" % w.name),
             "bytes_per_launch": int(att_bytes_mean),
             "us_per_launch": round(att_launch_s * 1e6, 3),
-            "timing": "mean over K back-to-back launches with FC_DECODE_OVERLAP"
+            "launches": ROOF_LAUNCHES,
+            "timing": "mean over %d back-to-back launches (one CUDA-graph "
+                      "replay, independent of --steps) with FC_DECODE_OVERLAP"
                       " | FC_DECODE_Q_FINAL (each launch's start overlaps the "
-                      "previous one's drain; independent archives)",
-            "isolated": {
-                "us_per_launch": round(iso_launch_s * 1e6, 3),
-                "achieved": round(att_bytes_mean / iso_launch_s / 1e9, 2),
-                "frac": round(att_bytes_mean / iso_launch_s / 1e9 / peak, 4),
-                "timing": "the same launches without overlap flags: each "
-                          "starts after the previous one completed",
-            },
+                      "previous one's drain; independent archives)"
+                      % ROOF_LAUNCHES,
+            "modes": {m: {"us_per_launch": round(t * 1e6, 3),
+                          "achieved": round(att_bytes_mean / t / 1e9, 2),
+                          "frac": round(att_bytes_mean / t / 1e9 / peak, 4)}
+                      for m, t in modes.items()},
+            "modes_note": "isolated: no flags, each launch starts after the "
+                          "previous one completed; overlap: FC_DECODE_OVERLAP "
+                          "only (the dependency a layer-by-layer decode "
+                          "has); overlap_q_final: the headline mode",
         },
         "compress": {
             "tokens_per_s": round(w.B * w.T / comp_s, 1),
@@ -483,6 +546,12 @@ def run_fc(args, world, rank, local):
         "gpu_launches": K,
         "clocks": clk.summary(),
     }
+    if args.workloads:
+        wl = {}
+        for name in args.workloads.split(","):
+            if name and name != w.name:
+                wl[name] = bench_workload(name, peak, W, world, dev, l2)
+        res["workloads"] = wl
     return res
 
 
@@ -525,13 +594,33 @@ def prepare_oracle_sample(w, blocks=None, heads=((0, 0),)):
     return arc
 
 
+def host_cores():
+    """Host cores this process may run on."""
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def blas_limit(n=1):
+    """Context that pins the BLAS / OpenMP pools to n threads (the oracle's
+    einsums then run on one core), or a no-op without threadpoolctl."""
+    try:
+        from threadpoolctl import threadpool_limits
+        return threadpool_limits(limits=n)
+    except Exception:
+        import contextlib
+        return contextlib.nullcontext()
+
+
 def cpu_cores_used():
+    """(threads the oracle runs on, host cores available, BLAS pools)."""
     try:
         from threadpoolctl import threadpool_info
         blas = [p.get("num_threads", 1) for p in threadpool_info()]
     except Exception:
         blas = []
-    return 1, blas
+    return 1, host_cores(), blas
 
 
 def run_cpu_baseline(w, budget_s=10.0):
@@ -540,25 +629,27 @@ def run_cpu_baseline(w, budget_s=10.0):
     heads = [(0, h) for h in range(w.Hk)]
     arc = prepare_oracle_sample(w, blocks=min(w.n_blocks, 2048),
                                 heads=heads[:1])
-    t0 = time.perf_counter()
-    nbytes = 0
-    reps = 0
-    while True:
-        nbytes += oracle_sample_step(arc, None, list(arc), w.R)
-        reps += 1
-        if time.perf_counter() - t0 >= budget_s or reps >= 50:
-            break
-    dt = time.perf_counter() - t0
-    cores, blas = cpu_cores_used()
+    with blas_limit(1):
+        cores, avail, blas = cpu_cores_used()
+        t0 = time.perf_counter()
+        nbytes = 0
+        reps = 0
+        while True:
+            nbytes += oracle_sample_step(arc, None, list(arc), w.R)
+            reps += 1
+            if time.perf_counter() - t0 >= budget_s or reps >= 50:
+                break
+        dt = time.perf_counter() - t0
     nb = min(w.n_blocks, 2048)
     return {"value": round(nbytes / dt / 1e9, 6), "unit": "GB/s",
-            "cores": cores, "kind": "oracle",
+            "cores": cores, "host_cores": avail, "blas_threads": blas,
+            "kind": "oracle",
             "sample": "%d x decode attention of 1 kv head (%d q heads) over "
                       "the first %d blocks + %d tail tokens of the %s "
                       "workload, decompress-then-softmax in float64 "
-                      "(%.1f s); numpy einsum runs on one thread%s"
-                      % (reps, w.G, nb, w.n_tail, w.name, dt,
-                         "" if not blas else ", BLAS pools %s" % blas)}
+                      "(%.1f s) on one thread (BLAS pools pinned to 1 of %d "
+                      "host cores)" % (reps, w.G, nb, w.n_tail, w.name, dt,
+                                       avail)}
 
 
 def run_reference(args, world, rank):
@@ -567,15 +658,16 @@ def run_reference(args, world, rank):
     w = synth.WORKLOADS[args.workload]
     blocks = 256
     arc = prepare_oracle_sample(w, blocks=blocks, heads=((0, 0),))
-    for _ in range(args.warmup):
-        oracle_sample_step(arc, None, list(arc), w.R)
-    t0 = time.perf_counter()
-    nbytes = 0
-    for _ in range(args.steps):
-        nbytes += oracle_sample_step(arc, None, list(arc), w.R)
-    dt = time.perf_counter() - t0
+    with blas_limit(1):
+        cores, avail, _ = cpu_cores_used()
+        for _ in range(args.warmup):
+            oracle_sample_step(arc, None, list(arc), w.R)
+        t0 = time.perf_counter()
+        nbytes = 0
+        for _ in range(args.steps):
+            nbytes += oracle_sample_step(arc, None, list(arc), w.R)
+        dt = time.perf_counter() - t0
     value = nbytes / dt / 1e9
-    cores, _ = cpu_cores_used()
     sample = ("each step: decode attention of 1 kv head (%d q heads) over "
               "%d blocks + %d tail tokens of the %s workload, fp64 oracle "
               "decompress-then-softmax" % (w.G, blocks, w.n_tail, w.name))
@@ -591,7 +683,8 @@ def run_reference(args, world, rank):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hk": w.Hk,
                    "D": w.D, "T": w.T, "R": w.R, "S": w.S},
         "cpu_baseline": {"value": round(value, 6), "unit": "GB/s",
-                         "cores": cores, "kind": "oracle", "sample": sample},
+                         "cores": cores, "host_cores": avail,
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 6), "unit": "GB/s",
                 "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
@@ -610,6 +703,9 @@ def main(argv=None):
                     help="archive copies visited round-robin (0 = enough to "
                          "exceed twice the L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="tiny,gqa,large,stream",
+                    help="comma-separated further workloads whose decode "
+                         "attention is timed at full size ('' = none)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -30,6 +30,9 @@ FC_DECODE_PORTABLE = 2
 FC_DECODE_OVERLAP = 4
 FC_DECODE_Q_FINAL = 8
 
+FC_KERNEL_CUDA_CORE = 0
+FC_KERNEL_TENSOR_CORE = 1
+
 FC_SELECT_MAX_BATCH = 1024
 
 FC_DTYPE_F32 = 0
@@ -46,6 +49,7 @@ EXPORTS = (
     "fc_combine", "fc_decode_attention_noalloc", "fc_workspace_status",
     "fc_storage_bytes", "fc_status_string", "fc_decode_step",
     "fc_read_view", "fc_crop", "fc_select_batch", "fc_noalloc_status",
+    "fc_decode_kernel",
 )
 
 
@@ -103,6 +107,8 @@ def load() -> ctypes.CDLL:
         "fc_decode_plan": (ctypes.c_int, [PA, PT, I64,
                                           ctypes.POINTER(ctypes.c_int32)]),
         "fc_decode_workspace_bytes": (ctypes.c_size_t, [I64, I64, I64, I32]),
+        "fc_decode_kernel": (ctypes.c_int, [PA, PA, I64, I32,
+                                            ctypes.POINTER(ctypes.c_int32)]),
         "fc_decode_attention": (ctypes.c_int, [P, I32, PI64, I64, PA, PA, PT,
                                                PT, ctypes.c_float, I32, I32,
                                                P, ctypes.c_size_t, P, I32,
@@ -214,6 +220,18 @@ def fc_decode_plan(ka: FcArchive, kt: Optional[FcTail], Hq: int) -> int:
     st = load().fc_decode_plan(ctypes.byref(ka), _ref(kt), int(Hq),
                                ctypes.byref(out))
     _check(st, "fc_decode_plan")
+    return int(out.value)
+
+
+def fc_decode_kernel(ka: FcArchive, va: FcArchive, Hq: int,
+                     portable: bool = False) -> int:
+    """FC_KERNEL_TENSOR_CORE or FC_KERNEL_CUDA_CORE: the kernel decode
+    attention runs for these archives."""
+    out = ctypes.c_int32(0)
+    st = load().fc_decode_kernel(ctypes.byref(ka), ctypes.byref(va), int(Hq),
+                                 FC_DECODE_PORTABLE if portable else 0,
+                                 ctypes.byref(out))
+    _check(st, "fc_decode_kernel")
     return int(out.value)
 
 

@@ -321,6 +321,11 @@ class CodecKVCache:
             self._plans[key] = ns
         return ns
 
+    def tensor_core_path(self, Hq: int, portable: bool = False) -> bool:
+        """Whether decode attention runs on the tensor-core kernel."""
+        return _lib.fc_decode_kernel(self.k.arc, self.v.arc, Hq, portable) \
+            == _lib.FC_KERNEL_TENSOR_CORE
+
     def workspace(self, Hq: int, num_splits: int) -> torch.Tensor:
         key = (Hq, num_splits)
         need = self._ws_need.get(key)

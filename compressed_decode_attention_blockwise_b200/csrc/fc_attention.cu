@@ -67,6 +67,20 @@ extern "C" int fc_decode_plan(const fc_archive* ka, const fc_tail* kt, int64_t H
   return FC_OK;
 }
 
+extern "C" int fc_decode_kernel(const fc_archive* ka, const fc_archive* va, int64_t Hq, int32_t flags,
+                                int32_t* kind_out) {
+  if (!kind_out || !va) return FC_ERR_INVALID;
+  int st = check_archive(ka);
+  if (st != FC_OK) return st;
+  st = check_archive(va);
+  if (st != FC_OK) return st;
+  if (Hq < 1 || Hq % ka->H) return FC_ERR_INVALID;
+  *kind_out = (!(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, int(Hq / ka->H)))
+                  ? FC_KERNEL_TENSOR_CORE
+                  : FC_KERNEL_CUDA_CORE;
+  return FC_OK;
+}
+
 namespace fc {
 namespace {
 

@@ -183,6 +183,17 @@ int fc_decode_plan(const fc_archive* ka, const fc_tail* kt, int64_t Hq,
                    int32_t* num_splits_out);
 
 /*
+ * fc_decode_kernel -- which kernel fc_decode_attention / fc_decode_step use
+ * for these archives, Hq and flags on the current device: FC_KERNEL_TENSOR_CORE
+ * (5th-generation tensor cores, the int8 paths of the header's supported
+ * sizes) or FC_KERNEL_CUDA_CORE (the portable kernel). Host query only; the
+ * results of the two kernels agree to rounding.
+ */
+enum { FC_KERNEL_CUDA_CORE = 0, FC_KERNEL_TENSOR_CORE = 1 };
+int fc_decode_kernel(const fc_archive* ka, const fc_archive* va, int64_t Hq,
+                     int32_t flags, int32_t* kind_out);
+
+/*
  * fc_decode_workspace_bytes -- bytes of workspace fc_decode_attention and
  * fc_combine need for (B, Hq, D, num_splits): a status word, one ticket per
  * (b, kv head), and the fp32 partials (max, sum, acc[D]) per (b, q head,

@@ -12,7 +12,8 @@ import oracle
 import synth
 from compressed_decode_attention_blockwise_b200 import (CodecKVCache, FcError,
                                                         _lib)
-from _helpers import check_out, f64, oracle_on_gpu_archive
+from _helpers import check_codes, check_out, check_scales, f64, \
+    oracle_on_gpu_archive
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
@@ -130,6 +131,7 @@ def test_workspace_tickets_return_to_zero():
 def test_full_size_workload(name):
     w = synth.WORKLOADS[name]
     cache, data = _cache_for(w)
+    assert cache.tensor_core_path(w.Hq) == (name != "tiny")
     q = data["q"].to(DEV)
     out = cache.attention(q)                 # benchmark launch configuration
     torch.cuda.synchronize()
@@ -157,10 +159,11 @@ def test_full_size_large_sampled_heads():
 
 def test_end_to_end_against_oracle_archive():
     """Oracle's own archive (fp64 encode) through the oracle's attention vs
-    the GPU pipeline: covers codec + attention together. The two archives may
-    differ by the permitted +-1 code flips near half-integers, each worth one
-    quantisation step of one coefficient, so this cross-archive check holds
-    the relative-L2 bar and a max-abs bound of 1e-2."""
+    the GPU pipeline: codec + attention together, at the full bar. Both
+    encoders take the rounding decision in fp64, so the two archives can only
+    differ where a pre-rounding value lies within rounding distance (~1e-14)
+    of a half-integer; the codes are compared first and the number of such
+    +-1 differences is asserted to be zero on this input."""
     w = synth.WORKLOADS["gqa"].replace(B=2, T=8 * 120 + 5, seed=8)
     cache, data = _cache_for(w)
     q = data["q"].to(DEV)
@@ -168,13 +171,15 @@ def test_end_to_end_against_oracle_archive():
     torch.cuda.synchronize()
     ek = oracle.encode_stream(f64(data["k"]), w.R, w.S, "i8")
     ev = oracle.encode_stream(f64(data["v"]), w.R, w.S, "i8")
+    flips = 0
+    for st, e in ((cache.k, ek), (cache.v, ev)):
+        flips += check_codes(st.live_coeffs().cpu().numpy(), e["y"])
+        check_scales(st.live_scales().cpu().numpy(), e["scales"])
+    assert flips == 0, flips
     ref = oracle.decode_attention_reference(f64(data["q"]), ek["C_hat"],
                                             ev["C_hat"], ek["tail"],
                                             ev["tail"], w.R)
-    got = f64(out)
-    err = np.max(np.abs(got - ref))
-    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
-    assert rel <= 1e-3 and err <= 1e-2, (err, rel)
+    check_out(f64(out), ref, "codec + attention end to end")
 
 
 # every (G, S, R / S) the tensor-core kernel is instantiated for: lanes with

@@ -9,7 +9,7 @@ import torch
 
 import oracle
 import synth
-from compressed_decode_attention_blockwise_b200 import CodecKVCache
+from compressed_decode_attention_blockwise_b200 import CodecKVCache, _lib
 from _helpers import check_codes, check_out, check_scales, f64, \
     oracle_on_gpu_archive
 
@@ -146,3 +146,77 @@ def test_fused_step_in_a_graph_and_portable_path():
         torch.cuda.synchronize()
         assert torch.equal(o_port, o_ref)
     _same_stream(port, ref)
+
+
+@pytest.mark.parametrize("name", ["long", "stream"])
+def test_benchmarked_decode_step_at_full_size(name):
+    """fc_decode_step exactly as the benchmark times it: the full-size
+    workload, the planner's split count (18 chunks per kv head on `long`), the
+    fused combine, FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL, the steps captured
+    in a CUDA graph and replayed, R + 1 steps so that one of them completes a
+    block (encoded in the kernel). The archive and tail end bitwise equal to
+    those of fc_append_step + fc_decode_attention, and every output element of
+    every step is checked against the fp64 oracle on the GPU's own archive
+    (the archive of step s is the first n_blocks(s) blocks of the final one,
+    which no step rewrites; its raw tail is the input tokens after them)."""
+    w = synth.WORKLOADS[name]
+    steps = w.R + 1
+    data = synth.generate(w.replace(steps=steps), q_steps=steps)
+    k, v, q = data["k"].to(DEV), data["v"].to(DEV), data["q"].to(DEV)
+    graphed, two = _twin_caches(w, data)
+    cap = (w.T + steps) // w.R + 1
+    for c in (graphed, two):
+        c._grow_to(cap)
+    ns = graphed.num_splits(w.Hq)
+    if name == "long":
+        assert ns == _lib.fc_decode_plan(graphed.k.arc, graphed.k.tail_desc,
+                                         w.Hq) and ns > 8
+    graphed.workspace(w.Hq, ns)
+    outs = [torch.full((w.B, w.Hq, 1, w.D), float("nan"), device=DEV)
+            for _ in range(steps)]
+    state = []                            # (n_blocks, tail_len) after step s
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for s in range(steps):
+            t = w.T + s
+            graphed.step(q[s], k[:, :, t:t + 1], v[:, :, t:t + 1],
+                         out=outs[s], overlap=True, q_final=True)
+            state.append((graphed.k.n_blocks, graphed.k.tail_len))
+    g.replay()
+    torch.cuda.synchronize()
+    assert any(nr == 0 for _, nr in state)          # a block was completed
+    two_outs = []
+    for s in range(steps):
+        t = w.T + s
+        two.append(k[:, :, t:t + 1], v[:, :, t:t + 1])
+        two_outs.append(two.attention(q[s]))
+    torch.cuda.synchronize()
+    _same_stream(graphed, two)
+    assert _lib.fc_workspace_status(graphed._ws) == 0
+    # the oracle at every step, over the final archive's prefix
+    ck_all = {}
+    for (b, h) in [(b, h) for b in range(w.B) for h in range(w.Hk)]:
+        ck_all[(b, h)] = (_dequant(graphed.k, b, h), _dequant(graphed.v, b, h))
+    G = w.G
+    for s, (nb, nr) in enumerate(state):
+        got = f64(outs[s])
+        assert np.isfinite(got).all()
+        ref = np.empty_like(got)
+        t_end = w.T + s + 1
+        for (b, h), (ck, cv) in ck_all.items():
+            tk = f64(data["k"][b:b + 1, h:h + 1, nb * w.R:t_end])
+            tv = f64(data["v"][b:b + 1, h:h + 1, nb * w.R:t_end])
+            assert tk.shape[2] == nr
+            ref[b:b + 1, h * G:(h + 1) * G] = oracle.decode_attention_reference(
+                f64(q[s][b:b + 1, h * G:(h + 1) * G]), ck[:, :, :nb],
+                cv[:, :, :nb], tk, tv, w.R)
+        check_out(got, ref, "%s step %d" % (name, s))
+        diff = (outs[s] - two_outs[s]).abs().max().item()
+        assert diff <= 2e-4, (s, diff)
+
+
+def _dequant(stream, b, h):
+    c = stream.coeffs[b:b + 1, h:h + 1, :stream.n_blocks].cpu().numpy()
+    sc = stream.scales[b:b + 1, h:h + 1, :stream.n_blocks].cpu().numpy()
+    return oracle.dequantize(c, sc)
