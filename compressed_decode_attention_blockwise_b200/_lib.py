@@ -49,7 +49,7 @@ EXPORTS = (
     "fc_combine", "fc_decode_attention_noalloc", "fc_workspace_status",
     "fc_storage_bytes", "fc_status_string", "fc_decode_step",
     "fc_read_view", "fc_crop", "fc_select_batch", "fc_noalloc_status",
-    "fc_decode_kernel",
+    "fc_decode_kernel", "fc_state_bytes", "fc_state_save", "fc_state_restore",
 )
 
 
@@ -69,6 +69,19 @@ class FcArchive(ctypes.Structure):
         ("capacity", ctypes.c_int64), ("n_blocks", ctypes.c_int64),
         ("coeff_stride_b", ctypes.c_int64), ("coeff_stride_h", ctypes.c_int64),
         ("scale_stride_b", ctypes.c_int64), ("scale_stride_h", ctypes.c_int64),
+    ]
+
+
+class FcStateHeader(ctypes.Structure):
+    """fc_state_header of include/fc_state.h."""
+    _fields_ = [
+        ("magic", ctypes.c_char * 8), ("version", ctypes.c_int32),
+        ("coeff_dtype", ctypes.c_int32), ("tail_dtype", ctypes.c_int32),
+        ("R", ctypes.c_int32), ("S", ctypes.c_int32),
+        ("tail_len", ctypes.c_int32), ("B", ctypes.c_int64),
+        ("H", ctypes.c_int64), ("D", ctypes.c_int64),
+        ("n_blocks", ctypes.c_int64), ("coeff_bytes", ctypes.c_int64),
+        ("scale_bytes", ctypes.c_int64), ("tail_bytes", ctypes.c_int64),
     ]
 
 
@@ -129,6 +142,9 @@ def load() -> ctypes.CDLL:
         "fc_noalloc_status": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32),
                                              P]),
         "fc_storage_bytes": (ctypes.c_int64, [PA, PT]),
+        "fc_state_bytes": (ctypes.c_size_t, [PA, PT]),
+        "fc_state_save": (ctypes.c_int, [PA, PT, P, ctypes.c_size_t, P]),
+        "fc_state_restore": (ctypes.c_int, [P, ctypes.c_size_t, PA, PT, P]),
         "fc_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "fc_read_view": (ctypes.c_int, [PA, PT, I64, P, I32, PI64, I64, P]),
         "fc_crop": (ctypes.c_int, [PA, PT, I64, P]),
@@ -340,6 +356,57 @@ def fc_storage_bytes(arc: FcArchive, tail: Optional[FcTail] = None) -> int:
     if n < 0:
         raise FcError(FC_ERR_INVALID, "fc_storage_bytes")
     return n
+
+
+# ------------------------------------------------- save / restore (state)
+
+def fc_state_bytes(arc: FcArchive, tail: Optional[FcTail] = None) -> int:
+    n = int(load().fc_state_bytes(ctypes.byref(arc), _ref(tail)))
+    if n == 0:
+        raise FcError(FC_ERR_INVALID, "fc_state_bytes")
+    return n
+
+
+def fc_state_save(arc: FcArchive, tail: Optional[FcTail], dst: torch.Tensor,
+                  stream=None, device=None) -> None:
+    """Write the stream's image into the CPU uint8 tensor ``dst`` (pinned
+    for an asynchronous copy); complete once the stream reaches the copies."""
+    if dst.device.type != "cpu" or dst.dtype != torch.uint8 or \
+            not dst.is_contiguous():
+        raise ValueError("dst must be a contiguous CPU uint8 tensor")
+    s = _stream(stream) if stream is not None or device is None else \
+        ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = load().fc_state_save(ctypes.byref(arc), _ref(tail), _ptr(dst),
+                              dst.numel(), s)
+    _check(st, "fc_state_save")
+
+
+def fc_state_header(src: torch.Tensor) -> FcStateHeader:
+    """The header of an image held in a CPU uint8 tensor."""
+    if src.numel() < ctypes.sizeof(FcStateHeader):
+        raise ValueError("image shorter than its header")
+    if src.device.type != "cpu" or src.dtype != torch.uint8 or \
+            not src.is_contiguous():
+        raise ValueError("src must be a contiguous CPU uint8 tensor")
+    hd = FcStateHeader()
+    ctypes.memmove(ctypes.byref(hd), src.data_ptr(),
+                   ctypes.sizeof(FcStateHeader))
+    return hd
+
+
+def fc_state_restore(src: torch.Tensor, arc: FcArchive,
+                     tail: Optional[FcTail], stream=None,
+                     device=None) -> None:
+    """Load an image (CPU uint8 tensor) into the stream; sets n_blocks and
+    the tail length on success."""
+    if src.device.type != "cpu" or src.dtype != torch.uint8 or \
+            not src.is_contiguous():
+        raise ValueError("src must be a contiguous CPU uint8 tensor")
+    s = _stream(stream) if stream is not None or device is None else \
+        ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    st = load().fc_state_restore(_ptr(src), src.numel(), ctypes.byref(arc),
+                                 _ref(tail), s)
+    _check(st, "fc_state_restore")
 
 
 # --------------------------------------------------- stream structure (view)

@@ -210,6 +210,27 @@ class CodecStream:
          self.tail_desc) = gathered
         self.discard_view()
 
+    def save_state(self) -> torch.Tensor:
+        """Exact image of the stream (header, live coefficients, scales and
+        raw tail rows) in a pinned CPU uint8 tensor; the call waits for the
+        copies."""
+        n = _lib.fc_state_bytes(self.arc, self.tail_desc)
+        pin = self.device.type == "cuda"
+        buf = torch.empty(n, dtype=torch.uint8, pin_memory=pin)
+        _lib.fc_state_save(self.arc, self.tail_desc, buf, device=self.device)
+        if pin:
+            torch.cuda.current_stream(self.device).synchronize()
+        return buf
+
+    def restore_state(self, buf: torch.Tensor):
+        """Replace the stream's content with a saved image (bitwise); the
+        archive grows first when the image holds more blocks than fit."""
+        hd = _lib.fc_state_header(buf)
+        self.ensure_capacity(int(hd.n_blocks))
+        _lib.fc_state_restore(buf, self.arc, self.tail_desc,
+                              device=self.device)
+        self.discard_view()
+
     def reset(self):
         """Empty the stream; capacity and buffers are kept
         (``_CodecStream.reset``)."""
@@ -430,6 +451,37 @@ class CodecKVCache:
     def discard_view(self):
         self.k.discard_view()
         self.v.discard_view()
+
+    # -- save / restore ------------------------------------------------------
+    def save_state(self) -> dict:
+        """Exact images of both streams (``CodecStream.save_state``)."""
+        return {"k": self.k.save_state(), "v": self.v.save_state()}
+
+    def restore_state(self, state: dict):
+        """Load images written by ``save_state``: the archives and raw tails
+        become bitwise the saved ones (same B, Hk, D, R, S and dtypes)."""
+        hk = _lib.fc_state_header(state["k"])
+        hv = _lib.fc_state_header(state["v"])
+        if (hk.n_blocks, hk.tail_len) != (hv.n_blocks, hv.tail_len):
+            raise ValueError("K and V images disagree on length")
+        self.k.restore_state(state["k"])
+        self.v.restore_state(state["v"])
+
+    def to_legacy(self):
+        """The pages' legacy export (``FlashCodecCache.to_legacy_cache`` for
+        one layer): the reconstructed (keys, values) views."""
+        return self.read()
+
+    @classmethod
+    def from_legacy(cls, keys: torch.Tensor, values: torch.Tensor, **cfg):
+        """The pages' legacy import (``from_legacy_cache`` for one layer):
+        a new cache whose streams take the full views through the codec
+        once more (lossy again, unlike ``restore_state``)."""
+        B, Hk, _, D = keys.shape
+        cache = cls(B, Hk, D, token_dtype=keys.dtype, device=keys.device,
+                    **cfg)
+        cache.prefill(keys, values)
+        return cache
 
     def reset(self):
         """Empty both streams, keeping their capacity."""

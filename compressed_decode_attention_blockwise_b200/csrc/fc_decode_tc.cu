@@ -75,19 +75,38 @@ struct Cfg {
   static constexpr int TB = kRows / S;             // blocks per tile
   static constexpr int BW = 32 / S;                // blocks per warp
   static constexpr int NI = G >= S ? G / S : 1;    // (block, head) items per lane
-  // compute groups of four warps (three where a lane's items need more
-  // registers than four groups leave)
-  static constexpr int NG = (S == 8 || G == 8) ? 3 : 4;
+  // Two compute groups of four warps, a TMA warp and an MMA warp in half an
+  // SM (shared memory, registers, TMEM), so that the CTA of the next launch
+  // on the stream (a programmatic dependent) can be resident beside this one
+  // and stream its archive while this one drains. Where a lane's items need
+  // more registers than that leaves (eight heads, or eight coefficients per
+  // block), three groups with deeper rings take the whole SM instead.
+  static constexpr int kCtasPerSm = (G == 8 || S == 8) ? 1 : 2;
+  static constexpr int NG = kCtasPerSm == 2 ? 2 : 3;
   static constexpr int HPG = (G + NG - 1) / NG;    // heads per group in the final merge
   static constexpr int NP = pad16(3 * G);          // MMA N: three limb columns per head
-  static constexpr int NKS = 4;                    // K ring stages
-  static constexpr int NVS = NP == 16 ? 7 : 6;     // V ring stages
-  static constexpr int kThreads = 128 * NG + 96;   // + TMA, K-MMA and V-MMA warps
+  static constexpr int NKS = kCtasPerSm == 2 ? 2 : 4;  // K ring stages
+  static constexpr int kThreads = 128 * NG + 64;   // + TMA and MMA warps
   // per group 2 K and 2 V buffers, allocated as a power of two
-  static constexpr uint32_t kTmemCols = 4 * NP * NG <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = 4 * NP * NG <= 128 ? 128 : 4 * NP * NG <= 256 ? 256 : 512;
   static constexpr uint32_t LBO = 16 * NP;         // W operand: K-direction core-matrix stride
   static constexpr int XP = S * (G + 1);           // transpose scratch floats per block
   static constexpr int XW = BW * XP;               // ... per warp
+  static constexpr int kBarsFor(int nvs) { return 2 * NKS + 2 * nvs + 10 * NG + 1; }
+  // shared memory with nvs V stages (before the 1024-byte alignment slack)
+  static constexpr uint32_t bytesFor(int nvs) {
+    return (NKS + nvs) * kTileBytes + NP * 128 + nvs * 2 * kScaleBytes + NG * 2 * NP * 128 +
+           NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + kBarsFor(nvs) * 8 + 16;
+  }
+  // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2 each; one: 227 KB
+  // (alignment slack included)
+  static constexpr uint32_t kSmemCap = kCtasPerSm == 2 ? 115712 : 232448;
+  static constexpr int vStages() {
+    int n = 2;
+    while (n < 7 && bytesFor(n + 1) + 1024 <= kSmemCap) ++n;
+    return n;
+  }
+  static constexpr int NVS = vStages();  // V ring stages
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr uint32_t kt = 0;
   static constexpr uint32_t vt = kt + NKS * kTileBytes;
@@ -99,13 +118,14 @@ struct Cfg {
   static constexpr uint32_t qu = red + NG * 2 * (G + 1) * 16;  // G limb units of q
   static constexpr uint32_t qs = qu + 64;                     // 4 x G floats: |q| maxima
   static constexpr uint32_t bars = qs + 128;
-  static constexpr int kBars = 2 * NKS + 2 * NVS + 10 * NG + 1;
+  static constexpr int kBars = kBarsFor(NVS);
   static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
   static constexpr uint32_t bytes = misc + 16;
   static constexpr uint32_t alloc = bytes + 1024;             // alignment slack
-  static_assert(alloc <= 232448, "shared memory");
+  static_assert(alloc <= kSmemCap, "shared memory");
+  static_assert(bytes == bytesFor(NVS), "layout");
   static_assert((NG * G * (kD + 5) + 4) * 4 <= int(NKS * kTileBytes), "merge scratch");
-  static_assert(4 * NP * NG <= 512, "TMEM allocation");
+  static_assert(4 * NP * NG <= int(kTmemCols) && int(kTmemCols) * kCtasPerSm <= 512, "TMEM allocation");
   static_assert(NI * R <= 32, "logits per lane");
   static_assert(R * HPG <= XW, "tail batch scratch");
 };
@@ -324,7 +344,7 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) 
 }
 
 template <int G, int S, int TPT>
-__global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
+__global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, Cfg<G, S, TPT>::kCtasPerSm)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const TcArgs ta, const TcBasis<S, S * TPT> basis) {
@@ -333,7 +353,6 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   constexpr int NG = C::NG;
   constexpr int NCW = 4 * NG;  // compute warps
   constexpr uint32_t kIdescK = ptx::idesc_i8(128, NP, false, false);
-  constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
   constexpr uint32_t kWBytes = NP * 128;  // one W buffer
 
   const DecodeArgs& a = ta.d;
@@ -361,8 +380,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   const int ntiles = max(0, tile1 - tile0);
   const bool producer = warp >= NCW;
   const bool tma_warp = warp == NCW;
-  const bool kmma_warp = warp == NCW + 1;  // also owns the TMEM allocation
-  const bool vmma_warp = warp == NCW + 2;
+  const bool mma_warp = warp == NCW + 1;  // also owns the TMEM allocation
 
   const int grp = producer ? 0 : warp >> 2;  // compute group
   const int w = warp & 3;                    // warp in the group = TMEM lane quadrant
@@ -431,7 +449,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
     *last_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (kmma_warp) {
+  if (mma_warp) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -518,7 +536,12 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
         if (a.status) atomicOr(a.status, 1u);
         break;
       }
-      __nanosleep(32);
+      // nothing free: suspend on the stage the older of the two next loads
+      // needs (bounded by the hardware's time limit) instead of spinning
+      if (nk < ntiles && (nk <= nv || nv >= ntiles))
+        ptx::mbar_try_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u);
+      else
+        ptx::mbar_try_wait(&vfree[nv % NVS], uint32_t(nv / NVS - 1) & 1u);
     }
     // after an abort, the newest load of every stage must land before the
     // CTA exits (older ones completed before their stage was reissued)
@@ -527,19 +550,26 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
     }
   }
-  if (kmma_warp && lane == 0) {
-    // ================= K-MMA thread: S_int of each tile into its group's
-    // TMEM buffer as soon as it lands
+  if (mma_warp && lane == 0) {
+    // ================= MMA thread: the K-side MMA of tile i (S_int into its
+    // group's TMEM buffer) once the tile has landed, then the V-side MMA of
+    // tile i - 1 (Acc_int) once its W is written. Neither waits on the other:
+    // K(i) needs only its tile and a group buffer freed by the softmax of
+    // tile i - 2 NG, V(i - 1) only the softmax of tile i - 1, and every wait
+    // suspends the thread instead of spinning.
     waiter.wait(qready, 0u);
-    int i = 0;
-    for (; i < ntiles; ++i) {
+    constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
+    const uint32_t qa = ptx::smem_u32(sm + C::qb);
+    uint64_t* last_bar = nullptr;  // commit barrier and phase of the newest MMA
+    uint32_t last_par = 0;
+    bool ok = true;
+    auto issue_k = [&](int i) {
       const int s = i % NKS, g = i % NG, k = i / NG, x = k & 1;
       uint64_t* gq = gbar + 10 * g;
-      if (!waiter.wait(&kfull[s], uint32_t(i / NKS) & 1u)) break;
-      if (!waiter.wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+      if (!waiter.wait(&kfull[s], uint32_t(i / NKS) & 1u)) return false;
+      if (!waiter.wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) return false;
       ptx::tc_fence_after();
       const uint32_t ka = ptx::smem_u32(sm + C::kt + s * kTileBytes);
-      const uint32_t qa = ptx::smem_u32(sm + C::qb);
       const uint32_t d = tmem + uint32_t(g * 4 * NP + x * NP);
 #pragma unroll
       for (int kk = 0; kk < kD / 32; ++kk)
@@ -547,20 +577,16 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
                     kIdescK, kk > 0 ? 1u : 0u);
       ptx::mma_commit(&kfree[s]);
       ptx::mma_commit(&gq[x]);
-    }
-    // after an abort, the MMAs already issued finish before TMEM is freed
-    if (i < ntiles && i > 0) drain_wait(&kfree[(i - 1) % NKS], uint32_t((i - 1) / NKS) & 1u);
-  }
-  if (vmma_warp && lane == 0) {
-    // ================= V-MMA thread: Acc_int of each tile as soon as its W is
-    // written
-    int i = 0;
-    for (; i < ntiles; ++i) {
+      last_bar = &kfree[s];
+      last_par = uint32_t(i / NKS) & 1u;
+      return true;
+    };
+    auto issue_v = [&](int i) {
       const int s = i % NVS, g = i % NG, k = i / NG, x = k & 1;
       uint64_t* gq = gbar + 10 * g;
-      if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) break;
-      if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) break;
-      if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+      if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) return false;
+      if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) return false;
+      if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) return false;
       ptx::tc_fence_after();
       const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
       const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
@@ -571,8 +597,17 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
                     ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
       ptx::mma_commit(&vfree[s]);
       ptx::mma_commit(&gq[6 + x]);
+      last_bar = &vfree[s];
+      last_par = uint32_t(i / NVS) & 1u;
+      return true;
+    };
+    for (int i = 0; ok && i <= ntiles; ++i) {
+      if (i < ntiles) ok = issue_k(i);
+      if (ok && i >= 1) ok = issue_v(i - 1);
     }
-    if (i < ntiles && i > 0) drain_wait(&vfree[(i - 1) % NVS], uint32_t((i - 1) / NVS) & 1u);
+    // after an abort, the MMAs already issued finish before TMEM is freed
+    // (the newest commit tracks every earlier MMA of this thread)
+    if (!ok && last_bar) drain_wait(last_bar, last_par);
   }
 
   // ================= compute groups
@@ -971,7 +1006,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (kmma_warp) {
+  if (mma_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -1044,7 +1079,11 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
   using C = Cfg<G, S, TPT>;
   const size_t smem = C::alloc;
   auto kern = decode_tc_kernel<G, S, TPT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+  // the whole unified L1 / shared memory as shared memory, so that two CTAs
+  // fit on an SM
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
+      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
     return FC_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(ta.d.ns), unsigned(ta.d.Hk), unsigned(ta.d.B));

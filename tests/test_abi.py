@@ -307,3 +307,54 @@ def test_view_crop_and_gather_validate_without_launching():
     assert lib.fc_select_batch(ctypes.byref(src), None, big, 1025,
                                ctypes.byref(dst), None, None) == \
         _lib.FC_ERR_UNSUPPORTED
+
+
+def test_state_save_restore_validate_on_the_host():
+    """Image size arithmetic and header checks of fc_state_* (no copy is
+    issued: every case fails validation, or has nothing to copy)."""
+    arc = _lib.FcArchive(coeffs=FAKE, scales=FAKE, coeff_dtype=_lib.FC_DTYPE_I8,
+                         R=8, S=2, B=2, H=3, D=64, capacity=32, n_blocks=10,
+                         coeff_stride_b=3 * 32 * 2 * 64,
+                         coeff_stride_h=32 * 2 * 64,
+                         scale_stride_b=3 * 32 * 2, scale_stride_h=32 * 2)
+    tail = _lib.FcTail(data=FAKE, dtype=_lib.FC_DTYPE_BF16, len=5,
+                       stride_b=3 * 8 * 64, stride_h=8 * 64)
+    hdr = ctypes.sizeof(_lib.FcStateHeader)
+    assert hdr == 88
+    n = _lib.fc_state_bytes(arc, tail)
+    assert n == hdr + 6 * 10 * 2 * 64 + 6 * 10 * 2 * 4 + 6 * 5 * 64 * 2
+    lib = _lib.load()
+    import torch
+    buf = torch.zeros(n, dtype=torch.uint8)
+    # a zeroed image: no magic
+    st = lib.fc_state_restore(ctypes.c_void_p(buf.data_ptr()), n,
+                              ctypes.byref(arc), ctypes.byref(tail), None)
+    assert st == _lib.FC_ERR_INVALID
+    # a correct header for another S
+    h = _lib.FcStateHeader(magic=b"FCSTATE1", version=1,
+                           coeff_dtype=_lib.FC_DTYPE_I8,
+                           tail_dtype=_lib.FC_DTYPE_BF16, R=8, S=3,
+                           tail_len=0, B=2, H=3, D=64, n_blocks=0)
+    ctypes.memmove(buf.data_ptr(), ctypes.byref(h), hdr)
+    st = lib.fc_state_restore(ctypes.c_void_p(buf.data_ptr()), n,
+                              ctypes.byref(arc), ctypes.byref(tail), None)
+    assert st == _lib.FC_ERR_INVALID
+    # the right geometry but more blocks than the capacity
+    h.S, h.n_blocks = 2, 33
+    h.coeff_bytes, h.scale_bytes = 6 * 33 * 2 * 64, 6 * 33 * 2 * 4
+    big = torch.zeros(hdr + h.coeff_bytes + h.scale_bytes, dtype=torch.uint8)
+    ctypes.memmove(big.data_ptr(), ctypes.byref(h), hdr)
+    st = lib.fc_state_restore(ctypes.c_void_p(big.data_ptr()), big.numel(),
+                              ctypes.byref(arc), ctypes.byref(tail), None)
+    assert st == _lib.FC_ERR_CAPACITY
+    assert (arc.n_blocks, tail.len) == (10, 5)
+    # payload sizes that do not match the geometry
+    h.n_blocks = 4
+    ctypes.memmove(big.data_ptr(), ctypes.byref(h), hdr)
+    st = lib.fc_state_restore(ctypes.c_void_p(big.data_ptr()), big.numel(),
+                              ctypes.byref(arc), ctypes.byref(tail), None)
+    assert st == _lib.FC_ERR_INVALID
+    # saving into a buffer that is too small
+    st = lib.fc_state_save(ctypes.byref(arc), ctypes.byref(tail),
+                           ctypes.c_void_p(buf.data_ptr()), n - 1, None)
+    assert st == _lib.FC_ERR_INVALID

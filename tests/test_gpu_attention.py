@@ -159,11 +159,14 @@ def test_full_size_large_sampled_heads():
 
 def test_end_to_end_against_oracle_archive():
     """Oracle's own archive (fp64 encode) through the oracle's attention vs
-    the GPU pipeline: codec + attention together, at the full bar. Both
-    encoders take the rounding decision in fp64, so the two archives can only
-    differ where a pre-rounding value lies within rounding distance (~1e-14)
-    of a half-integer; the codes are compared first and the number of such
-    +-1 differences is asserted to be zero on this input."""
+    the GPU pipeline: codec + attention together. Both encoders decide in
+    fp64, but the pre-rounding value 127 * C / max|C| of bf16 inputs hits a
+    half-integer exactly now and then (a ratio of two short dyadic sums), and
+    the two fp64 evaluations may round such a tie either way: those +-1 code
+    flips are counted and each is checked to be a tie to 1e-9. Their effect
+    on the output is measured exactly (fp64 oracle on the GPU's archive
+    against fp64 oracle on the oracle's), and the GPU output must lie within
+    the full bar of the oracle's result plus that measured effect."""
     w = synth.WORKLOADS["gqa"].replace(B=2, T=8 * 120 + 5, seed=8)
     cache, data = _cache_for(w)
     q = data["q"].to(DEV)
@@ -173,13 +176,27 @@ def test_end_to_end_against_oracle_archive():
     ev = oracle.encode_stream(f64(data["v"]), w.R, w.S, "i8")
     flips = 0
     for st, e in ((cache.k, ek), (cache.v, ev)):
-        flips += check_codes(st.live_coeffs().cpu().numpy(), e["y"])
+        codes = st.live_coeffs().cpu().numpy()
+        flips += check_codes(codes, e["y"])
+        diff = codes.astype(np.int64) != e["codes"].astype(np.int64)
+        y = e["y"][diff]
+        assert np.all(np.abs(np.abs(y - np.floor(y)) - 0.5) < 1e-9), y
         check_scales(st.live_scales().cpu().numpy(), e["scales"])
-    assert flips == 0, flips
     ref = oracle.decode_attention_reference(f64(data["q"]), ek["C_hat"],
                                             ev["C_hat"], ek["tail"],
                                             ev["tail"], w.R)
-    check_out(f64(out), ref, "codec + attention end to end")
+    on_gpu_archive = oracle_on_gpu_archive(cache, q)
+    effect = float(np.max(np.abs(on_gpu_archive - ref)))
+    effect_rel = float(np.linalg.norm(on_gpu_archive - ref) /
+                       np.linalg.norm(ref))
+    got = f64(out)
+    err = float(np.max(np.abs(got - ref)))
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    print("end to end: %d code flips, their effect %.3g (rel L2 %.3g); "
+          "GPU vs oracle archive max abs %.3g, rel L2 %.3g"
+          % (flips, effect, effect_rel, err, rel))
+    assert flips <= 1e-4 * 2 * codes.size, flips
+    assert err <= 2e-3 + effect and rel <= 1e-3 + effect_rel, (err, rel)
 
 
 # every (G, S, R / S) the tensor-core kernel is instantiated for: lanes with
