@@ -326,7 +326,7 @@ class CodecKVCache:
         _lib.fc_decode_step(
             q, k_new, v_new, self.k.arc, self.v.arc, self.k.tail_desc,
             self.v.tail_desc, out, ws, softmax_scale=0.0 if softmax_scale is
-            None else float(softmax_scale), num_splits=ns,
+            None else float(softmax_scale), num_splits=num_splits,
             fuse_combine=fuse_combine, portable=portable, overlap=overlap,
             q_final=q_final)
         if not fuse_combine:
@@ -381,7 +381,8 @@ class CodecKVCache:
         _lib.fc_decode_attention(
             q, self.k.arc, self.v.arc, self.k.tail_desc, self.v.tail_desc,
             out, ws, softmax_scale=0.0 if softmax_scale is None else
-            float(softmax_scale), num_splits=ns, fuse_combine=fuse_combine,
+            float(softmax_scale), num_splits=num_splits,
+            fuse_combine=fuse_combine,
             portable=portable, overlap=overlap, q_final=q_final)
         if not fuse_combine:
             _lib.fc_combine(ws, self.B, Hq, self.D, ns, out)

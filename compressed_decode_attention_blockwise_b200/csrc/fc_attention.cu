@@ -8,11 +8,12 @@
 namespace fc {
 namespace {
 
-// Split count. The tensor-core kernel runs one CTA per SM (its two rings of
-// 128-row tiles fill the shared memory): split each kv head into tile-aligned
-// chunks so that all chunks of all kv heads fit in one wave. The portable
-// kernel fits four CTAs per SM (registers) and aims at one wave of them, with
-// chunks of at least 16 blocks.
+// Split count. The tensor-core kernel runs one CTA per SM: with an automatic
+// split the kv heads take ceil(SMs / heads) or one chunk fewer so that the
+// launch has exactly one CTA per SM, and the planner returns the larger
+// count (the workspace's split slots), at most one chunk per 128-row tile.
+// The portable kernel fits four CTAs per SM (registers) and aims at one wave
+// of them, with chunks of at least 16 blocks.
 // Results do not depend on the split beyond rounding.
 int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   if (nb <= 0) return 1;
@@ -20,7 +21,7 @@ int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   const bool tiles = D == 128 && S >= 1 && 32 % S == 0;
   int64_t ns;
   if (tiles) {
-    ns = int64_t(sm_count()) / units;
+    ns = (int64_t(sm_count()) + units - 1) / units;
     const int64_t t = tc_tiles_per_head(nb, S);
     if (ns > t) ns = t;
   } else {
@@ -40,7 +41,7 @@ __global__ void __launch_bounds__(128) combine_kernel(CombineArgs a) {
   extern __shared__ float wts[];  // ns + 1
   const int hq = blockIdx.x, b = blockIdx.y;
   const int64_t row = (int64_t(b) * a.Hq + hq) * a.ns;
-  combine_heads(a.pm + row, a.pl + row, a.pacc + row * a.D, 1, a.ns, a.D, wts, a.out,
+  combine_heads(a.pm + row, a.pl + row, a.pacc + row * a.D, 1, a.ns, a.ns, a.D, wts, a.out,
                 b * a.os_b + hq * a.os_h, a.os_h, a.out_dtype);
 }
 
@@ -168,6 +169,11 @@ int prepare_decode(const void* q, int32_t q_dtype, const int64_t* q_strides, int
   a.nb = ka->n_blocks;
   a.ns = ns;
   a.chunk = ka->n_blocks > 0 ? (ka->n_blocks + ns - 1) / ns : 0;
+  // the uneven automatic split needs the fused combine (fc_combine merges
+  // ns slots for every head)
+  a.auto_split = (num_splits == 0 && fuse_combine) ? 1 : 0;
+  a.bal_q = ns;
+  a.bal_rem = 0;
   const float sigma = softmax_scale > 0.f ? softmax_scale : float(1.0 / std::sqrt(double(ka->D)));
   a.qscale = float(double(sigma) * 1.4426950408889634);  // log2(e)
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -364,7 +370,7 @@ extern "C" int fc_decode_attention_noalloc(const void* q, int32_t q_dtype, const
   // kernel reported stays readable through fc_noalloc_status
   if (cudaMemsetAsync(static_cast<uint8_t*>(scratch) + wl.tickets, 0, wl.m - wl.tickets, stream) != cudaSuccess)
     return FC_ERR_CUDA;
-  return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, ns,
+  return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits,
                              FC_DECODE_FUSE_COMBINE, scratch, FC_NOALLOC_SCRATCH_BYTES, out, out_dtype,
                              out_strides, stream);
 }

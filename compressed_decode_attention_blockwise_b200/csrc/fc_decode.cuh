@@ -50,8 +50,12 @@ struct DecodeArgs {
   int nr;  // live tail tokens
   int B, Hk, G, R, S, D;
   int64_t nb;
-  int ns;
+  int ns;         // split slots per (b, q head) in the workspace
   int64_t chunk;
+  // tensor-core kernel, automatic split: the first bal_rem kv heads take
+  // bal_q + 1 chunks, the others bal_q (one CTA per SM in all); 0 = ns each
+  int bal_q, bal_rem;
+  int auto_split;  // num_splits was 0: ns is the planner's slot count
   float qscale;  // sigma * log2(e)
   uint32_t* status;
   uint32_t* tickets;
@@ -86,7 +90,8 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, int dtype, flo
 // outputs: M = max_c m_c, L = sum_c l_c e^(m_c - M), out = sum_c acc_c
 // e^(m_c - M) / L, chunks with l_c = 0 skipped (base-2 exponentials: the
 // partial maxima are kept in log2 units). Head i's partials are rows
-// pm[i * ns + c], pl[i * ns + c], pacc[(i * ns + c) * D + d]; its output goes to
+// pm[i * stride + c], pl[i * stride + c], pacc[(i * stride + c) * D + d]
+// (stride >= ns: the workspace's split slots per head); its output goes to
 // out[out_off + i * out_stride_h + d]. All threads of the CTA take part. Each
 // thread first issues the loads of the partial accumulators of its first
 // (head, channel) output (up to kPre of them) and only then do warps compute
@@ -95,8 +100,8 @@ __device__ __forceinline__ void store_out(void* out, int64_t idx, int dtype, flo
 // than threads) and partials beyond kPre use batched loads. Partials written
 // by other CTAs of the same launch are read through L2 (ld.cg).
 __device__ __forceinline__ void combine_heads(const float* pm, const float* pl, const float* pacc, int NH,
-                                              int ns, int D, float* wts, void* out, int64_t out_off,
-                                              int64_t out_stride_h, int out_dtype) {
+                                              int ns, int stride, int D, float* wts, void* out,
+                                              int64_t out_off, int64_t out_stride_h, int out_dtype) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
   const int n_out = NH * D;
@@ -104,15 +109,15 @@ __device__ __forceinline__ void combine_heads(const float* pm, const float* pl, 
   // partials of my first output, requested before the weights are known
   const bool has_first = tid < n_out;
   const int fi = has_first ? tid / D : 0, fd = has_first ? tid - fi * D : 0;
-  const float* fsrc = pacc + int64_t(fi) * ns * D + fd;
+  const float* fsrc = pacc + int64_t(fi) * stride * D + fd;
   float pre[kPre];
 #pragma unroll
   for (int u = 0; u < kPre; ++u) pre[u] = (has_first && u < ns) ? __ldcg(fsrc + int64_t(u) * D) : 0.f;
 
   constexpr int kReg = 4;  // partial rows per lane kept in registers (ns <= 128)
   for (int i = warp; i < NH; i += nwarps) {
-    const float* m = pm + int64_t(i) * ns;
-    const float* l = pl + int64_t(i) * ns;
+    const float* m = pm + int64_t(i) * stride;
+    const float* l = pl + int64_t(i) * stride;
     float* w = wts + i * (ns + 1);
     float mx = -INFINITY, L = 0.f;
     if (ns <= 32 * kReg) {
@@ -162,7 +167,7 @@ __device__ __forceinline__ void combine_heads(const float* pm, const float* pl, 
   for (int o = tid + blockDim.x; o < n_out; o += blockDim.x) {
     const int i = o / D, d = o - i * D;
     const float* w = wts + i * (ns + 1);
-    const float* src = pacc + int64_t(i) * ns * D + d;
+    const float* src = pacc + int64_t(i) * stride * D + d;
     float acc = 0.f;
     for (int c0 = 0; c0 < ns; c0 += 16) {
       float v[16];
@@ -240,7 +245,7 @@ __device__ __forceinline__ void finish_cta(const DecodeArgs& a, int b, int h, in
   __shared__ int s_last;
   if (!last_cta_ticket(a.tickets + (b * a.Hk + h), a.ns, &s_last)) return;
   const int64_t row = (int64_t(b) * Hq + h * G) * a.ns;
-  combine_heads(a.pm + row, a.pl + row, a.pacc + row * D, G, a.ns, D, scratch, a.out,
+  combine_heads(a.pm + row, a.pl + row, a.pacc + row * D, G, a.ns, a.ns, D, scratch, a.out,
                 b * a.os_b + (h * G) * a.os_h, a.os_h, a.out_dtype);
   if (tid == 0) a.tickets[b * a.Hk + h] = 0u;
 }

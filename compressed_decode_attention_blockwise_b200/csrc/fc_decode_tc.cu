@@ -49,6 +49,7 @@
 // issued (also bounded), frees its TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -69,23 +70,25 @@ constexpr int kMagicBits = 0x4B400000;
 
 __host__ __device__ constexpr int pad16(int x) { return (x + 15) / 16 * 16; }
 
-template <int G, int S, int TPT>
+template <int G, int S, int TPT, bool HALF>
 struct Cfg {
   static constexpr int R = S * TPT;
   static constexpr int TB = kRows / S;             // blocks per tile
   static constexpr int BW = 32 / S;                // blocks per warp
   static constexpr int NI = G >= S ? G / S : 1;    // (block, head) items per lane
-  // Two compute groups of four warps, a TMA warp and an MMA warp in half an
-  // SM (shared memory, registers, TMEM), so that the CTA of the next launch
-  // on the stream (a programmatic dependent) can be resident beside this one
-  // and stream its archive while this one drains. Where a lane's items need
-  // more registers than that leaves (eight heads, or eight coefficients per
-  // block), three groups with deeper rings take the whole SM instead.
-  static constexpr int kCtasPerSm = (G == 8 || S == 8) ? 1 : 2;
-  static constexpr int NG = kCtasPerSm == 2 ? 2 : 3;
+  // Two layouts. Full: one CTA per SM with deep rings and four compute
+  // groups of four warps (three where a lane's items need more registers:
+  // eight heads, or eight coefficients per block). HALF (launches with
+  // FC_DECODE_OVERLAP, G <= 4 and S <= 4): two groups and shallow rings in
+  // half an SM (shared memory, registers, TMEM), so that the CTA of the next
+  // launch on the stream (a programmatic dependent) is resident beside this
+  // one and streams its archive while this one drains. Both add a TMA warp
+  // and an MMA warp.
+  static constexpr int kCtasPerSm = HALF ? 2 : 1;
+  static constexpr int NG = HALF ? 2 : (S == 8 || G == 8) ? 3 : 4;
   static constexpr int HPG = (G + NG - 1) / NG;    // heads per group in the final merge
   static constexpr int NP = pad16(3 * G);          // MMA N: three limb columns per head
-  static constexpr int NKS = kCtasPerSm == 2 ? 2 : 4;  // K ring stages
+  static constexpr int NKS = HALF ? 2 : 4;         // K ring stages
   static constexpr int kThreads = 128 * NG + 64;   // + TMA and MMA warps
   // per group 2 K and 2 V buffers, allocated as a power of two
   static constexpr uint32_t kTmemCols = 4 * NP * NG <= 128 ? 128 : 4 * NP * NG <= 256 ? 256 : 512;
@@ -103,7 +106,7 @@ struct Cfg {
   static constexpr uint32_t kSmemCap = kCtasPerSm == 2 ? 115712 : 232448;
   static constexpr int vStages() {
     int n = 2;
-    while (n < 7 && bytesFor(n + 1) + 1024 <= kSmemCap) ++n;
+    while (n < (HALF ? 3 : 7) && bytesFor(n + 1) + 1024 <= kSmemCap) ++n;
     return n;
   }
   static constexpr int NVS = vStages();  // V ring stages
@@ -133,7 +136,6 @@ struct Cfg {
 struct TcArgs {
   DecodeArgs d;
   int tiles_per_head;
-  int chunk_tiles;
 };
 
 // The DCT basis rows the kernel needs, sized for its (S, R): fp32 for the
@@ -343,12 +345,12 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) 
   }
 }
 
-template <int G, int S, int TPT>
-__global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, Cfg<G, S, TPT>::kCtasPerSm)
+template <int G, int S, int TPT, bool HALF>
+__global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT, HALF>::kCtasPerSm)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const TcArgs ta, const TcBasis<S, S * TPT> basis) {
-  using C = Cfg<G, S, TPT>;
+  using C = Cfg<G, S, TPT, HALF>;
   constexpr int R = C::R, NP = C::NP, NI = C::NI, NKS = C::NKS, NVS = C::NVS, XP = C::XP;
   constexpr int NG = C::NG;
   constexpr int NCW = 4 * NG;  // compute warps
@@ -371,13 +373,29 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, Cfg<G, S, TPT>::kCta
   int* last_flag = reinterpret_cast<int*>(sm + C::misc + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // CTA -> (kv head unit, chunk c of its ns_u): the first bal_rem units take
+  // bal_q + 1 chunks, the others bal_q; a unit's tiles split evenly
+  int unit, c, ns_u;
+  {
+    const int bx = blockIdx.x, hi = a.bal_q + 1;
+    if (bx < a.bal_rem * hi) {
+      unit = bx / hi;
+      c = bx - unit * hi;
+      ns_u = hi;
+    } else {
+      const int r = bx - a.bal_rem * hi;
+      unit = a.bal_rem + r / a.bal_q;
+      c = r - (unit - a.bal_rem) * a.bal_q;
+      ns_u = a.bal_q;
+    }
+  }
+  const int h = unit % a.Hk, b = unit / a.Hk;
   const int Hq = a.Hk * G;
   Waiter waiter{abort_flag, a.status};
 
-  const int tile0 = c * ta.chunk_tiles;
-  const int tile1 = min(tile0 + ta.chunk_tiles, ta.tiles_per_head);
-  const int ntiles = max(0, tile1 - tile0);
+  const int tile0 = int(int64_t(c) * ta.tiles_per_head / ns_u);
+  const int tile1 = int(int64_t(c + 1) * ta.tiles_per_head / ns_u);
+  const int ntiles = tile1 - tile0;
   const bool producer = warp >= NCW;
   const bool tma_warp = warp == NCW;
   const bool mma_warp = warp == NCW + 1;  // also owns the TMEM allocation
@@ -787,7 +805,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, Cfg<G, S, TPT>::kCta
   }
 
   // ---- merge the four groups' states, fold the raw tail, write the partials
-  const bool direct = a.fuse && a.ns == 1;
+  const bool direct = a.fuse && ns_u == 1;
   if (!producer) {
     // softmax sums of my items over the warp's blocks
 #pragma unroll
@@ -841,7 +859,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, Cfg<G, S, TPT>::kCta
       Ah[y] = As;
     }
     const bool active = grp < G;  // uniform per group
-    const bool last_chunk = c == a.ns - 1;
+    const bool last_chunk = c == ns_u - 1;
     // fused decode step whose token completes a block: warps 0 and 1 of group
     // 0 encode it (tail rows 0..R-2 and the new token) into archive slot
     // new_slot with the codec's own device code, so the archive is bitwise
@@ -1012,10 +1030,10 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, Cfg<G, S, TPT>::kCta
   }
 
   if (direct || !a.fuse) return;
-  if (!last_cta_ticket(a.tickets + (b * a.Hk + h), a.ns, last_flag)) return;
+  if (!last_cta_ticket(a.tickets + (b * a.Hk + h), ns_u, last_flag)) return;
   float* wts = reinterpret_cast<float*>(sm);  // the rings are free now
   const int64_t row = (int64_t(b) * Hq + h * G) * a.ns;
-  combine_heads(a.pm + row, a.pl + row, a.pacc + row * kD, G, a.ns, kD, wts, a.out,
+  combine_heads(a.pm + row, a.pl + row, a.pacc + row * kD, G, ns_u, a.ns, kD, wts, a.out,
                 b * a.os_b + (h * G) * a.os_h, a.os_h, a.out_dtype);
   if (tid == 0) a.tickets[b * a.Hk + h] = 0u;
 }
@@ -1067,7 +1085,7 @@ bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G, int S, int TPT>
+template <int G, int S, int TPT, bool HALF>
 int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CUtensorMap* maps,
            cudaStream_t stream) {
   TcBasis<S, S * TPT> basis;
@@ -1076,9 +1094,9 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
       basis.m[j][t] = full.m[j][t];
       basis.m64[j][t] = full64.m[j][t];
     }
-  using C = Cfg<G, S, TPT>;
+  using C = Cfg<G, S, TPT, HALF>;
   const size_t smem = C::alloc;
-  auto kern = decode_tc_kernel<G, S, TPT>;
+  auto kern = decode_tc_kernel<G, S, TPT, HALF>;
   // the whole unified L1 / shared memory as shared memory, so that two CTAs
   // fit on an SM
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
@@ -1086,7 +1104,8 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
                            int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
     return FC_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(unsigned(ta.d.ns), unsigned(ta.d.Hk), unsigned(ta.d.B));
+  const unsigned units = unsigned(ta.d.B) * unsigned(ta.d.Hk);
+  cfg.gridDim = dim3(unsigned(ta.d.bal_rem) + units * unsigned(ta.d.bal_q));
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -1125,16 +1144,31 @@ int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive
   tc::TcArgs ta;
   ta.d = d;
   ta.tiles_per_head = tc_tiles_per_head(d.nb, d.S);
-  ta.chunk_tiles = (ta.tiles_per_head + d.ns - 1) / d.ns;
+  const int64_t units = int64_t(d.B) * d.Hk;
+  if (d.auto_split) {
+    // one CTA per SM (or one per kv head when there are more of them): the
+    // chunk counts of the kv heads differ by at most one
+    const int64_t ctas = units >= sm_count() ? units : std::min<int64_t>(sm_count(), units * ta.tiles_per_head);
+    ta.d.bal_q = int(ctas / units);
+    ta.d.bal_rem = int(ctas % units);
+    if (ta.d.bal_q + (ta.d.bal_rem > 0 ? 1 : 0) > d.ns) return FC_ERR_INVALID;
+  } else {
+    ta.d.bal_q = d.ns;
+    ta.d.bal_rem = 0;
+  }
   CUtensorMap maps[4];
   const int64_t rows = d.nb * d.S;
   if (!tc::make_code_map(&maps[0], ka, rows) || !tc::make_code_map(&maps[1], va, rows) ||
       !tc::make_scale_map(&maps[2], ka, rows) || !tc::make_scale_map(&maps[3], va, rows))
     return FC_ERR_CUDA;
   const int key = d.G * 10000 + d.S * 100 + d.R / d.S;
+  // the half-SM layout serves overlapped launches where its registers suffice
+  const bool half = d.overlap && d.G <= 4 && d.S <= 4;
   switch (key) {
-#define FC_TC_CASE(G, S, T) \
-  case G * 10000 + S * 100 + T: return tc::launch<G, S, T>(ta, basis, basis64, maps, stream);
+#define FC_TC_CASE(G, S, T)                                                                              \
+  case G * 10000 + S * 100 + T:                                                                         \
+    return half ? tc::launch<G, S, T, (G <= 4 && S <= 4)>(ta, basis, basis64, maps, stream)              \
+                : tc::launch<G, S, T, false>(ta, basis, basis64, maps, stream);
     FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
     FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
     FC_TC_CASE(1, 2, 4) FC_TC_CASE(2, 2, 4) FC_TC_CASE(4, 2, 4) FC_TC_CASE(8, 2, 4)
