@@ -65,6 +65,8 @@ constexpr uint32_t kTileBytes = kRows * kD;
 constexpr uint32_t kScaleBytes = kRows * 4;
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 2 GHz
 constexpr int kFinBar = 8;   // named barrier over every compute warp
+constexpr int kTailBar = 9;  // compute warps + the tail warp: its partial is ready
+constexpr uint32_t kPollNs = 200;  // producer's suspension when nothing is ready
 constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
@@ -82,8 +84,9 @@ struct Cfg {
   // FC_DECODE_OVERLAP, G <= 4 and S <= 4): two groups and shallow rings in
   // half an SM (shared memory, registers, TMEM), so that the CTA of the next
   // launch on the stream (a programmatic dependent) is resident beside this
-  // one and streams its archive while this one drains. Both add a TMA warp
-  // and an MMA warp.
+  // one and streams its archive while this one drains. Both add a producer
+  // warp (TMA loads and every MMA) and a tail warp (TMEM allocation; the
+  // raw-tail tokens, a fused step's new token or block).
   static constexpr int kCtasPerSm = HALF ? 2 : 1;
   static constexpr int NG = HALF ? 2 : (S == 8 || G == 8) ? 3 : 4;
   static constexpr int HPG = (G + NG - 1) / NG;    // heads per group in the final merge
@@ -99,7 +102,7 @@ struct Cfg {
   // shared memory with nvs V stages (before the 1024-byte alignment slack)
   static constexpr uint32_t bytesFor(int nvs) {
     return (NKS + nvs) * kTileBytes + NP * 128 + nvs * 2 * kScaleBytes + NG * 2 * NP * 128 +
-           NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + kBarsFor(nvs) * 8 + 16;
+           NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + G * (kD + 4) * 4 + kBarsFor(nvs) * 8 + 16;
   }
   // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2 each; one: 227 KB
   // (alignment slack included)
@@ -120,7 +123,8 @@ struct Cfg {
   static constexpr uint32_t red = xs + NG * 4 * XW * 4;      // NG x 2 x (G + 1) x 4 floats
   static constexpr uint32_t qu = red + NG * 2 * (G + 1) * 16;  // G limb units of q
   static constexpr uint32_t qs = qu + 64;                     // 4 x G floats: |q| maxima
-  static constexpr uint32_t bars = qs + 128;
+  static constexpr uint32_t tp = qs + 128;                    // tail partial: G x (acc[D], m, l, pad)
+  static constexpr uint32_t bars = tp + G * (kD + 4) * 4;
   static constexpr int kBars = kBarsFor(NVS);
   static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
   static constexpr uint32_t bytes = misc + 16;
@@ -130,7 +134,7 @@ struct Cfg {
   static_assert((NG * G * (kD + 5) + 4) * 4 <= int(NKS * kTileBytes), "merge scratch");
   static_assert(4 * NP * NG <= int(kTmemCols) && int(kTmemCols) * kCtasPerSm <= 512, "TMEM allocation");
   static_assert(NI * R <= 32, "logits per lane");
-  static_assert(R * HPG <= XW, "tail batch scratch");
+  static_assert(R <= 32, "tail tokens");
 };
 
 struct TcArgs {
@@ -335,6 +339,174 @@ __device__ __forceinline__ void encode_new_block(const DecodeArgs& a, int which,
     run(__nv_bfloat16());
 }
 
+// Softmax partial (base-2 maximum m, sum l, acc[d]) of the tokens that are
+// not in archive tiles, computed by one warp (lane = channels 4 lane ..
+// 4 lane + 3) while the compute groups stream the tiles: the raw-tail rows
+// [0, nr) of kv head (b, h), and in a fused decode step the new token (step
+// 1: also stored at tail row nr) or the block it completes (step 2: tail rows
+// 0..R-2 and the token, encoded into archive slot new_slot with the codec's
+// own device code, exactly as the append kernel does, and folded in the
+// coefficient domain: s_j = scale_k,j C_k[j] . q, logits = A s, w = p A,
+// acc = sum_j w_j scale_v,j C_v[j]). Writes m, l, acc of every head to `tp`
+// (head g at tp + g * (kD + 4): acc[0..kD), m, l).
+template <int G, int S, int R>
+__device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<S, R>& basis, int b, int h,
+                                             int lane, float* tp) {
+  constexpr int VEC = kD / 32;
+  const int d0 = lane * VEC;
+  float qv[G][VEC];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v)
+      qv[g][v] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + d0 + v, a.q_dtype) * a.qscale;
+  float m[G], l[G], acc[G][VEC];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m[g] = -INFINITY;
+    l[g] = 0.f;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[g][v] = 0.f;
+  }
+  if (a.step == 2) {
+    encode_new_block<S, R>(a, 0, lane, basis, b, h);
+    encode_new_block<S, R>(a, 1, lane, basis, b, h);
+    __syncwarp();
+    const StreamOut& ko = a.kout;
+    const StreamOut& vo = a.vout;
+    const signed char* kc =
+        static_cast<const signed char*>(ko.coeffs) + b * ko.cs_b + h * ko.cs_h + a.new_slot * S * kD;
+    const signed char* vc =
+        static_cast<const signed char*>(vo.coeffs) + b * vo.cs_b + h * vo.cs_h + a.new_slot * S * kD;
+    const float* ksp = ko.scales + b * ko.ss_b + h * ko.ss_h + a.new_slot * S;
+    const float* vsp = vo.scales + b * vo.ss_b + h * vo.ss_h + a.new_slot * S;
+    // s_j of every head (written by this warp just above: read through L2)
+    float sj[S][G];
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      const float ks = __ldcg(ksp + j);
+      float kf[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) kf[v] = float(__ldcg(kc + j * kD + d0 + v));
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float x = 0.f;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) x = fmaf(kf[v], qv[g][v], x);
+        sj[j][g] = warp_sum(x) * ks;
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float lg[R], mx = -INFINITY;
+#pragma unroll
+      for (int tk = 0; tk < R; ++tk) {
+        float v = 0.f;
+#pragma unroll
+        for (int j = 0; j < S; ++j) v = fmaf(basis.m[j][tk], sj[j][g], v);
+        lg[tk] = v;
+        mx = fmaxf(mx, v);
+      }
+      float ps = 0.f, wv[S];
+#pragma unroll
+      for (int j = 0; j < S; ++j) wv[j] = 0.f;
+#pragma unroll
+      for (int tk = 0; tk < R; ++tk) {
+        const float p = ptx::ex2(lg[tk] - mx);
+        ps += p;
+#pragma unroll
+        for (int j = 0; j < S; ++j) wv[j] = fmaf(p, basis.m[j][tk], wv[j]);
+      }
+      m[g] = mx;
+      l[g] = ps;
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        const float wj = wv[j] * __ldcg(vsp + j);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wj, float(__ldcg(vc + j * kD + d0 + v)), acc[g][v]);
+      }
+    }
+  } else {
+    // raw tail rows [0, nr), then (step 1) the new token, four at a time
+    const int n_raw = a.nr;
+    const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
+    constexpr int kB = 4;
+    for (int t0 = 0; t0 < n_tok; t0 += kB) {
+      float kv[kB][VEC], vv[kB][VEC];
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int tt = t0 + u;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          kv[u][v] = 0.f;
+          vv[u][v] = 0.f;
+        }
+        if (tt < n_raw) {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) {
+            kv[u][v] = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + d0 + v, a.t_dtype);
+            vv[u][v] = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + d0 + v, a.t_dtype);
+          }
+        } else if (tt < n_tok) {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) {
+            kv[u][v] = load_any(a.kn, b * a.kns_b + h * a.kns_h + d0 + v, a.t_dtype);
+            vv[u][v] = load_any(a.vn, b * a.vns_b + h * a.vns_h + d0 + v, a.t_dtype);
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float lg[kB], mx = m[g];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          float x = 0.f;
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) x = fmaf(qv[g][v], kv[u][v], x);
+          lg[u] = warp_sum(x);
+          if (t0 + u < n_tok) mx = fmaxf(mx, lg[u]);
+        }
+        const float al = ptx::ex2(m[g] - mx);
+        float ps = 0.f, add[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) add[v] = 0.f;
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          if (t0 + u < n_tok) {
+            const float p = ptx::ex2(lg[u] - mx);
+            ps += p;
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) add[v] = fmaf(p, vv[u][v], add[v]);
+          }
+        }
+        l[g] = fmaf(l[g], al, ps);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(acc[g][v], al, add[v]);
+        m[g] = mx;
+      }
+    }
+    if (a.step == 1) {  // the token joins the tail at row nr
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) {
+        copy_elem(a.kt, b * a.kts_b + h * a.kts_h + int64_t(n_raw) * kD + d0 + v, a.kn,
+                  b * a.kns_b + h * a.kns_h + d0 + v, a.t_dtype);
+        copy_elem(a.vt, b * a.vts_b + h * a.vts_h + int64_t(n_raw) * kD + d0 + v, a.vn,
+                  b * a.vns_b + h * a.vns_h + d0 + v, a.t_dtype);
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float* o = tp + g * (kD + 4);
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) o[d0 + v] = acc[g][v];
+    if (lane == 0) {
+      o[kD] = m[g];
+      o[kD + 1] = l[g];
+    }
+  }
+}
+
 template <int NP>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) {
   if constexpr (NP == 16) {
@@ -397,8 +569,8 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   const int tile1 = int(int64_t(c + 1) * ta.tiles_per_head / ns_u);
   const int ntiles = tile1 - tile0;
   const bool producer = warp >= NCW;
-  const bool tma_warp = warp == NCW;
-  const bool mma_warp = warp == NCW + 1;  // also owns the TMEM allocation
+  const bool tma_warp = warp == NCW;       // TMA loads and every MMA (lane 0)
+  const bool tail_warp = warp == NCW + 1;  // TMEM allocation; the tail partial
 
   const int grp = producer ? 0 : warp >> 2;  // compute group
   const int w = warp & 3;                    // warp in the group = TMEM lane quadrant
@@ -467,7 +639,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
     *last_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (mma_warp) {
+  if (tail_warp) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -532,10 +704,64 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
 
   if (tma_warp && lane == 0) {
     // ================= TMA thread: both rings, in tile order each, whichever
-    // has a free stage (every stage was filled once before the setup barrier)
+    // has a free stage (every stage was filled once before the setup
+    // barrier), and the K-side MMA of each tile (S_int into its group's TMEM
+    // buffer) as soon as the tile has landed and the group's buffer is free,
+    // so that K sums run up to 2 NG tiles ahead of the softmax
+    const uint32_t qa = ptx::smem_u32(sm + C::qb);
+    constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
+    int nm = 0;           // K-side MMAs issued
+    int nw = 0;           // V-side MMAs issued
+    bool q_ok = false;    // the query limbs are in shared memory
+    uint64_t* last_k = nullptr;  // commit barrier and phase of the newest MMA
+    uint32_t last_kp = 0;
     unsigned long long t_last = clock64();
-    while (nk < ntiles || nv < ntiles) {
+    while (nk < ntiles || nv < ntiles || nm < ntiles || nw < ntiles) {
       bool prog = false;
+      if (nm < nk) {
+        const int s = nm % NKS, g = nm % NG, k = nm / NG, x = k & 1;
+        uint64_t* gq = gbar + 10 * g;
+        if (!q_ok) q_ok = ptx::mbar_test_wait(qready, 0u);
+        if (q_ok && ptx::mbar_test_wait(&kfull[s], uint32_t(nm / NKS) & 1u) &&
+            ptx::mbar_test_wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) {
+          ptx::tc_fence_after();
+          const uint32_t ka = ptx::smem_u32(sm + C::kt + s * kTileBytes);
+          const uint32_t d = tmem + uint32_t(g * 4 * NP + x * NP);
+#pragma unroll
+          for (int kk = 0; kk < kD / 32; ++kk)
+            ptx::mma_i8(d, ptx::desc_sw128(ka + 32 * kk, 16, 1024), ptx::desc_sw128(qa + 32 * kk, 16, 1024),
+                        kIdescK, kk > 0 ? 1u : 0u);
+          ptx::mma_commit(&kfree[s]);
+          ptx::mma_commit(&gq[x]);
+          last_k = &kfree[s];
+          last_kp = uint32_t(nm / NKS) & 1u;
+          ++nm;
+          prog = true;
+        }
+      }
+      // V-side MMA (Acc_int) of the oldest tile whose W is written
+      if (nw < nm) {
+        const int s = nw % NVS, g = nw % NG, k = nw / NG, x = k & 1;
+        uint64_t* gq = gbar + 10 * g;
+        if (ptx::mbar_test_wait(&gq[4 + x], uint32_t(k >> 1) & 1u) &&
+            ptx::mbar_test_wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u) &&
+            ptx::mbar_test_wait(&vfull[s], uint32_t(nw / NVS) & 1u)) {
+          ptx::tc_fence_after();
+          const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
+          const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
+          const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
+#pragma unroll
+          for (int kk = 0; kk < kRows / 32; ++kk)
+            ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
+                        ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
+          ptx::mma_commit(&vfree[s]);
+          ptx::mma_commit(&gq[6 + x]);
+          last_k = &vfree[s];
+          last_kp = uint32_t(nw / NVS) & 1u;
+          ++nw;
+          prog = true;
+        }
+      }
       if (nk < ntiles && ptx::mbar_test_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u)) {
         load_k(nk++);
         prog = true;
@@ -554,78 +780,44 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
         if (a.status) atomicOr(a.status, 1u);
         break;
       }
-      // nothing free: suspend on the stage the older of the two next loads
-      // needs (bounded by the hardware's time limit) instead of spinning
-      if (nk < ntiles && (nk <= nv || nv >= ntiles))
+      // nothing ready: a short suspension (bounded) on what the next
+      // K-side MMA lacks, else on the next V-side MMA's W, else on the stage
+      // the older of the two next loads needs
+      if (nm < nk) {
+        const int s = nm % NKS, k = nm / NG;
+        if (!q_ok)
+          ptx::mbar_try_wait_ns(qready, 0u, kPollNs);
+        else if (!ptx::mbar_test_wait(&kfull[s], uint32_t(nm / NKS) & 1u))
+          ptx::mbar_try_wait_ns(&kfull[s], uint32_t(nm / NKS) & 1u, kPollNs);
+        else
+          ptx::mbar_try_wait_ns(&gbar[10 * (nm % NG) + 2 + (k & 1)], (uint32_t(k >> 1) & 1u) ^ 1u, kPollNs);
+      } else if (nw < nm) {
+        const int k = nw / NG;
+        ptx::mbar_try_wait_ns(&gbar[10 * (nw % NG) + 4 + (k & 1)], uint32_t(k >> 1) & 1u, kPollNs);
+      } else if (nk < ntiles && (nk <= nv || nv >= ntiles)) {
         ptx::mbar_try_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u);
-      else
+      } else if (nv < ntiles) {
         ptx::mbar_try_wait(&vfree[nv % NVS], uint32_t(nv / NVS - 1) & 1u);
+      }
     }
-    // after an abort, the newest load of every stage must land before the
-    // CTA exits (older ones completed before their stage was reissued)
+    // after an abort, the MMAs issued finish (the newest commit tracks every
+    // earlier one of this thread) and the newest load of every stage lands
+    // before the CTA exits (older ones completed before their stage was
+    // reissued)
     if (*reinterpret_cast<volatile int*>(abort_flag)) {
+      if (last_k) drain_wait(last_k, last_kp);
       for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
       for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
     }
   }
-  if (mma_warp && lane == 0) {
-    // ================= MMA thread: the K-side MMA of tile i (S_int into its
-    // group's TMEM buffer) once the tile has landed, then the V-side MMA of
-    // tile i - 1 (Acc_int) once its W is written. Neither waits on the other:
-    // K(i) needs only its tile and a group buffer freed by the softmax of
-    // tile i - 2 NG, V(i - 1) only the softmax of tile i - 1, and every wait
-    // suspends the thread instead of spinning.
-    waiter.wait(qready, 0u);
-    constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
-    const uint32_t qa = ptx::smem_u32(sm + C::qb);
-    uint64_t* last_bar = nullptr;  // commit barrier and phase of the newest MMA
-    uint32_t last_par = 0;
-    bool ok = true;
-    auto issue_k = [&](int i) {
-      const int s = i % NKS, g = i % NG, k = i / NG, x = k & 1;
-      uint64_t* gq = gbar + 10 * g;
-      if (!waiter.wait(&kfull[s], uint32_t(i / NKS) & 1u)) return false;
-      if (!waiter.wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) return false;
-      ptx::tc_fence_after();
-      const uint32_t ka = ptx::smem_u32(sm + C::kt + s * kTileBytes);
-      const uint32_t d = tmem + uint32_t(g * 4 * NP + x * NP);
-#pragma unroll
-      for (int kk = 0; kk < kD / 32; ++kk)
-        ptx::mma_i8(d, ptx::desc_sw128(ka + 32 * kk, 16, 1024), ptx::desc_sw128(qa + 32 * kk, 16, 1024),
-                    kIdescK, kk > 0 ? 1u : 0u);
-      ptx::mma_commit(&kfree[s]);
-      ptx::mma_commit(&gq[x]);
-      last_bar = &kfree[s];
-      last_par = uint32_t(i / NKS) & 1u;
-      return true;
-    };
-    auto issue_v = [&](int i) {
-      const int s = i % NVS, g = i % NG, k = i / NG, x = k & 1;
-      uint64_t* gq = gbar + 10 * g;
-      if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) return false;
-      if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) return false;
-      if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) return false;
-      ptx::tc_fence_after();
-      const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
-      const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
-      const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
-#pragma unroll
-      for (int kk = 0; kk < kRows / 32; ++kk)
-        ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
-                    ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
-      ptx::mma_commit(&vfree[s]);
-      ptx::mma_commit(&gq[6 + x]);
-      last_bar = &vfree[s];
-      last_par = uint32_t(i / NVS) & 1u;
-      return true;
-    };
-    for (int i = 0; ok && i <= ntiles; ++i) {
-      if (i < ntiles) ok = issue_k(i);
-      if (ok && i >= 1) ok = issue_v(i - 1);
-    }
-    // after an abort, the MMAs already issued finish before TMEM is freed
-    // (the newest commit tracks every earlier MMA of this thread)
-    if (!ok && last_bar) drain_wait(last_bar, last_par);
+  // ================= tail warp: the tokens outside the archive tiles (last
+  // chunk of a kv head), concurrently with the tiles
+  const bool last_chunk = c == ns_u - 1;
+  const bool has_extra = last_chunk && (a.nr > 0 || a.step != 0);
+  if (tail_warp && has_extra) {
+    if (a.overlap) ptx::grid_dep_wait();  // tails and new tokens: after the preceding work
+    tail_partial<G, S, R>(a, basis, b, h, lane, reinterpret_cast<float*>(sm + C::tp));
+    ptx::named_bar_arrive(kTailBar, 128 * NG + 32);
   }
 
   // ================= compute groups
@@ -812,7 +1004,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
     for (int ii = 0; ii < NI; ++ii)
 #pragma unroll
       for (int o = S; o < 32; o <<= 1) lsum[ii] += __shfl_xor_sync(0xffffffffu, lsum[ii], o);
-    // the tails, the workspace and out: after the preceding work
+    // the workspace and out: after the preceding work
     if (a.overlap) ptx::grid_dep_wait();
     // every group is done with both rings: the K ring becomes merge scratch
     ptx::named_bar_sync(kFinBar, 128 * NG);
@@ -830,19 +1022,26 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
 #pragma unroll
     for (int g = 0; g < G; ++g) fa[(grp * G + g) * kD + t] = acc[g];
     ptx::named_bar_sync(kFinBar, 128 * NG);
+    // the tail warp's partial (last chunk with raw tokens or a new token)
+    if (has_extra) ptx::named_bar_sync(kTailBar, 128 * NG + 32);
+    const float* tpart = reinterpret_cast<const float*>(sm + C::tp);
 
-    // group grp finishes heads grp, grp + 4, ...: thread t = channel d
+    // group grp finishes heads grp, grp + NG, ...: thread t = channel d
     constexpr int HPG = C::HPG;
-    float Mh[HPG], Lh[HPG], Ah[HPG];
+    const bool active = grp < G;  // uniform per group
 #pragma unroll
     for (int y = 0; y < HPG; ++y) {
-      const int g = min(grp + NG * y, G - 1);
+      const int g = grp + NG * y;
+      if (!active || g >= G) continue;
       float M = -INFINITY;
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) {
         const float4 l4 = reinterpret_cast<const float4*>(fl)[gg * G + g];
         if (l4.x + l4.y + l4.z + l4.w > 0.f) M = fmaxf(M, fm[gg * G + g]);
       }
+      const float* tg = tpart + g * (kD + 4);
+      const float tl = has_extra ? tg[kD + 1] : 0.f;
+      if (tl > 0.f) M = fmaxf(M, tg[kD]);
       float Ls = 0.f, As = 0.f;
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) {
@@ -854,177 +1053,27 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
           As = fmaf(fa[(gg * G + g) * kD + t], e, As);
         }
       }
-      Mh[y] = M;
-      Lh[y] = Ls;
-      Ah[y] = As;
-    }
-    const bool active = grp < G;  // uniform per group
-    const bool last_chunk = c == ns_u - 1;
-    // fused decode step whose token completes a block: warps 0 and 1 of group
-    // 0 encode it (tail rows 0..R-2 and the new token) into archive slot
-    // new_slot with the codec's own device code, so the archive is bitwise
-    // what fc_append_step writes; the barrier publishes codes and scales to
-    // the CTA
-    if (last_chunk && a.step == 2) {
-      if (grp == 0 && w < 2) encode_new_block<S, S * TPT>(a, w, lane, basis, b, h);
-      ptx::named_bar_sync(kFinBar, 128 * NG);
-    }
-    // raw tail tokens, then the step's new token or block (last chunk)
-    if (active && last_chunk && (a.nr > 0 || a.step != 0)) {
-      float* red2 = reinterpret_cast<float*>(sm + C::xs) + grp * 4 * C::XW;
-      float qh[HPG];
-#pragma unroll
-      for (int y = 0; y < HPG; ++y) {
-        const int g = min(grp + NG * y, G - 1);
-        qh[y] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
+      if (tl > 0.f) {
+        const float e = ptx::ex2(tg[kD] - M);
+        Ls = fmaf(tl, e, Ls);
+        As = fmaf(tg[t], e, As);
       }
-      // the raw tokens of the tail, and the step's new token, in one batch:
-      // one reduction over the group for every logit, then one online-softmax
-      // update (thread t = channel d)
-      const int n_raw = a.step == 2 ? 0 : a.nr;  // a completed block is folded coded
-      const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
-      constexpr int kTok = S * TPT;  // at most R tokens: R - 1 tail rows + the new one
-      if (n_tok > 0) {
-        float kv[kTok], vv[kTok];
-#pragma unroll
-        for (int tt = 0; tt < kTok; ++tt) {
-          kv[tt] = 0.f;
-          vv[tt] = 0.f;
-          if (tt < n_raw) {
-            kv[tt] = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, a.t_dtype);
-            vv[tt] = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, a.t_dtype);
-          } else if (tt == n_raw && a.step == 1) {
-            kv[tt] = load_any(a.kn, b * a.kns_b + h * a.kns_h + t, a.t_dtype);
-            vv[tt] = load_any(a.vn, b * a.vns_b + h * a.vns_h + t, a.t_dtype);
-          }
-        }
-        float lgt[kTok][HPG];
-#pragma unroll
-        for (int tt = 0; tt < kTok; ++tt)
-#pragma unroll
-          for (int y = 0; y < HPG; ++y) lgt[tt][y] = tt < n_tok ? warp_sum(qh[y] * kv[tt]) : 0.f;
-        if (lane == 0) {
-#pragma unroll
-          for (int tt = 0; tt < kTok; ++tt)
-#pragma unroll
-            for (int y = 0; y < HPG; ++y) red2[(w * kTok + tt) * HPG + y] = lgt[tt][y];
-        }
-        ptx::named_bar_sync(1 + grp, 128);
-#pragma unroll
-        for (int tt = 0; tt < kTok; ++tt)
-#pragma unroll
-          for (int y = 0; y < HPG; ++y)
-            lgt[tt][y] = red2[(0 * kTok + tt) * HPG + y] + red2[(1 * kTok + tt) * HPG + y] +
-                         red2[(2 * kTok + tt) * HPG + y] + red2[(3 * kTok + tt) * HPG + y];
-        ptx::named_bar_sync(1 + grp, 128);  // red2 is reused below
-#pragma unroll
-        for (int y = 0; y < HPG; ++y) {
-          float mn = Mh[y];
-#pragma unroll
-          for (int tt = 0; tt < kTok; ++tt)
-            if (tt < n_tok) mn = fmaxf(mn, lgt[tt][y]);
-          const float al = ptx::ex2(Mh[y] - mn);
-          float ps = 0.f, add = 0.f;
-#pragma unroll
-          for (int tt = 0; tt < kTok; ++tt) {
-            if (tt < n_tok) {
-              const float p = ptx::ex2(lgt[tt][y] - mn);
-              ps += p;
-              add = fmaf(p, vv[tt], add);
-            }
-          }
-          Ah[y] = fmaf(Ah[y], al, add);
-          Lh[y] = fmaf(Lh[y], al, ps);
-          Mh[y] = mn;
-        }
-      }
-      if (a.step == 1 && grp == 0) {  // the token joins the tail at row nr
-        copy_elem(a.kt, b * a.kts_b + h * a.kts_h + int64_t(a.nr) * kD + t, a.kn,
-                  b * a.kns_b + h * a.kns_h + t, a.t_dtype);
-        copy_elem(a.vt, b * a.vts_b + h * a.vts_h + int64_t(a.nr) * kD + t, a.vn,
-                  b * a.vns_b + h * a.vns_h + t, a.t_dtype);
-      }
-      if (a.step == 2) {
-        // the new block in the coefficient domain, as a tile row set would be:
-        // s_j = scale_k,j C_k[j] . q, logits = A s, p, w = p A, acc += w scale_v C_v
-        const StreamOut& ko = a.kout;
-        const StreamOut& vo = a.vout;
-        // (written by this CTA before the barrier above: read through L2)
-        const signed char* kc = static_cast<const signed char*>(ko.coeffs) + b * ko.cs_b + h * ko.cs_h + a.new_slot * S * kD;
-        const signed char* vc = static_cast<const signed char*>(vo.coeffs) + b * vo.cs_b + h * vo.cs_h + a.new_slot * S * kD;
-        const float* ksp = ko.scales + b * ko.ss_b + h * ko.ss_h + a.new_slot * S;
-        const float* vsp = vo.scales + b * vo.ss_b + h * vo.ss_h + a.new_slot * S;
-        float ksc[S], vsc[S];
-#pragma unroll
-        for (int j = 0; j < S; ++j) {
-          ksc[j] = __ldcg(ksp + j);
-          vsc[j] = __ldcg(vsp + j);
-        }
-        float sj[S * HPG];
-#pragma unroll
-        for (int j = 0; j < S; ++j) {
-          const float kv = float(__ldcg(kc + j * kD + t));
-#pragma unroll
-          for (int y = 0; y < HPG; ++y) sj[j * HPG + y] = kv * qh[y];
-        }
-        group_sum<S * HPG>(sj, red2, w, lane, 1 + grp);
-        float vcode[S];
-#pragma unroll
-        for (int j = 0; j < S; ++j) vcode[j] = float(__ldcg(vc + j * kD + t));
-#pragma unroll
-        for (int y = 0; y < HPG; ++y) {
-          float lg[S * TPT];
-          float mx = Mh[y];
-#pragma unroll
-          for (int tk = 0; tk < S * TPT; ++tk) {
-            float v = 0.f;
-#pragma unroll
-            for (int j = 0; j < S; ++j) v = fmaf(basis.m[j][tk], sj[j * HPG + y] * ksc[j], v);
-            lg[tk] = v;
-            mx = fmaxf(mx, v);
-          }
-          const float al = ptx::ex2(Mh[y] - mx);
-          float ps = 0.f, wv[S];
-#pragma unroll
-          for (int j = 0; j < S; ++j) wv[j] = 0.f;
-#pragma unroll
-          for (int tk = 0; tk < S * TPT; ++tk) {
-            const float p = ptx::ex2(lg[tk] - mx);
-            ps += p;
-#pragma unroll
-            for (int j = 0; j < S; ++j) wv[j] = fmaf(p, basis.m[j][tk], wv[j]);
-          }
-          float add = 0.f;
-#pragma unroll
-          for (int j = 0; j < S; ++j) add = fmaf(wv[j] * vsc[j], vcode[j], add);
-          Ah[y] = fmaf(Ah[y], al, add);
-          Lh[y] = fmaf(Lh[y], al, ps);
-          Mh[y] = mx;
-        }
-      }
-    }
-    if (active) {
-#pragma unroll
-      for (int y = 0; y < HPG; ++y) {
-        const int g = grp + NG * y;
-        if (g >= G) continue;
-        const int hq = h * G + g;
-        if (direct) {
-          store_out(a.out, b * a.os_b + hq * a.os_h + t, a.out_dtype, Ah[y] / Lh[y]);
-        } else {
-          const int64_t row = (int64_t(b) * Hq + hq) * a.ns + c;
-          a.pacc[row * kD + t] = Ah[y];
-          if (t == 0) {
-            a.pm[row] = Lh[y] > 0.f ? Mh[y] : -INFINITY;
-            a.pl[row] = Lh[y];
-          }
+      const int hq = h * G + g;
+      if (direct) {
+        store_out(a.out, b * a.os_b + hq * a.os_h + t, a.out_dtype, As / Ls);
+      } else {
+        const int64_t row = (int64_t(b) * Hq + hq) * a.ns + c;
+        a.pacc[row * kD + t] = As;
+        if (t == 0) {
+          a.pm[row] = Ls > 0.f ? M : -INFINITY;
+          a.pl[row] = Ls;
         }
       }
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (mma_warp) {
+  if (tail_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }

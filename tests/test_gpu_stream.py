@@ -212,8 +212,10 @@ def test_benchmarked_decode_step_at_full_size(name):
                 f64(q[s][b:b + 1, h * G:(h + 1) * G]), ck[:, :, :nb],
                 cv[:, :, :nb], tk, tv, w.R)
         check_out(got, ref, "%s step %d" % (name, s))
+        # the fused launch (overlapped: the half-SM layout) and the plain
+        # attention launch sum in different orders over 131k tokens
         diff = (outs[s] - two_outs[s]).abs().max().item()
-        assert diff <= 2e-4, (s, diff)
+        assert diff <= 2e-5 * float(np.abs(ref).max()) + 1e-4, (s, diff)
 
 
 def _dequant(stream, b, h):
