@@ -85,8 +85,9 @@ struct Cfg {
   // half an SM (shared memory, registers, TMEM), so that the CTA of the next
   // launch on the stream (a programmatic dependent) is resident beside this
   // one and streams its archive while this one drains. Both add a producer
-  // warp (TMA loads and every MMA) and a tail warp (TMEM allocation; the
-  // raw-tail tokens, a fused step's new token or block).
+  // warp (TMA loads, K-side MMAs) and a warp for TMEM, the V-side MMAs and
+  // then the tokens outside the tiles (raw tail, a fused step's new token or
+  // block).
   static constexpr int kCtasPerSm = HALF ? 2 : 1;
   static constexpr int NG = HALF ? 2 : (S == 8 || G == 8) ? 3 : 4;
   static constexpr int HPG = (G + NG - 1) / NG;    // heads per group in the final merge
@@ -102,7 +103,8 @@ struct Cfg {
   // shared memory with nvs V stages (before the 1024-byte alignment slack)
   static constexpr uint32_t bytesFor(int nvs) {
     return (NKS + nvs) * kTileBytes + NP * 128 + nvs * 2 * kScaleBytes + NG * 2 * NP * 128 +
-           NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + G * (kD + 4) * 4 + kBarsFor(nvs) * 8 + 16;
+           NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + G * (kD + 4) * 4 + G * kD * 4 +
+           kBarsFor(nvs) * 8 + 16;
   }
   // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2 each; one: 227 KB
   // (alignment slack included)
@@ -124,7 +126,8 @@ struct Cfg {
   static constexpr uint32_t qu = red + NG * 2 * (G + 1) * 16;  // G limb units of q
   static constexpr uint32_t qs = qu + 64;                     // 4 x G floats: |q| maxima
   static constexpr uint32_t tp = qs + 128;                    // tail partial: G x (acc[D], m, l, pad)
-  static constexpr uint32_t bars = tp + G * (kD + 4) * 4;
+  static constexpr uint32_t qf = tp + G * (kD + 4) * 4;       // scaled query, G x D floats
+  static constexpr uint32_t bars = qf + G * kD * 4;
   static constexpr int kBars = kBarsFor(NVS);
   static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
   static constexpr uint32_t bytes = misc + 16;
@@ -339,27 +342,51 @@ __device__ __forceinline__ void encode_new_block(const DecodeArgs& a, int which,
     run(__nv_bfloat16());
 }
 
+// Four consecutive token elements (16-byte aligned for fp32, 8-byte for
+// bf16) as floats, one vector load.
+template <typename T>
+__device__ __forceinline__ void load4(const void* base, int64_t idx, float (&o)[4]) {
+  if constexpr (sizeof(T) == 4) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx));
+    o[0] = x.x;
+    o[1] = x.y;
+    o[2] = x.z;
+    o[3] = x.w;
+  } else {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(static_cast<const unsigned short*>(base) + idx));
+    o[0] = __uint_as_float(x.x << 16);
+    o[1] = __uint_as_float(x.x & 0xffff0000u);
+    o[2] = __uint_as_float(x.y << 16);
+    o[3] = __uint_as_float(x.y & 0xffff0000u);
+  }
+}
+
 // Softmax partial (base-2 maximum m, sum l, acc[d]) of the tokens that are
 // not in archive tiles, computed by one warp (lane = channels 4 lane ..
-// 4 lane + 3) while the compute groups stream the tiles: the raw-tail rows
+// 4 lane + 3) while the compute groups finish the tiles: the raw-tail rows
 // [0, nr) of kv head (b, h), and in a fused decode step the new token (step
 // 1: also stored at tail row nr) or the block it completes (step 2: tail rows
 // 0..R-2 and the token, encoded into archive slot new_slot with the codec's
 // own device code, exactly as the append kernel does, and folded in the
 // coefficient domain: s_j = scale_k,j C_k[j] . q, logits = A s, w = p A,
-// acc = sum_j w_j scale_v,j C_v[j]). Writes m, l, acc of every head to `tp`
-// (head g at tp + g * (kD + 4): acc[0..kD), m, l).
-template <int G, int S, int R>
+// acc = sum_j w_j scale_v,j C_v[j]). qs: the scaled query (G x kD floats in
+// shared memory). Writes m, l, acc of every head to `tp` (head g at
+// tp + g * (kD + 4): acc[0..kD), m, l). T: the token dtype.
+template <int G, int S, int R, typename T>
 __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<S, R>& basis, int b, int h,
-                                             int lane, float* tp) {
+                                             int lane, const float* qs, float* tp) {
   constexpr int VEC = kD / 32;
+  static_assert(VEC == 4, "four channels per lane");
   const int d0 = lane * VEC;
   float qv[G][VEC];
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int v = 0; v < VEC; ++v)
-      qv[g][v] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + d0 + v, a.q_dtype) * a.qscale;
+  for (int g = 0; g < G; ++g) {
+    const float4 x = *reinterpret_cast<const float4*>(qs + g * kD + d0);
+    qv[g][0] = x.x;
+    qv[g][1] = x.y;
+    qv[g][2] = x.z;
+    qv[g][3] = x.w;
+  }
   float m[G], l[G], acc[G][VEC];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -380,22 +407,30 @@ __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<
         static_cast<const signed char*>(vo.coeffs) + b * vo.cs_b + h * vo.cs_h + a.new_slot * S * kD;
     const float* ksp = ko.scales + b * ko.ss_b + h * ko.ss_h + a.new_slot * S;
     const float* vsp = vo.scales + b * vo.ss_b + h * vo.ss_h + a.new_slot * S;
-    // s_j of every head (written by this warp just above: read through L2)
-    float sj[S][G];
+    // codes and scales written by this warp just above: read through L2
+    float kf[S][VEC], vf[S][VEC], ksc[S], vsc[S];
 #pragma unroll
     for (int j = 0; j < S; ++j) {
-      const float ks = __ldcg(ksp + j);
-      float kf[VEC];
+      const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int*>(kc + j * kD + d0));
+      const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int*>(vc + j * kD + d0));
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) kf[v] = float(__ldcg(kc + j * kD + d0 + v));
+      for (int v = 0; v < VEC; ++v) {
+        kf[j][v] = float(int8_t(kw >> (8 * v)));
+        vf[j][v] = float(int8_t(vw >> (8 * v)));
+      }
+      ksc[j] = __ldcg(ksp + j);
+      vsc[j] = __ldcg(vsp + j);
+    }
+    float sj[S][G];
+#pragma unroll
+    for (int j = 0; j < S; ++j)
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float x = 0.f;
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) x = fmaf(kf[v], qv[g][v], x);
-        sj[j][g] = warp_sum(x) * ks;
+        for (int v = 0; v < VEC; ++v) x = fmaf(kf[j][v], qv[g][v], x);
+        sj[j][g] = warp_sum(x) * ksc[j];
       }
-    }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float lg[R], mx = -INFINITY;
@@ -421,13 +456,14 @@ __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<
       l[g] = ps;
 #pragma unroll
       for (int j = 0; j < S; ++j) {
-        const float wj = wv[j] * __ldcg(vsp + j);
+        const float wj = wv[j] * vsc[j];
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wj, float(__ldcg(vc + j * kD + d0 + v)), acc[g][v]);
+        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wj, vf[j][v], acc[g][v]);
       }
     }
   } else {
-    // raw tail rows [0, nr), then (step 1) the new token, four at a time
+    // raw tail rows [0, nr), then (step 1) the new token, four at a time:
+    // every row of a batch requested before any is used
     const int n_raw = a.nr;
     const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
     constexpr int kB = 4;
@@ -436,22 +472,17 @@ __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<
 #pragma unroll
       for (int u = 0; u < kB; ++u) {
         const int tt = t0 + u;
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-          kv[u][v] = 0.f;
-          vv[u][v] = 0.f;
-        }
         if (tt < n_raw) {
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) {
-            kv[u][v] = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + d0 + v, a.t_dtype);
-            vv[u][v] = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + d0 + v, a.t_dtype);
-          }
+          load4<T>(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + d0, kv[u]);
+          load4<T>(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + d0, vv[u]);
         } else if (tt < n_tok) {
+          load4<T>(a.kn, b * a.kns_b + h * a.kns_h + d0, kv[u]);
+          load4<T>(a.vn, b * a.vns_b + h * a.vns_h + d0, vv[u]);
+        } else {
 #pragma unroll
           for (int v = 0; v < VEC; ++v) {
-            kv[u][v] = load_any(a.kn, b * a.kns_b + h * a.kns_h + d0 + v, a.t_dtype);
-            vv[u][v] = load_any(a.vn, b * a.vns_b + h * a.vns_h + d0 + v, a.t_dtype);
+            kv[u][v] = 0.f;
+            vv[u][v] = 0.f;
           }
         }
       }
@@ -485,21 +516,28 @@ __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<
         m[g] = mx;
       }
     }
-    if (a.step == 1) {  // the token joins the tail at row nr
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) {
-        copy_elem(a.kt, b * a.kts_b + h * a.kts_h + int64_t(n_raw) * kD + d0 + v, a.kn,
-                  b * a.kns_b + h * a.kns_h + d0 + v, a.t_dtype);
-        copy_elem(a.vt, b * a.vts_b + h * a.vts_h + int64_t(n_raw) * kD + d0 + v, a.vn,
-                  b * a.vns_b + h * a.vns_h + d0 + v, a.t_dtype);
+    if (a.step == 1) {  // the token joins the tail at row nr (bits copied)
+      const int64_t dk = b * a.kts_b + h * a.kts_h + int64_t(n_raw) * kD + d0;
+      const int64_t dv = b * a.vts_b + h * a.vts_h + int64_t(n_raw) * kD + d0;
+      const int64_t sk = b * a.kns_b + h * a.kns_h + d0, sv = b * a.vns_b + h * a.vns_h + d0;
+      if constexpr (sizeof(T) == 4) {
+        *reinterpret_cast<float4*>(const_cast<float*>(static_cast<const float*>(a.kt)) + dk) =
+            __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.kn) + sk));
+        *reinterpret_cast<float4*>(const_cast<float*>(static_cast<const float*>(a.vt)) + dv) =
+            __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.vn) + sv));
+      } else {
+        using U = unsigned short;
+        *reinterpret_cast<uint2*>(const_cast<U*>(static_cast<const U*>(a.kt)) + dk) =
+            __ldg(reinterpret_cast<const uint2*>(static_cast<const U*>(a.kn) + sk));
+        *reinterpret_cast<uint2*>(const_cast<U*>(static_cast<const U*>(a.vt)) + dv) =
+            __ldg(reinterpret_cast<const uint2*>(static_cast<const U*>(a.vn) + sv));
       }
     }
   }
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     float* o = tp + g * (kD + 4);
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) o[d0 + v] = acc[g][v];
+    *reinterpret_cast<float4*>(o + d0) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
     if (lane == 0) {
       o[kD] = m[g];
       o[kD + 1] = l[g];
@@ -569,8 +607,8 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   const int tile1 = int(int64_t(c + 1) * ta.tiles_per_head / ns_u);
   const int ntiles = tile1 - tile0;
   const bool producer = warp >= NCW;
-  const bool tma_warp = warp == NCW;       // TMA loads and every MMA (lane 0)
-  const bool tail_warp = warp == NCW + 1;  // TMEM allocation; the tail partial
+  const bool tma_warp = warp == NCW;       // TMA loads and the K-side MMAs (lane 0)
+  const bool vmma_warp = warp == NCW + 1;  // TMEM allocation, V-side MMAs, the tail partial
 
   const int grp = producer ? 0 : warp >> 2;  // compute group
   const int w = warp & 3;                    // warp in the group = TMEM lane quadrant
@@ -639,7 +677,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
     *last_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (tail_warp) {
+  if (vmma_warp) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -678,8 +716,10 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
       load_q();
     }
     float* qmx = reinterpret_cast<float*>(sm + C::qs);
+    float* qfs = reinterpret_cast<float*>(sm + C::qf);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
+      qfs[g * kD + t] = qd[g];
       const float mx = warp_max(fabsf(qd[g]));
       if (lane == 0) qmx[w * G + g] = mx;
     }
@@ -709,14 +749,12 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
     // buffer) as soon as the tile has landed and the group's buffer is free,
     // so that K sums run up to 2 NG tiles ahead of the softmax
     const uint32_t qa = ptx::smem_u32(sm + C::qb);
-    constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
     int nm = 0;           // K-side MMAs issued
-    int nw = 0;           // V-side MMAs issued
     bool q_ok = false;    // the query limbs are in shared memory
-    uint64_t* last_k = nullptr;  // commit barrier and phase of the newest MMA
+    uint64_t* last_k = nullptr;  // commit barrier and phase of the newest K-side MMA
     uint32_t last_kp = 0;
     unsigned long long t_last = clock64();
-    while (nk < ntiles || nv < ntiles || nm < ntiles || nw < ntiles) {
+    while (nk < ntiles || nv < ntiles || nm < ntiles) {
       bool prog = false;
       if (nm < nk) {
         const int s = nm % NKS, g = nm % NG, k = nm / NG, x = k & 1;
@@ -739,29 +777,6 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
           prog = true;
         }
       }
-      // V-side MMA (Acc_int) of the oldest tile whose W is written
-      if (nw < nm) {
-        const int s = nw % NVS, g = nw % NG, k = nw / NG, x = k & 1;
-        uint64_t* gq = gbar + 10 * g;
-        if (ptx::mbar_test_wait(&gq[4 + x], uint32_t(k >> 1) & 1u) &&
-            ptx::mbar_test_wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u) &&
-            ptx::mbar_test_wait(&vfull[s], uint32_t(nw / NVS) & 1u)) {
-          ptx::tc_fence_after();
-          const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
-          const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
-          const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
-#pragma unroll
-          for (int kk = 0; kk < kRows / 32; ++kk)
-            ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
-                        ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
-          ptx::mma_commit(&vfree[s]);
-          ptx::mma_commit(&gq[6 + x]);
-          last_k = &vfree[s];
-          last_kp = uint32_t(nw / NVS) & 1u;
-          ++nw;
-          prog = true;
-        }
-      }
       if (nk < ntiles && ptx::mbar_test_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u)) {
         load_k(nk++);
         prog = true;
@@ -781,8 +796,8 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
         break;
       }
       // nothing ready: a short suspension (bounded) on what the next
-      // K-side MMA lacks, else on the next V-side MMA's W, else on the stage
-      // the older of the two next loads needs
+      // K-side MMA lacks, else on the stage the older of the two next loads
+      // needs
       if (nm < nk) {
         const int s = nm % NKS, k = nm / NG;
         if (!q_ok)
@@ -791,33 +806,68 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
           ptx::mbar_try_wait_ns(&kfull[s], uint32_t(nm / NKS) & 1u, kPollNs);
         else
           ptx::mbar_try_wait_ns(&gbar[10 * (nm % NG) + 2 + (k & 1)], (uint32_t(k >> 1) & 1u) ^ 1u, kPollNs);
-      } else if (nw < nm) {
-        const int k = nw / NG;
-        ptx::mbar_try_wait_ns(&gbar[10 * (nw % NG) + 4 + (k & 1)], uint32_t(k >> 1) & 1u, kPollNs);
       } else if (nk < ntiles && (nk <= nv || nv >= ntiles)) {
         ptx::mbar_try_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u);
       } else if (nv < ntiles) {
         ptx::mbar_try_wait(&vfree[nv % NVS], uint32_t(nv / NVS - 1) & 1u);
       }
     }
-    // after an abort, the MMAs issued finish (the newest commit tracks every
-    // earlier one of this thread) and the newest load of every stage lands
-    // before the CTA exits (older ones completed before their stage was
-    // reissued)
+    // after an abort, the K-side MMAs issued finish (the newest commit
+    // tracks every earlier one of this thread) and the newest load of every
+    // stage lands before the CTA exits (older ones completed before their
+    // stage was reissued)
     if (*reinterpret_cast<volatile int*>(abort_flag)) {
       if (last_k) drain_wait(last_k, last_kp);
       for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
       for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
     }
   }
-  // ================= tail warp: the tokens outside the archive tiles (last
-  // chunk of a kv head), concurrently with the tiles
   const bool last_chunk = c == ns_u - 1;
   const bool has_extra = last_chunk && (a.nr > 0 || a.step != 0);
-  if (tail_warp && has_extra) {
-    if (a.overlap) ptx::grid_dep_wait();  // tails and new tokens: after the preceding work
-    tail_partial<G, S, R>(a, basis, b, h, lane, reinterpret_cast<float*>(sm + C::tp));
-    ptx::named_bar_arrive(kTailBar, 128 * NG + 32);
+  if (vmma_warp) {
+    if (lane == 0) {
+      // ================= V-MMA thread: Acc_int of each tile, in tile order,
+      // as soon as its W is written (every wait suspends the thread)
+      constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
+      uint64_t* last_bar = nullptr;  // commit barrier and phase of the newest MMA
+      uint32_t last_par = 0;
+      int i = 0;
+      for (; i < ntiles; ++i) {
+        const int s = i % NVS, g = i % NG, k = i / NG, x = k & 1;
+        uint64_t* gq = gbar + 10 * g;
+        if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) break;
+        if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) break;
+        if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+        ptx::tc_fence_after();
+        const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
+        const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
+        const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
+#pragma unroll
+        for (int kk = 0; kk < kRows / 32; ++kk)
+          ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
+                      ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
+        ptx::mma_commit(&vfree[s]);
+        ptx::mma_commit(&gq[6 + x]);
+        last_bar = &vfree[s];
+        last_par = uint32_t(i / NVS) & 1u;
+      }
+      // after an abort, the MMAs already issued finish before TMEM is freed
+      if (i < ntiles && last_bar) drain_wait(last_bar, last_par);
+    }
+    __syncwarp();
+    // ================= then the whole warp: the tokens outside the archive
+    // tiles (last chunk of a kv head), while the groups finish their tiles
+    if (has_extra) {
+      if (a.overlap) ptx::grid_dep_wait();  // tails and new tokens: after the preceding work
+      waiter.wait(qready, 0u);              // the scaled query is in shared memory
+      float* tpo = reinterpret_cast<float*>(sm + C::tp);
+      const float* qsm = reinterpret_cast<const float*>(sm + C::qf);
+      if (a.t_dtype == FC_DTYPE_F32)
+        tail_partial<G, S, R, float>(a, basis, b, h, lane, qsm, tpo);
+      else
+        tail_partial<G, S, R, __nv_bfloat16>(a, basis, b, h, lane, qsm, tpo);
+      ptx::named_bar_arrive(kTailBar, 128 * NG + 32);
+    }
   }
 
   // ================= compute groups
@@ -1073,7 +1123,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (tail_warp) {
+  if (vmma_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
