@@ -99,12 +99,12 @@ struct Cfg {
   static constexpr uint32_t LBO = 16 * NP;         // W operand: K-direction core-matrix stride
   static constexpr int XP = S * (G + 1);           // transpose scratch floats per block
   static constexpr int XW = BW * XP;               // ... per warp
-  static constexpr int kBarsFor(int nvs) { return 2 * NKS + 2 * nvs + 10 * NG + 1; }
+  static constexpr int kBarsFor(int nvs) { return 2 * NKS + 2 * nvs + 10 * NG + 2; }
   // shared memory with nvs V stages (before the 1024-byte alignment slack)
   static constexpr uint32_t bytesFor(int nvs) {
     return (NKS + nvs) * kTileBytes + NP * 128 + nvs * 2 * kScaleBytes + NG * 2 * NP * 128 +
            NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + G * (kD + 4) * 4 + G * kD * 4 +
-           kBarsFor(nvs) * 8 + 16;
+           2 * R * kD * 2 + kBarsFor(nvs) * 8 + 16;
   }
   // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2 each; one: 227 KB
   // (alignment slack included)
@@ -127,7 +127,8 @@ struct Cfg {
   static constexpr uint32_t qs = qu + 64;                     // 4 x G floats: |q| maxima
   static constexpr uint32_t tp = qs + 128;                    // tail partial: G x (acc[D], m, l, pad)
   static constexpr uint32_t qf = tp + G * (kD + 4) * 4;       // scaled query, G x D floats
-  static constexpr uint32_t bars = qf + G * kD * 4;
+  static constexpr uint32_t ts = qf + G * kD * 4;             // bf16 raw rows: K [R][D], V [R][D]
+  static constexpr uint32_t bars = ts + 2 * R * kD * 2;
   static constexpr int kBars = kBarsFor(NVS);
   static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
   static constexpr uint32_t bytes = misc + 16;
@@ -374,7 +375,7 @@ __device__ __forceinline__ void load4(const void* base, int64_t idx, float (&o)[
 // tp + g * (kD + 4): acc[0..kD), m, l). T: the token dtype.
 template <int G, int S, int R, typename T>
 __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<S, R>& basis, int b, int h,
-                                             int lane, const float* qs, float* tp) {
+                                             int lane, const float* qs, float* tp, const unsigned short* rows) {
   constexpr int VEC = kD / 32;
   static_assert(VEC == 4, "four channels per lane");
   const int d0 = lane * VEC;
@@ -462,57 +463,45 @@ __device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<
       }
     }
   } else {
-    // raw tail rows [0, nr), then (step 1) the new token, four at a time:
-    // every row of a batch requested before any is used
+    // raw tail rows [0, nr), then (step 1) the new token, one at a time by a
+    // short rolled loop: from the bf16 rows staged in shared memory (`rows`:
+    // K row t at rows + t D, V row t at rows + (R + t) D), else (fp32 tails)
+    // from global memory
     const int n_raw = a.nr;
     const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
-    constexpr int kB = 4;
-    for (int t0 = 0; t0 < n_tok; t0 += kB) {
-      float kv[kB][VEC], vv[kB][VEC];
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const int tt = t0 + u;
-        if (tt < n_raw) {
-          load4<T>(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + d0, kv[u]);
-          load4<T>(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + d0, vv[u]);
-        } else if (tt < n_tok) {
-          load4<T>(a.kn, b * a.kns_b + h * a.kns_h + d0, kv[u]);
-          load4<T>(a.vn, b * a.vns_b + h * a.vns_h + d0, vv[u]);
-        } else {
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) {
-            kv[u][v] = 0.f;
-            vv[u][v] = 0.f;
-          }
-        }
+#pragma unroll 1
+    for (int tt = 0; tt < n_tok; ++tt) {
+      float kv[VEC], vv[VEC];
+      if (rows) {
+        const uint2 ku = *reinterpret_cast<const uint2*>(rows + tt * kD + d0);
+        const uint2 vu = *reinterpret_cast<const uint2*>(rows + (R + tt) * kD + d0);
+        kv[0] = __uint_as_float(ku.x << 16);
+        kv[1] = __uint_as_float(ku.x & 0xffff0000u);
+        kv[2] = __uint_as_float(ku.y << 16);
+        kv[3] = __uint_as_float(ku.y & 0xffff0000u);
+        vv[0] = __uint_as_float(vu.x << 16);
+        vv[1] = __uint_as_float(vu.x & 0xffff0000u);
+        vv[2] = __uint_as_float(vu.y << 16);
+        vv[3] = __uint_as_float(vu.y & 0xffff0000u);
+      } else if (tt < n_raw) {
+        load4<T>(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + d0, kv);
+        load4<T>(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + d0, vv);
+      } else {
+        load4<T>(a.kn, b * a.kns_b + h * a.kns_h + d0, kv);
+        load4<T>(a.vn, b * a.vns_b + h * a.vns_h + d0, vv);
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float lg[kB], mx = m[g];
+        float x = 0.f;
 #pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          float x = 0.f;
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) x = fmaf(qv[g][v], kv[u][v], x);
-          lg[u] = warp_sum(x);
-          if (t0 + u < n_tok) mx = fmaxf(mx, lg[u]);
-        }
+        for (int v = 0; v < VEC; ++v) x = fmaf(qv[g][v], kv[v], x);
+        const float lg = warp_sum(x);
+        const float mx = fmaxf(m[g], lg);
         const float al = ptx::ex2(m[g] - mx);
-        float ps = 0.f, add[VEC];
+        const float p = ptx::ex2(lg - mx);
+        l[g] = fmaf(l[g], al, p);
 #pragma unroll
-        for (int v = 0; v < VEC; ++v) add[v] = 0.f;
-#pragma unroll
-        for (int u = 0; u < kB; ++u) {
-          if (t0 + u < n_tok) {
-            const float p = ptx::ex2(lg[u] - mx);
-            ps += p;
-#pragma unroll
-            for (int v = 0; v < VEC; ++v) add[v] = fmaf(p, vv[u][v], add[v]);
-          }
-        }
-        l[g] = fmaf(l[g], al, ps);
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(acc[g][v], al, add[v]);
+        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(acc[g][v], al, p * vv[v]);
         m[g] = mx;
       }
     }
@@ -578,6 +567,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   uint64_t* vfree = vfull + NVS;  // V-side MMA done with the stage (-> TMA)
   uint64_t* gbar = vfree + NVS;   // per group: kres[2] kemp[2] wrdy[2] vres[2] vemp[2]
   uint64_t* qready = gbar + 10 * NG;
+  uint64_t* tbar = qready + 1;  // the raw rows landed in shared memory (TMA -> tail warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::misc);
   int* abort_flag = reinterpret_cast<int*>(sm + C::misc + 4);
   int* last_flag = reinterpret_cast<int*>(sm + C::misc + 8);
@@ -631,8 +621,36 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   // scale rows) into stage nv % NVS
   // (under FC_DECODE_OVERLAP the head's last tile, which holds the block the
   // preceding work may have just written, waits for that work)
+  // the raw rows of this kv head (tail rows [0, nr), and a fused step's new
+  // token at row nr) go to shared memory by bulk copies on `tbar`, so that
+  // the tail partial reads no global memory while the archive streams
+  const bool has_extra = c == ns_u - 1 && (a.nr > 0 || a.step != 0);
+  const bool staged = has_extra && a.t_dtype == FC_DTYPE_BF16;
+  bool tail_issued = false;  // (TMA thread)
+  auto load_tail = [&]() {
+    tail_issued = true;
+    constexpr uint32_t kRow = kD * 2;
+    const uint32_t n_new = a.step != 0 ? 1u : 0u;
+    ptx::mbar_arrive_expect_tx(tbar, 2u * (uint32_t(a.nr) + n_new) * kRow);
+    uint8_t* tsm = sm + C::ts;
+    if (a.nr > 0) {
+      ptx::bulk_load(tsm, static_cast<const unsigned short*>(a.kt) + b * a.kts_b + h * a.kts_h,
+                     uint32_t(a.nr) * kRow, tbar);
+      ptx::bulk_load(tsm + R * kRow, static_cast<const unsigned short*>(a.vt) + b * a.vts_b + h * a.vts_h,
+                     uint32_t(a.nr) * kRow, tbar);
+    }
+    if (n_new) {
+      ptx::bulk_load(tsm + a.nr * kRow, static_cast<const unsigned short*>(a.kn) + b * a.kns_b + h * a.kns_h,
+                     kRow, tbar);
+      ptx::bulk_load(tsm + (R + a.nr) * kRow,
+                     static_cast<const unsigned short*>(a.vn) + b * a.vns_b + h * a.vns_h, kRow, tbar);
+    }
+  };
   auto load_k = [&](int nk) {
-    if (a.overlap && tile0 + nk == ta.tiles_per_head - 1) ptx::grid_dep_wait();
+    if (a.overlap && tile0 + nk == ta.tiles_per_head - 1) {
+      ptx::grid_dep_wait();
+      if (staged) load_tail();  // written by the preceding work
+    }
     const int s = nk % NKS;
     ptx::mbar_arrive_expect_tx(&kfull[s], kTileBytes);
     ptx::tma_load_4d(sm + C::kt + s * kTileBytes, &tm_k, &kfull[s], 0, (tile0 + nk) * kRows, h, b);
@@ -673,6 +691,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
         ptx::mbar_init(&gbar[10 * g + 8 + x], 128);  // vemp: the group read the V sums
       }
     ptx::mbar_init(qready, 128);
+    ptx::mbar_init(tbar, 1);
     *abort_flag = 0;
     *last_flag = 0;
     ptx::fence_mbar_init();
@@ -691,8 +710,10 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   // archive until this grid has completed
   if (a.overlap) ptx::grid_dep_launch();
   if (tma_warp && lane == 0) {
-    // fill every stage at once, K and V of a tile together, while group 0
-    // prepares the query limbs
+    // the raw rows first (without FC_DECODE_OVERLAP nothing writes them
+    // concurrently), then every stage at once, K and V of a tile together,
+    // while group 0 prepares the query limbs
+    if (staged && !a.overlap) load_tail();
     const int fk = min(NKS, ntiles), fv = min(NVS, ntiles);
     for (int i = 0; i < fk || i < fv; ++i) {
       if (i < fk) load_k(i);
@@ -818,12 +839,11 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
     // stage was reissued)
     if (*reinterpret_cast<volatile int*>(abort_flag)) {
       if (last_k) drain_wait(last_k, last_kp);
+      if (tail_issued) drain_wait(tbar, 0u);
       for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
       for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
     }
   }
-  const bool last_chunk = c == ns_u - 1;
-  const bool has_extra = last_chunk && (a.nr > 0 || a.step != 0);
   if (vmma_warp) {
     if (lane == 0) {
       // ================= V-MMA thread: Acc_int of each tile, in tile order,
@@ -862,10 +882,13 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
       waiter.wait(qready, 0u);              // the scaled query is in shared memory
       float* tpo = reinterpret_cast<float*>(sm + C::tp);
       const float* qsm = reinterpret_cast<const float*>(sm + C::qf);
-      if (a.t_dtype == FC_DTYPE_F32)
-        tail_partial<G, S, R, float>(a, basis, b, h, lane, qsm, tpo);
-      else
-        tail_partial<G, S, R, __nv_bfloat16>(a, basis, b, h, lane, qsm, tpo);
+      if (staged) {
+        waiter.wait(tbar, 0u);
+        tail_partial<G, S, R, __nv_bfloat16>(a, basis, b, h, lane, qsm, tpo,
+                                             reinterpret_cast<const unsigned short*>(sm + C::ts));
+      } else {
+        tail_partial<G, S, R, float>(a, basis, b, h, lane, qsm, tpo, nullptr);
+      }
       ptx::named_bar_arrive(kTailBar, 128 * NG + 32);
     }
   }
