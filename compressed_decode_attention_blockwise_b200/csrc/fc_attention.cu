@@ -8,12 +8,12 @@
 namespace fc {
 namespace {
 
-// Split count. The tensor-core kernel runs one CTA per SM: with an automatic
-// split the kv heads take ceil(SMs / heads) or one chunk fewer so that the
-// launch has exactly one CTA per SM, and the planner returns the larger
-// count (the workspace's split slots), at most one chunk per 128-row tile.
-// The portable kernel fits four CTAs per SM (registers) and aims at one wave
-// of them, with chunks of at least 16 blocks.
+// Split count. The tensor-core kernel runs one CTA per SM (its two rings of
+// 128-row tiles fill the shared memory): split each kv head into tile-aligned
+// chunks so that all chunks of all kv heads fit in one wave (rounded down:
+// the SMs left over let the next launch on the stream start early). The
+// portable kernel fits four CTAs per SM (registers) and aims at one wave of
+// them, with chunks of at least 16 blocks.
 // Results do not depend on the split beyond rounding.
 int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   if (nb <= 0) return 1;
@@ -21,7 +21,7 @@ int plan_splits(int64_t nb, int64_t B, int64_t Hk, int S, int D) {
   const bool tiles = D == 128 && S >= 1 && 32 % S == 0;
   int64_t ns;
   if (tiles) {
-    ns = (int64_t(sm_count()) + units - 1) / units;
+    ns = int64_t(sm_count()) / units;
     const int64_t t = tc_tiles_per_head(nb, S);
     if (ns > t) ns = t;
   } else {

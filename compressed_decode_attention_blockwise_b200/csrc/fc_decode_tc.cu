@@ -65,56 +65,30 @@ constexpr uint32_t kTileBytes = kRows * kD;
 constexpr uint32_t kScaleBytes = kRows * 4;
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 2 GHz
 constexpr int kFinBar = 8;   // named barrier over every compute warp
-constexpr int kTailBar = 9;  // compute warps + the tail warp: its partial is ready
-constexpr uint32_t kPollNs = 200;  // producer's suspension when nothing is ready
 constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
 
 __host__ __device__ constexpr int pad16(int x) { return (x + 15) / 16 * 16; }
 
-template <int G, int S, int TPT, bool HALF>
+template <int G, int S, int TPT>
 struct Cfg {
   static constexpr int R = S * TPT;
   static constexpr int TB = kRows / S;             // blocks per tile
   static constexpr int BW = 32 / S;                // blocks per warp
   static constexpr int NI = G >= S ? G / S : 1;    // (block, head) items per lane
-  // Two layouts. Full: one CTA per SM with deep rings and four compute
-  // groups of four warps (three where a lane's items need more registers:
-  // eight heads, or eight coefficients per block). HALF (launches with
-  // FC_DECODE_OVERLAP, G <= 4 and S <= 4): two groups and shallow rings in
-  // half an SM (shared memory, registers, TMEM), so that the CTA of the next
-  // launch on the stream (a programmatic dependent) is resident beside this
-  // one and streams its archive while this one drains. Both add a producer
-  // warp (TMA loads, K-side MMAs) and a warp for TMEM, the V-side MMAs and
-  // then the tokens outside the tiles (raw tail, a fused step's new token or
-  // block).
-  static constexpr int kCtasPerSm = HALF ? 2 : 1;
-  static constexpr int NG = HALF ? 2 : (S == 8 || G == 8) ? 3 : 4;
+  // compute groups of four warps (three where a lane's items need more
+  // registers than four groups leave)
+  static constexpr int NG = (S == 8 || G == 8) ? 3 : 4;
   static constexpr int HPG = (G + NG - 1) / NG;    // heads per group in the final merge
   static constexpr int NP = pad16(3 * G);          // MMA N: three limb columns per head
-  static constexpr int NKS = HALF ? 2 : 4;         // K ring stages
-  static constexpr int kThreads = 128 * NG + 64;   // + TMA and MMA warps
+  static constexpr int NKS = 4;                    // K ring stages
+  static constexpr int NVS = NP == 16 ? 7 : 6;     // V ring stages
+  static constexpr int kThreads = 128 * NG + 96;   // + TMA, K-MMA and V-MMA warps
   // per group 2 K and 2 V buffers, allocated as a power of two
-  static constexpr uint32_t kTmemCols = 4 * NP * NG <= 128 ? 128 : 4 * NP * NG <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = 4 * NP * NG <= 256 ? 256 : 512;
   static constexpr uint32_t LBO = 16 * NP;         // W operand: K-direction core-matrix stride
   static constexpr int XP = S * (G + 1);           // transpose scratch floats per block
   static constexpr int XW = BW * XP;               // ... per warp
-  static constexpr int kBarsFor(int nvs) { return 2 * NKS + 2 * nvs + 10 * NG + 2; }
-  // shared memory with nvs V stages (before the 1024-byte alignment slack)
-  static constexpr uint32_t bytesFor(int nvs) {
-    return (NKS + nvs) * kTileBytes + NP * 128 + nvs * 2 * kScaleBytes + NG * 2 * NP * 128 +
-           NG * 4 * XW * 4 + NG * 2 * (G + 1) * 16 + 64 + 128 + G * (kD + 4) * 4 + G * kD * 4 +
-           2 * R * kD * 2 + kBarsFor(nvs) * 8 + 16;
-  }
-  // two CTAs per SM: (228 KB - 2 x 1 KB reserved) / 2 each; one: 227 KB
-  // (alignment slack included)
-  static constexpr uint32_t kSmemCap = kCtasPerSm == 2 ? 115712 : 232448;
-  static constexpr int vStages() {
-    int n = 2;
-    while (n < (HALF ? 3 : 7) && bytesFor(n + 1) + 1024 <= kSmemCap) ++n;
-    return n;
-  }
-  static constexpr int NVS = vStages();  // V ring stages
   // shared memory (offsets from a 1024-byte aligned base)
   static constexpr uint32_t kt = 0;
   static constexpr uint32_t vt = kt + NKS * kTileBytes;
@@ -125,20 +99,16 @@ struct Cfg {
   static constexpr uint32_t red = xs + NG * 4 * XW * 4;      // NG x 2 x (G + 1) x 4 floats
   static constexpr uint32_t qu = red + NG * 2 * (G + 1) * 16;  // G limb units of q
   static constexpr uint32_t qs = qu + 64;                     // 4 x G floats: |q| maxima
-  static constexpr uint32_t tp = qs + 128;                    // tail partial: G x (acc[D], m, l, pad)
-  static constexpr uint32_t qf = tp + G * (kD + 4) * 4;       // scaled query, G x D floats
-  static constexpr uint32_t ts = qf + G * kD * 4;             // bf16 raw rows: K [R][D], V [R][D]
-  static constexpr uint32_t bars = ts + 2 * R * kD * 2;
-  static constexpr int kBars = kBarsFor(NVS);
+  static constexpr uint32_t bars = qs + 128;
+  static constexpr int kBars = 2 * NKS + 2 * NVS + 10 * NG + 1;
   static constexpr uint32_t misc = bars + kBars * 8;          // tmem slot, abort, last
   static constexpr uint32_t bytes = misc + 16;
   static constexpr uint32_t alloc = bytes + 1024;             // alignment slack
-  static_assert(alloc <= kSmemCap, "shared memory");
-  static_assert(bytes == bytesFor(NVS), "layout");
+  static_assert(alloc <= 232448, "shared memory");
   static_assert((NG * G * (kD + 5) + 4) * 4 <= int(NKS * kTileBytes), "merge scratch");
-  static_assert(4 * NP * NG <= int(kTmemCols) && int(kTmemCols) * kCtasPerSm <= 512, "TMEM allocation");
+  static_assert(4 * NP * NG <= 512, "TMEM allocation");
   static_assert(NI * R <= 32, "logits per lane");
-  static_assert(R <= 32, "tail tokens");
+  static_assert(R * HPG <= XW, "tail batch scratch");
 };
 
 struct TcArgs {
@@ -343,197 +313,6 @@ __device__ __forceinline__ void encode_new_block(const DecodeArgs& a, int which,
     run(__nv_bfloat16());
 }
 
-// Four consecutive token elements (16-byte aligned for fp32, 8-byte for
-// bf16) as floats, one vector load.
-template <typename T>
-__device__ __forceinline__ void load4(const void* base, int64_t idx, float (&o)[4]) {
-  if constexpr (sizeof(T) == 4) {
-    const float4 x = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx));
-    o[0] = x.x;
-    o[1] = x.y;
-    o[2] = x.z;
-    o[3] = x.w;
-  } else {
-    const uint2 x = __ldg(reinterpret_cast<const uint2*>(static_cast<const unsigned short*>(base) + idx));
-    o[0] = __uint_as_float(x.x << 16);
-    o[1] = __uint_as_float(x.x & 0xffff0000u);
-    o[2] = __uint_as_float(x.y << 16);
-    o[3] = __uint_as_float(x.y & 0xffff0000u);
-  }
-}
-
-// Softmax partial (base-2 maximum m, sum l, acc[d]) of the tokens that are
-// not in archive tiles, computed by one warp (lane = channels 4 lane ..
-// 4 lane + 3) while the compute groups finish the tiles: the raw-tail rows
-// [0, nr) of kv head (b, h), and in a fused decode step the new token (step
-// 1: also stored at tail row nr) or the block it completes (step 2: tail rows
-// 0..R-2 and the token, encoded into archive slot new_slot with the codec's
-// own device code, exactly as the append kernel does, and folded in the
-// coefficient domain: s_j = scale_k,j C_k[j] . q, logits = A s, w = p A,
-// acc = sum_j w_j scale_v,j C_v[j]). qs: the scaled query (G x kD floats in
-// shared memory). Writes m, l, acc of every head to `tp` (head g at
-// tp + g * (kD + 4): acc[0..kD), m, l). T: the token dtype.
-template <int G, int S, int R, typename T>
-__device__ __forceinline__ void tail_partial(const DecodeArgs& a, const TcBasis<S, R>& basis, int b, int h,
-                                             int lane, const float* qs, float* tp, const unsigned short* rows) {
-  constexpr int VEC = kD / 32;
-  static_assert(VEC == 4, "four channels per lane");
-  const int d0 = lane * VEC;
-  float qv[G][VEC];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float4 x = *reinterpret_cast<const float4*>(qs + g * kD + d0);
-    qv[g][0] = x.x;
-    qv[g][1] = x.y;
-    qv[g][2] = x.z;
-    qv[g][3] = x.w;
-  }
-  float m[G], l[G], acc[G][VEC];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    m[g] = -INFINITY;
-    l[g] = 0.f;
-#pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[g][v] = 0.f;
-  }
-  if (a.step == 2) {
-    encode_new_block<S, R>(a, 0, lane, basis, b, h);
-    encode_new_block<S, R>(a, 1, lane, basis, b, h);
-    __syncwarp();
-    const StreamOut& ko = a.kout;
-    const StreamOut& vo = a.vout;
-    const signed char* kc =
-        static_cast<const signed char*>(ko.coeffs) + b * ko.cs_b + h * ko.cs_h + a.new_slot * S * kD;
-    const signed char* vc =
-        static_cast<const signed char*>(vo.coeffs) + b * vo.cs_b + h * vo.cs_h + a.new_slot * S * kD;
-    const float* ksp = ko.scales + b * ko.ss_b + h * ko.ss_h + a.new_slot * S;
-    const float* vsp = vo.scales + b * vo.ss_b + h * vo.ss_h + a.new_slot * S;
-    // codes and scales written by this warp just above: read through L2
-    float kf[S][VEC], vf[S][VEC], ksc[S], vsc[S];
-#pragma unroll
-    for (int j = 0; j < S; ++j) {
-      const uint32_t kw = __ldcg(reinterpret_cast<const unsigned int*>(kc + j * kD + d0));
-      const uint32_t vw = __ldcg(reinterpret_cast<const unsigned int*>(vc + j * kD + d0));
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) {
-        kf[j][v] = float(int8_t(kw >> (8 * v)));
-        vf[j][v] = float(int8_t(vw >> (8 * v)));
-      }
-      ksc[j] = __ldcg(ksp + j);
-      vsc[j] = __ldcg(vsp + j);
-    }
-    float sj[S][G];
-#pragma unroll
-    for (int j = 0; j < S; ++j)
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float x = 0.f;
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) x = fmaf(kf[j][v], qv[g][v], x);
-        sj[j][g] = warp_sum(x) * ksc[j];
-      }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float lg[R], mx = -INFINITY;
-#pragma unroll
-      for (int tk = 0; tk < R; ++tk) {
-        float v = 0.f;
-#pragma unroll
-        for (int j = 0; j < S; ++j) v = fmaf(basis.m[j][tk], sj[j][g], v);
-        lg[tk] = v;
-        mx = fmaxf(mx, v);
-      }
-      float ps = 0.f, wv[S];
-#pragma unroll
-      for (int j = 0; j < S; ++j) wv[j] = 0.f;
-#pragma unroll
-      for (int tk = 0; tk < R; ++tk) {
-        const float p = ptx::ex2(lg[tk] - mx);
-        ps += p;
-#pragma unroll
-        for (int j = 0; j < S; ++j) wv[j] = fmaf(p, basis.m[j][tk], wv[j]);
-      }
-      m[g] = mx;
-      l[g] = ps;
-#pragma unroll
-      for (int j = 0; j < S; ++j) {
-        const float wj = wv[j] * vsc[j];
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wj, vf[j][v], acc[g][v]);
-      }
-    }
-  } else {
-    // raw tail rows [0, nr), then (step 1) the new token, one at a time by a
-    // short rolled loop: from the bf16 rows staged in shared memory (`rows`:
-    // K row t at rows + t D, V row t at rows + (R + t) D), else (fp32 tails)
-    // from global memory
-    const int n_raw = a.nr;
-    const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
-#pragma unroll 1
-    for (int tt = 0; tt < n_tok; ++tt) {
-      float kv[VEC], vv[VEC];
-      if (rows) {
-        const uint2 ku = *reinterpret_cast<const uint2*>(rows + tt * kD + d0);
-        const uint2 vu = *reinterpret_cast<const uint2*>(rows + (R + tt) * kD + d0);
-        kv[0] = __uint_as_float(ku.x << 16);
-        kv[1] = __uint_as_float(ku.x & 0xffff0000u);
-        kv[2] = __uint_as_float(ku.y << 16);
-        kv[3] = __uint_as_float(ku.y & 0xffff0000u);
-        vv[0] = __uint_as_float(vu.x << 16);
-        vv[1] = __uint_as_float(vu.x & 0xffff0000u);
-        vv[2] = __uint_as_float(vu.y << 16);
-        vv[3] = __uint_as_float(vu.y & 0xffff0000u);
-      } else if (tt < n_raw) {
-        load4<T>(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + d0, kv);
-        load4<T>(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + d0, vv);
-      } else {
-        load4<T>(a.kn, b * a.kns_b + h * a.kns_h + d0, kv);
-        load4<T>(a.vn, b * a.vns_b + h * a.vns_h + d0, vv);
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float x = 0.f;
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) x = fmaf(qv[g][v], kv[v], x);
-        const float lg = warp_sum(x);
-        const float mx = fmaxf(m[g], lg);
-        const float al = ptx::ex2(m[g] - mx);
-        const float p = ptx::ex2(lg - mx);
-        l[g] = fmaf(l[g], al, p);
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(acc[g][v], al, p * vv[v]);
-        m[g] = mx;
-      }
-    }
-    if (a.step == 1) {  // the token joins the tail at row nr (bits copied)
-      const int64_t dk = b * a.kts_b + h * a.kts_h + int64_t(n_raw) * kD + d0;
-      const int64_t dv = b * a.vts_b + h * a.vts_h + int64_t(n_raw) * kD + d0;
-      const int64_t sk = b * a.kns_b + h * a.kns_h + d0, sv = b * a.vns_b + h * a.vns_h + d0;
-      if constexpr (sizeof(T) == 4) {
-        *reinterpret_cast<float4*>(const_cast<float*>(static_cast<const float*>(a.kt)) + dk) =
-            __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.kn) + sk));
-        *reinterpret_cast<float4*>(const_cast<float*>(static_cast<const float*>(a.vt)) + dv) =
-            __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.vn) + sv));
-      } else {
-        using U = unsigned short;
-        *reinterpret_cast<uint2*>(const_cast<U*>(static_cast<const U*>(a.kt)) + dk) =
-            __ldg(reinterpret_cast<const uint2*>(static_cast<const U*>(a.kn) + sk));
-        *reinterpret_cast<uint2*>(const_cast<U*>(static_cast<const U*>(a.vt)) + dv) =
-            __ldg(reinterpret_cast<const uint2*>(static_cast<const U*>(a.vn) + sv));
-      }
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float* o = tp + g * (kD + 4);
-    *reinterpret_cast<float4*>(o + d0) = make_float4(acc[g][0], acc[g][1], acc[g][2], acc[g][3]);
-    if (lane == 0) {
-      o[kD] = m[g];
-      o[kD + 1] = l[g];
-    }
-  }
-}
-
 template <int NP>
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) {
   if constexpr (NP == 16) {
@@ -544,16 +323,17 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) 
   }
 }
 
-template <int G, int S, int TPT, bool HALF>
-__global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT, HALF>::kCtasPerSm)
+template <int G, int S, int TPT>
+__global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                      const TcArgs ta, const TcBasis<S, S * TPT> basis) {
-  using C = Cfg<G, S, TPT, HALF>;
+  using C = Cfg<G, S, TPT>;
   constexpr int R = C::R, NP = C::NP, NI = C::NI, NKS = C::NKS, NVS = C::NVS, XP = C::XP;
   constexpr int NG = C::NG;
   constexpr int NCW = 4 * NG;  // compute warps
   constexpr uint32_t kIdescK = ptx::idesc_i8(128, NP, false, false);
+  constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
   constexpr uint32_t kWBytes = NP * 128;  // one W buffer
 
   const DecodeArgs& a = ta.d;
@@ -567,7 +347,6 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   uint64_t* vfree = vfull + NVS;  // V-side MMA done with the stage (-> TMA)
   uint64_t* gbar = vfree + NVS;   // per group: kres[2] kemp[2] wrdy[2] vres[2] vemp[2]
   uint64_t* qready = gbar + 10 * NG;
-  uint64_t* tbar = qready + 1;  // the raw rows landed in shared memory (TMA -> tail warp)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + C::misc);
   int* abort_flag = reinterpret_cast<int*>(sm + C::misc + 4);
   int* last_flag = reinterpret_cast<int*>(sm + C::misc + 8);
@@ -593,12 +372,16 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   const int Hq = a.Hk * G;
   Waiter waiter{abort_flag, a.status};
 
-  const int tile0 = int(int64_t(c) * ta.tiles_per_head / ns_u);
-  const int tile1 = int(int64_t(c + 1) * ta.tiles_per_head / ns_u);
-  const int ntiles = tile1 - tile0;
+  // chunks of ceil(tiles / ns_u) tiles: the last chunk, which also folds
+  // in the raw tail, gets what is left (at most as many tiles as the others)
+  const int chunk_tiles = (ta.tiles_per_head + ns_u - 1) / ns_u;
+  const int tile0 = c * chunk_tiles;
+  const int tile1 = min(tile0 + chunk_tiles, ta.tiles_per_head);
+  const int ntiles = max(0, tile1 - tile0);
   const bool producer = warp >= NCW;
-  const bool tma_warp = warp == NCW;       // TMA loads and the K-side MMAs (lane 0)
-  const bool vmma_warp = warp == NCW + 1;  // TMEM allocation, V-side MMAs, the tail partial
+  const bool tma_warp = warp == NCW;
+  const bool kmma_warp = warp == NCW + 1;  // also owns the TMEM allocation
+  const bool vmma_warp = warp == NCW + 2;
 
   const int grp = producer ? 0 : warp >> 2;  // compute group
   const int w = warp & 3;                    // warp in the group = TMEM lane quadrant
@@ -621,36 +404,8 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   // scale rows) into stage nv % NVS
   // (under FC_DECODE_OVERLAP the head's last tile, which holds the block the
   // preceding work may have just written, waits for that work)
-  // the raw rows of this kv head (tail rows [0, nr), and a fused step's new
-  // token at row nr) go to shared memory by bulk copies on `tbar`, so that
-  // the tail partial reads no global memory while the archive streams
-  const bool has_extra = c == ns_u - 1 && (a.nr > 0 || a.step != 0);
-  const bool staged = has_extra && a.t_dtype == FC_DTYPE_BF16;
-  bool tail_issued = false;  // (TMA thread)
-  auto load_tail = [&]() {
-    tail_issued = true;
-    constexpr uint32_t kRow = kD * 2;
-    const uint32_t n_new = a.step != 0 ? 1u : 0u;
-    ptx::mbar_arrive_expect_tx(tbar, 2u * (uint32_t(a.nr) + n_new) * kRow);
-    uint8_t* tsm = sm + C::ts;
-    if (a.nr > 0) {
-      ptx::bulk_load(tsm, static_cast<const unsigned short*>(a.kt) + b * a.kts_b + h * a.kts_h,
-                     uint32_t(a.nr) * kRow, tbar);
-      ptx::bulk_load(tsm + R * kRow, static_cast<const unsigned short*>(a.vt) + b * a.vts_b + h * a.vts_h,
-                     uint32_t(a.nr) * kRow, tbar);
-    }
-    if (n_new) {
-      ptx::bulk_load(tsm + a.nr * kRow, static_cast<const unsigned short*>(a.kn) + b * a.kns_b + h * a.kns_h,
-                     kRow, tbar);
-      ptx::bulk_load(tsm + (R + a.nr) * kRow,
-                     static_cast<const unsigned short*>(a.vn) + b * a.vns_b + h * a.vns_h, kRow, tbar);
-    }
-  };
   auto load_k = [&](int nk) {
-    if (a.overlap && tile0 + nk == ta.tiles_per_head - 1) {
-      ptx::grid_dep_wait();
-      if (staged) load_tail();  // written by the preceding work
-    }
+    if (a.overlap && tile0 + nk == ta.tiles_per_head - 1) ptx::grid_dep_wait();
     const int s = nk % NKS;
     ptx::mbar_arrive_expect_tx(&kfull[s], kTileBytes);
     ptx::tma_load_4d(sm + C::kt + s * kTileBytes, &tm_k, &kfull[s], 0, (tile0 + nk) * kRows, h, b);
@@ -691,12 +446,11 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
         ptx::mbar_init(&gbar[10 * g + 8 + x], 128);  // vemp: the group read the V sums
       }
     ptx::mbar_init(qready, 128);
-    ptx::mbar_init(tbar, 1);
     *abort_flag = 0;
     *last_flag = 0;
     ptx::fence_mbar_init();
   }
-  if (vmma_warp) {
+  if (kmma_warp) {
     ptx::tmem_alloc(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -710,10 +464,8 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
   // archive until this grid has completed
   if (a.overlap) ptx::grid_dep_launch();
   if (tma_warp && lane == 0) {
-    // the raw rows first (without FC_DECODE_OVERLAP nothing writes them
-    // concurrently), then every stage at once, K and V of a tile together,
-    // while group 0 prepares the query limbs
-    if (staged && !a.overlap) load_tail();
+    // fill every stage at once, K and V of a tile together, while group 0
+    // prepares the query limbs
     const int fk = min(NKS, ntiles), fv = min(NVS, ntiles);
     for (int i = 0; i < fk || i < fv; ++i) {
       if (i < fk) load_k(i);
@@ -737,10 +489,8 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
       load_q();
     }
     float* qmx = reinterpret_cast<float*>(sm + C::qs);
-    float* qfs = reinterpret_cast<float*>(sm + C::qf);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      qfs[g * kD + t] = qd[g];
       const float mx = warp_max(fabsf(qd[g]));
       if (lane == 0) qmx[w * G + g] = mx;
     }
@@ -765,39 +515,10 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
 
   if (tma_warp && lane == 0) {
     // ================= TMA thread: both rings, in tile order each, whichever
-    // has a free stage (every stage was filled once before the setup
-    // barrier), and the K-side MMA of each tile (S_int into its group's TMEM
-    // buffer) as soon as the tile has landed and the group's buffer is free,
-    // so that K sums run up to 2 NG tiles ahead of the softmax
-    const uint32_t qa = ptx::smem_u32(sm + C::qb);
-    int nm = 0;           // K-side MMAs issued
-    bool q_ok = false;    // the query limbs are in shared memory
-    uint64_t* last_k = nullptr;  // commit barrier and phase of the newest K-side MMA
-    uint32_t last_kp = 0;
+    // has a free stage (every stage was filled once before the setup barrier)
     unsigned long long t_last = clock64();
-    while (nk < ntiles || nv < ntiles || nm < ntiles) {
+    while (nk < ntiles || nv < ntiles) {
       bool prog = false;
-      if (nm < nk) {
-        const int s = nm % NKS, g = nm % NG, k = nm / NG, x = k & 1;
-        uint64_t* gq = gbar + 10 * g;
-        if (!q_ok) q_ok = ptx::mbar_test_wait(qready, 0u);
-        if (q_ok && ptx::mbar_test_wait(&kfull[s], uint32_t(nm / NKS) & 1u) &&
-            ptx::mbar_test_wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) {
-          ptx::tc_fence_after();
-          const uint32_t ka = ptx::smem_u32(sm + C::kt + s * kTileBytes);
-          const uint32_t d = tmem + uint32_t(g * 4 * NP + x * NP);
-#pragma unroll
-          for (int kk = 0; kk < kD / 32; ++kk)
-            ptx::mma_i8(d, ptx::desc_sw128(ka + 32 * kk, 16, 1024), ptx::desc_sw128(qa + 32 * kk, 16, 1024),
-                        kIdescK, kk > 0 ? 1u : 0u);
-          ptx::mma_commit(&kfree[s]);
-          ptx::mma_commit(&gq[x]);
-          last_k = &kfree[s];
-          last_kp = uint32_t(nm / NKS) & 1u;
-          ++nm;
-          prog = true;
-        }
-      }
       if (nk < ntiles && ptx::mbar_test_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u)) {
         load_k(nk++);
         prog = true;
@@ -816,81 +537,61 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
         if (a.status) atomicOr(a.status, 1u);
         break;
       }
-      // nothing ready: a short suspension (bounded) on what the next
-      // K-side MMA lacks, else on the stage the older of the two next loads
-      // needs
-      if (nm < nk) {
-        const int s = nm % NKS, k = nm / NG;
-        if (!q_ok)
-          ptx::mbar_try_wait_ns(qready, 0u, kPollNs);
-        else if (!ptx::mbar_test_wait(&kfull[s], uint32_t(nm / NKS) & 1u))
-          ptx::mbar_try_wait_ns(&kfull[s], uint32_t(nm / NKS) & 1u, kPollNs);
-        else
-          ptx::mbar_try_wait_ns(&gbar[10 * (nm % NG) + 2 + (k & 1)], (uint32_t(k >> 1) & 1u) ^ 1u, kPollNs);
-      } else if (nk < ntiles && (nk <= nv || nv >= ntiles)) {
-        ptx::mbar_try_wait(&kfree[nk % NKS], uint32_t(nk / NKS - 1) & 1u);
-      } else if (nv < ntiles) {
-        ptx::mbar_try_wait(&vfree[nv % NVS], uint32_t(nv / NVS - 1) & 1u);
-      }
+      __nanosleep(32);
     }
-    // after an abort, the K-side MMAs issued finish (the newest commit
-    // tracks every earlier one of this thread) and the newest load of every
-    // stage lands before the CTA exits (older ones completed before their
-    // stage was reissued)
+    // after an abort, the newest load of every stage must land before the
+    // CTA exits (older ones completed before their stage was reissued)
     if (*reinterpret_cast<volatile int*>(abort_flag)) {
-      if (last_k) drain_wait(last_k, last_kp);
-      if (tail_issued) drain_wait(tbar, 0u);
       for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
       for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
     }
   }
-  if (vmma_warp) {
-    if (lane == 0) {
-      // ================= V-MMA thread: Acc_int of each tile, in tile order,
-      // as soon as its W is written (every wait suspends the thread)
-      constexpr uint32_t kIdescV = ptx::idesc_i8(128, NP, true, false);
-      uint64_t* last_bar = nullptr;  // commit barrier and phase of the newest MMA
-      uint32_t last_par = 0;
-      int i = 0;
-      for (; i < ntiles; ++i) {
-        const int s = i % NVS, g = i % NG, k = i / NG, x = k & 1;
-        uint64_t* gq = gbar + 10 * g;
-        if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) break;
-        if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) break;
-        if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
-        ptx::tc_fence_after();
-        const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
-        const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
-        const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
+  if (kmma_warp && lane == 0) {
+    // ================= K-MMA thread: S_int of each tile into its group's
+    // TMEM buffer as soon as it lands
+    waiter.wait(qready, 0u);
+    int i = 0;
+    for (; i < ntiles; ++i) {
+      const int s = i % NKS, g = i % NG, k = i / NG, x = k & 1;
+      uint64_t* gq = gbar + 10 * g;
+      if (!waiter.wait(&kfull[s], uint32_t(i / NKS) & 1u)) break;
+      if (!waiter.wait(&gq[2 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+      ptx::tc_fence_after();
+      const uint32_t ka = ptx::smem_u32(sm + C::kt + s * kTileBytes);
+      const uint32_t qa = ptx::smem_u32(sm + C::qb);
+      const uint32_t d = tmem + uint32_t(g * 4 * NP + x * NP);
 #pragma unroll
-        for (int kk = 0; kk < kRows / 32; ++kk)
-          ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
-                      ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
-        ptx::mma_commit(&vfree[s]);
-        ptx::mma_commit(&gq[6 + x]);
-        last_bar = &vfree[s];
-        last_par = uint32_t(i / NVS) & 1u;
-      }
-      // after an abort, the MMAs already issued finish before TMEM is freed
-      if (i < ntiles && last_bar) drain_wait(last_bar, last_par);
+      for (int kk = 0; kk < kD / 32; ++kk)
+        ptx::mma_i8(d, ptx::desc_sw128(ka + 32 * kk, 16, 1024), ptx::desc_sw128(qa + 32 * kk, 16, 1024),
+                    kIdescK, kk > 0 ? 1u : 0u);
+      ptx::mma_commit(&kfree[s]);
+      ptx::mma_commit(&gq[x]);
     }
-    __syncwarp();
-    // ================= then the whole warp: the tokens outside the archive
-    // tiles (last chunk of a kv head), while the groups finish their tiles
-    if (has_extra) {
-      if (a.overlap) ptx::grid_dep_wait();  // tails and new tokens: after the preceding work
-      waiter.wait(qready, 0u);              // the scaled query is in shared memory
-      float* tpo = reinterpret_cast<float*>(sm + C::tp);
-      const float* qsm = reinterpret_cast<const float*>(sm + C::qf);
-      if (staged) {
-        waiter.wait(tbar, 0u);
-        tail_partial<G, S, R, __nv_bfloat16>(a, basis, b, h, lane, qsm, tpo,
-                                             reinterpret_cast<const unsigned short*>(sm + C::ts));
-      } else {
-        tail_partial<G, S, R, float>(a, basis, b, h, lane, qsm, tpo, nullptr);
-      }
-      ptx::named_bar_arrive(kTailBar, 128 * NG + 32);
+    // after an abort, the MMAs already issued finish before TMEM is freed
+    if (i < ntiles && i > 0) drain_wait(&kfree[(i - 1) % NKS], uint32_t((i - 1) / NKS) & 1u);
+  }
+  if (vmma_warp && lane == 0) {
+    // ================= V-MMA thread: Acc_int of each tile as soon as its W is
+    // written
+    int i = 0;
+    for (; i < ntiles; ++i) {
+      const int s = i % NVS, g = i % NG, k = i / NG, x = k & 1;
+      uint64_t* gq = gbar + 10 * g;
+      if (!waiter.wait(&vfull[s], uint32_t(i / NVS) & 1u)) break;
+      if (!waiter.wait(&gq[4 + x], uint32_t(k >> 1) & 1u)) break;
+      if (!waiter.wait(&gq[8 + x], (uint32_t(k >> 1) & 1u) ^ 1u)) break;
+      ptx::tc_fence_after();
+      const uint32_t va = ptx::smem_u32(sm + C::vt + s * kTileBytes);
+      const uint32_t wa = ptx::smem_u32(sm + C::wb + (g * 2 + x) * kWBytes);
+      const uint32_t d = tmem + uint32_t(g * 4 * NP + 2 * NP + x * NP);
+#pragma unroll
+      for (int kk = 0; kk < kRows / 32; ++kk)
+        ptx::mma_i8(d, ptx::desc_sw128(va + 4096 * kk, kTileBytes, 1024),
+                    ptx::desc_noswizzle(wa + kk * 2 * C::LBO, C::LBO, 128), kIdescV, kk > 0 ? 1u : 0u);
+      ptx::mma_commit(&vfree[s]);
+      ptx::mma_commit(&gq[6 + x]);
     }
+    if (i < ntiles && i > 0) drain_wait(&vfree[(i - 1) % NVS], uint32_t((i - 1) / NVS) & 1u);
   }
 
   // ================= compute groups
@@ -1077,7 +778,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
     for (int ii = 0; ii < NI; ++ii)
 #pragma unroll
       for (int o = S; o < 32; o <<= 1) lsum[ii] += __shfl_xor_sync(0xffffffffu, lsum[ii], o);
-    // the workspace and out: after the preceding work
+    // the tails, the workspace and out: after the preceding work
     if (a.overlap) ptx::grid_dep_wait();
     // every group is done with both rings: the K ring becomes merge scratch
     ptx::named_bar_sync(kFinBar, 128 * NG);
@@ -1095,26 +796,19 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
 #pragma unroll
     for (int g = 0; g < G; ++g) fa[(grp * G + g) * kD + t] = acc[g];
     ptx::named_bar_sync(kFinBar, 128 * NG);
-    // the tail warp's partial (last chunk with raw tokens or a new token)
-    if (has_extra) ptx::named_bar_sync(kTailBar, 128 * NG + 32);
-    const float* tpart = reinterpret_cast<const float*>(sm + C::tp);
 
-    // group grp finishes heads grp, grp + NG, ...: thread t = channel d
+    // group grp finishes heads grp, grp + 4, ...: thread t = channel d
     constexpr int HPG = C::HPG;
-    const bool active = grp < G;  // uniform per group
+    float Mh[HPG], Lh[HPG], Ah[HPG];
 #pragma unroll
     for (int y = 0; y < HPG; ++y) {
-      const int g = grp + NG * y;
-      if (!active || g >= G) continue;
+      const int g = min(grp + NG * y, G - 1);
       float M = -INFINITY;
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) {
         const float4 l4 = reinterpret_cast<const float4*>(fl)[gg * G + g];
         if (l4.x + l4.y + l4.z + l4.w > 0.f) M = fmaxf(M, fm[gg * G + g]);
       }
-      const float* tg = tpart + g * (kD + 4);
-      const float tl = has_extra ? tg[kD + 1] : 0.f;
-      if (tl > 0.f) M = fmaxf(M, tg[kD]);
       float Ls = 0.f, As = 0.f;
 #pragma unroll
       for (int gg = 0; gg < NG; ++gg) {
@@ -1126,27 +820,177 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT, HALF>::kThreads, Cfg<G, S, TPT,
           As = fmaf(fa[(gg * G + g) * kD + t], e, As);
         }
       }
-      if (tl > 0.f) {
-        const float e = ptx::ex2(tg[kD] - M);
-        Ls = fmaf(tl, e, Ls);
-        As = fmaf(tg[t], e, As);
+      Mh[y] = M;
+      Lh[y] = Ls;
+      Ah[y] = As;
+    }
+    const bool active = grp < G;  // uniform per group
+    const bool last_chunk = c == ns_u - 1;
+    // fused decode step whose token completes a block: warps 0 and 1 of group
+    // 0 encode it (tail rows 0..R-2 and the new token) into archive slot
+    // new_slot with the codec's own device code, so the archive is bitwise
+    // what fc_append_step writes; the barrier publishes codes and scales to
+    // the CTA
+    if (last_chunk && a.step == 2) {
+      if (grp == 0 && w < 2) encode_new_block<S, S * TPT>(a, w, lane, basis, b, h);
+      ptx::named_bar_sync(kFinBar, 128 * NG);
+    }
+    // raw tail tokens, then the step's new token or block (last chunk)
+    if (active && last_chunk && (a.nr > 0 || a.step != 0)) {
+      float* red2 = reinterpret_cast<float*>(sm + C::xs) + grp * 4 * C::XW;
+      float qh[HPG];
+#pragma unroll
+      for (int y = 0; y < HPG; ++y) {
+        const int g = min(grp + NG * y, G - 1);
+        qh[y] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
       }
-      const int hq = h * G + g;
-      if (direct) {
-        store_out(a.out, b * a.os_b + hq * a.os_h + t, a.out_dtype, As / Ls);
-      } else {
-        const int64_t row = (int64_t(b) * Hq + hq) * a.ns + c;
-        a.pacc[row * kD + t] = As;
-        if (t == 0) {
-          a.pm[row] = Ls > 0.f ? M : -INFINITY;
-          a.pl[row] = Ls;
+      // the raw tokens of the tail, and the step's new token, in one batch:
+      // one reduction over the group for every logit, then one online-softmax
+      // update (thread t = channel d)
+      const int n_raw = a.step == 2 ? 0 : a.nr;  // a completed block is folded coded
+      const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
+      constexpr int kTok = S * TPT;  // at most R tokens: R - 1 tail rows + the new one
+      if (n_tok > 0) {
+        float kv[kTok], vv[kTok];
+#pragma unroll
+        for (int tt = 0; tt < kTok; ++tt) {
+          kv[tt] = 0.f;
+          vv[tt] = 0.f;
+          if (tt < n_raw) {
+            kv[tt] = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, a.t_dtype);
+            vv[tt] = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, a.t_dtype);
+          } else if (tt == n_raw && a.step == 1) {
+            kv[tt] = load_any(a.kn, b * a.kns_b + h * a.kns_h + t, a.t_dtype);
+            vv[tt] = load_any(a.vn, b * a.vns_b + h * a.vns_h + t, a.t_dtype);
+          }
+        }
+        float lgt[kTok][HPG];
+#pragma unroll
+        for (int tt = 0; tt < kTok; ++tt)
+#pragma unroll
+          for (int y = 0; y < HPG; ++y) lgt[tt][y] = tt < n_tok ? warp_sum(qh[y] * kv[tt]) : 0.f;
+        if (lane == 0) {
+#pragma unroll
+          for (int tt = 0; tt < kTok; ++tt)
+#pragma unroll
+            for (int y = 0; y < HPG; ++y) red2[(w * kTok + tt) * HPG + y] = lgt[tt][y];
+        }
+        ptx::named_bar_sync(1 + grp, 128);
+#pragma unroll
+        for (int tt = 0; tt < kTok; ++tt)
+#pragma unroll
+          for (int y = 0; y < HPG; ++y)
+            lgt[tt][y] = red2[(0 * kTok + tt) * HPG + y] + red2[(1 * kTok + tt) * HPG + y] +
+                         red2[(2 * kTok + tt) * HPG + y] + red2[(3 * kTok + tt) * HPG + y];
+        ptx::named_bar_sync(1 + grp, 128);  // red2 is reused below
+#pragma unroll
+        for (int y = 0; y < HPG; ++y) {
+          float mn = Mh[y];
+#pragma unroll
+          for (int tt = 0; tt < kTok; ++tt)
+            if (tt < n_tok) mn = fmaxf(mn, lgt[tt][y]);
+          const float al = ptx::ex2(Mh[y] - mn);
+          float ps = 0.f, add = 0.f;
+#pragma unroll
+          for (int tt = 0; tt < kTok; ++tt) {
+            if (tt < n_tok) {
+              const float p = ptx::ex2(lgt[tt][y] - mn);
+              ps += p;
+              add = fmaf(p, vv[tt], add);
+            }
+          }
+          Ah[y] = fmaf(Ah[y], al, add);
+          Lh[y] = fmaf(Lh[y], al, ps);
+          Mh[y] = mn;
+        }
+      }
+      if (a.step == 1 && grp == 0) {  // the token joins the tail at row nr
+        copy_elem(a.kt, b * a.kts_b + h * a.kts_h + int64_t(a.nr) * kD + t, a.kn,
+                  b * a.kns_b + h * a.kns_h + t, a.t_dtype);
+        copy_elem(a.vt, b * a.vts_b + h * a.vts_h + int64_t(a.nr) * kD + t, a.vn,
+                  b * a.vns_b + h * a.vns_h + t, a.t_dtype);
+      }
+      if (a.step == 2) {
+        // the new block in the coefficient domain, as a tile row set would be:
+        // s_j = scale_k,j C_k[j] . q, logits = A s, p, w = p A, acc += w scale_v C_v
+        const StreamOut& ko = a.kout;
+        const StreamOut& vo = a.vout;
+        // (written by this CTA before the barrier above: read through L2)
+        const signed char* kc = static_cast<const signed char*>(ko.coeffs) + b * ko.cs_b + h * ko.cs_h + a.new_slot * S * kD;
+        const signed char* vc = static_cast<const signed char*>(vo.coeffs) + b * vo.cs_b + h * vo.cs_h + a.new_slot * S * kD;
+        const float* ksp = ko.scales + b * ko.ss_b + h * ko.ss_h + a.new_slot * S;
+        const float* vsp = vo.scales + b * vo.ss_b + h * vo.ss_h + a.new_slot * S;
+        float ksc[S], vsc[S];
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+          ksc[j] = __ldcg(ksp + j);
+          vsc[j] = __ldcg(vsp + j);
+        }
+        float sj[S * HPG];
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+          const float kv = float(__ldcg(kc + j * kD + t));
+#pragma unroll
+          for (int y = 0; y < HPG; ++y) sj[j * HPG + y] = kv * qh[y];
+        }
+        group_sum<S * HPG>(sj, red2, w, lane, 1 + grp);
+        float vcode[S];
+#pragma unroll
+        for (int j = 0; j < S; ++j) vcode[j] = float(__ldcg(vc + j * kD + t));
+#pragma unroll
+        for (int y = 0; y < HPG; ++y) {
+          float lg[S * TPT];
+          float mx = Mh[y];
+#pragma unroll
+          for (int tk = 0; tk < S * TPT; ++tk) {
+            float v = 0.f;
+#pragma unroll
+            for (int j = 0; j < S; ++j) v = fmaf(basis.m[j][tk], sj[j * HPG + y] * ksc[j], v);
+            lg[tk] = v;
+            mx = fmaxf(mx, v);
+          }
+          const float al = ptx::ex2(Mh[y] - mx);
+          float ps = 0.f, wv[S];
+#pragma unroll
+          for (int j = 0; j < S; ++j) wv[j] = 0.f;
+#pragma unroll
+          for (int tk = 0; tk < S * TPT; ++tk) {
+            const float p = ptx::ex2(lg[tk] - mx);
+            ps += p;
+#pragma unroll
+            for (int j = 0; j < S; ++j) wv[j] = fmaf(p, basis.m[j][tk], wv[j]);
+          }
+          float add = 0.f;
+#pragma unroll
+          for (int j = 0; j < S; ++j) add = fmaf(wv[j] * vsc[j], vcode[j], add);
+          Ah[y] = fmaf(Ah[y], al, add);
+          Lh[y] = fmaf(Lh[y], al, ps);
+          Mh[y] = mx;
+        }
+      }
+    }
+    if (active) {
+#pragma unroll
+      for (int y = 0; y < HPG; ++y) {
+        const int g = grp + NG * y;
+        if (g >= G) continue;
+        const int hq = h * G + g;
+        if (direct) {
+          store_out(a.out, b * a.os_b + hq * a.os_h + t, a.out_dtype, Ah[y] / Lh[y]);
+        } else {
+          const int64_t row = (int64_t(b) * Hq + hq) * a.ns + c;
+          a.pacc[row * kD + t] = Ah[y];
+          if (t == 0) {
+            a.pm[row] = Lh[y] > 0.f ? Mh[y] : -INFINITY;
+            a.pl[row] = Lh[y];
+          }
         }
       }
     }
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (vmma_warp) {
+  if (kmma_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -1207,7 +1051,7 @@ bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G, int S, int TPT, bool HALF>
+template <int G, int S, int TPT>
 int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CUtensorMap* maps,
            cudaStream_t stream) {
   TcBasis<S, S * TPT> basis;
@@ -1216,14 +1060,10 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
       basis.m[j][t] = full.m[j][t];
       basis.m64[j][t] = full64.m[j][t];
     }
-  using C = Cfg<G, S, TPT, HALF>;
+  using C = Cfg<G, S, TPT>;
   const size_t smem = C::alloc;
-  auto kern = decode_tc_kernel<G, S, TPT, HALF>;
-  // the whole unified L1 / shared memory as shared memory, so that two CTAs
-  // fit on an SM
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess ||
-      cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           int(cudaSharedmemCarveoutMaxShared)) != cudaSuccess)
+  auto kern = decode_tc_kernel<G, S, TPT>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return FC_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   const unsigned units = unsigned(ta.d.B) * unsigned(ta.d.Hk);
@@ -1267,30 +1107,18 @@ int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive
   ta.d = d;
   ta.tiles_per_head = tc_tiles_per_head(d.nb, d.S);
   const int64_t units = int64_t(d.B) * d.Hk;
-  if (d.auto_split) {
-    // one CTA per SM (or one per kv head when there are more of them): the
-    // chunk counts of the kv heads differ by at most one
-    const int64_t ctas = units >= sm_count() ? units : std::min<int64_t>(sm_count(), units * ta.tiles_per_head);
-    ta.d.bal_q = int(ctas / units);
-    ta.d.bal_rem = int(ctas % units);
-    if (ta.d.bal_q + (ta.d.bal_rem > 0 ? 1 : 0) > d.ns) return FC_ERR_INVALID;
-  } else {
-    ta.d.bal_q = d.ns;
-    ta.d.bal_rem = 0;
-  }
+  (void)units;
+  ta.d.bal_q = d.ns;  // every kv head takes ns chunks
+  ta.d.bal_rem = 0;
   CUtensorMap maps[4];
   const int64_t rows = d.nb * d.S;
   if (!tc::make_code_map(&maps[0], ka, rows) || !tc::make_code_map(&maps[1], va, rows) ||
       !tc::make_scale_map(&maps[2], ka, rows) || !tc::make_scale_map(&maps[3], va, rows))
     return FC_ERR_CUDA;
   const int key = d.G * 10000 + d.S * 100 + d.R / d.S;
-  // the half-SM layout serves overlapped launches where its registers suffice
-  const bool half = d.overlap && d.G <= 4 && d.S <= 4;
   switch (key) {
-#define FC_TC_CASE(G, S, T)                                                                              \
-  case G * 10000 + S * 100 + T:                                                                         \
-    return half ? tc::launch<G, S, T, (G <= 4 && S <= 4)>(ta, basis, basis64, maps, stream)              \
-                : tc::launch<G, S, T, false>(ta, basis, basis64, maps, stream);
+#define FC_TC_CASE(G, S, T) \
+  case G * 10000 + S * 100 + T: return tc::launch<G, S, T>(ta, basis, basis64, maps, stream);
     FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
     FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
     FC_TC_CASE(1, 2, 4) FC_TC_CASE(2, 2, 4) FC_TC_CASE(4, 2, 4) FC_TC_CASE(8, 2, 4)

@@ -215,15 +215,13 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *              there is no mask. n_blocks == 0 is allowed (tail-only softmax);
  *              n_blocks == 0 with an empty tail is FC_ERR_INVALID.
  *   softmax_scale   sigma; <= 0 selects D^-0.5.
- *   num_splits      split-K chunks per kv head; 0 = automatic. Chunks
- *                   partition each kv head's blocks contiguously and in order
- *                   (the kernel places the boundaries: on whole 128-row
- *                   coefficient tiles on the tensor-core kernel); the raw tail
- *                   belongs to the last chunk. Automatic: fc_decode_plan's
- *                   count, which is also the workspace's split slots; with
- *                   FC_DECODE_FUSE_COMBINE the tensor-core kernel gives each
- *                   kv head that many chunks or one fewer, so that the launch
- *                   has one CTA per SM.
+ *   num_splits      split-K chunks per kv head, 0 = fc_decode_plan's
+ *                   choice. Chunks partition each kv head's blocks
+ *                   contiguously and in order: c * chunk .. (c + 1) * chunk
+ *                   with chunk = ceil(n / num_splits) of the kernel's units
+ *                   (blocks; whole 128-row coefficient tiles on the
+ *                   tensor-core kernel), so the last chunk may be shorter or
+ *                   empty; the raw tail belongs to the last chunk.
  *   flags      FC_DECODE_FUSE_COMBINE: the last CTA to finish a kv head
  *              merges the partials and writes `out` (one launch, no
  *              spin-waits: an atomic ticket); without it only the partials
@@ -233,9 +231,7 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *              S dividing 32, R / S in {2, 4, 8}, G <= 8).
  *              FC_DECODE_OVERLAP (tensor-core kernel; ignored otherwise):
  *              launch as a programmatic dependent of the preceding work on
- *              `stream`, in a layout that takes half an SM where G <= 4 and
- *              S <= 4, so that this launch's CTAs run beside the preceding
- *              launch's. The kernel then streams archive blocks
+ *              `stream`. The kernel then streams archive blocks
  *              [0, n_blocks - 1) while that work is still running, and waits
  *              for it before it reads q, the tails or block n_blocks - 1 and
  *              before it writes the workspace or `out`. Precondition: no

@@ -213,17 +213,16 @@ def test_product_path_has_no_oracle_or_fallback():
 def test_split_planner():
     """fc_decode_plan on the host (148 SMs: the B200 count, also the
     fallback when no device is visible). Tensor-core shapes (int8, D = 128):
-    the automatic split runs one CTA per SM, the (b, kv head) pairs taking
-    ceil(148 / pairs) chunks or one fewer; the plan is the larger count, at
-    most one chunk per 128-row tile. Other shapes: four CTAs per SM rounded
-    down to one wave, at least 16 blocks per split."""
+    one CTA per SM over the (b, kv head) pairs, rounded down, at most one
+    split per 128-row tile. Other shapes: four CTAs per SM rounded down to
+    one wave, at least 16 blocks per split."""
     def plan(B, H, D, R, S, nb, Hq, dt=_lib.FC_DTYPE_I8):
         a = _arc(B=B, H=H, D=D, R=R, S=S, dtype=dt, cap=nb, nb=nb)
         return _lib.fc_decode_plan(a, None, Hq)
 
-    assert plan(1, 8, 128, 16, 4, 8192, 32) == 19      # long: 4 x 19 + 4 x 18
+    assert plan(1, 8, 128, 16, 4, 8192, 32) == 18      # long: 144 CTAs
     assert plan(1, 8, 128, 16, 4, 40, 32) == 2         # capped by 2 tiles
-    assert plan(8, 8, 128, 8, 2, 512, 32) == 3         # gqa: 20 x 3 + 44 x 2
+    assert plan(8, 8, 128, 8, 2, 512, 32) == 2         # gqa: 64 pairs
     assert plan(64, 8, 64, 8, 3, 1024, 64) == 1        # 512 pairs > 148 * 4 / 2
     assert plan(16, 8, 64, 8, 3, 1024, 64) == 4        # floor(592 / 128)
     assert plan(1, 4, 64, 8, 2, 32, 4, _lib.FC_DTYPE_F32) == 2  # nb / 16
