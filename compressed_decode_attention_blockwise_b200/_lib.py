@@ -35,6 +35,9 @@ FC_KERNEL_TENSOR_CORE = 1
 
 FC_SELECT_MAX_BATCH = 1024
 
+FC_CODEC_DCT = 0
+FC_CODEC_PNG = 1
+
 FC_DTYPE_F32 = 0
 FC_DTYPE_BF16 = 1
 FC_DTYPE_I8 = 2
@@ -64,7 +67,7 @@ class FcArchive(ctypes.Structure):
     _fields_ = [
         ("coeffs", ctypes.c_void_p), ("scales", ctypes.c_void_p),
         ("coeff_dtype", ctypes.c_int32), ("R", ctypes.c_int32),
-        ("S", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("S", ctypes.c_int32), ("codec", ctypes.c_int32),
         ("B", ctypes.c_int64), ("H", ctypes.c_int64), ("D", ctypes.c_int64),
         ("capacity", ctypes.c_int64), ("n_blocks", ctypes.c_int64),
         ("coeff_stride_b", ctypes.c_int64), ("coeff_stride_h", ctypes.c_int64),

@@ -37,10 +37,13 @@ def grown_capacity(capacity: int, need: int) -> int:
 
 
 class CodecStream:
-    """One (B, H, T, D) K or V stream on the device."""
+    """One (B, H, T, D) K or V stream on the device. ``codec`` is "dct" (the
+    block DCT, S kept rows) or "png" (the lossless tier: anchor and fp32
+    first differences, S = R, coeff "f32")."""
 
     def __init__(self, B: int, H: int, D: int, R: int, S: int, coeff: str,
-                 token_dtype: torch.dtype, device, capacity: int = 0):
+                 token_dtype: torch.dtype, device, capacity: int = 0,
+                 codec: str = "dct"):
         self.B, self.H, self.D, self.R, self.S = B, H, D, R, S
         self.coeff = coeff
         self.token_dtype = token_dtype
@@ -52,6 +55,9 @@ class CodecStream:
         self.arc = _lib.FcArchive()
         self.arc.coeff_dtype = _lib.dtype_code(_COEFF[coeff])
         self.arc.R, self.arc.S = R, S
+        self.codec = codec
+        self.arc.codec = {"dct": _lib.FC_CODEC_DCT,
+                          "png": _lib.FC_CODEC_PNG}[codec]
         self.arc.B, self.arc.H, self.arc.D = B, H, D
         self.tail_desc = _lib.FcTail()
         self.tail_desc.data = self.tail.data_ptr()
@@ -256,17 +262,23 @@ class CodecKVCache:
 
     ``coeff_k`` / ``coeff_v`` choose the archive storage: "i8" (int8 codes
     with one fp32 scale per (block, frequency)), "bf16" or "f32".
+    ``codec="png"`` selects the lossless PNG tier (anchor + fp32 first
+    differences, flashcodec-kv README "Math"): S becomes R and both streams
+    store fp32 rows.
     """
 
     def __init__(self, B: int, Hk: int, D: int, R: int = 8, S: int = 2,
                  coeff_k: str = "i8", coeff_v: str = "i8",
                  token_dtype: torch.dtype = torch.bfloat16, device="cuda",
-                 capacity: int = 0):
+                 capacity: int = 0, codec: str = "dct"):
+        if codec == "png":
+            S, coeff_k, coeff_v = R, "f32", "f32"
         self.B, self.Hk, self.D, self.R, self.S = B, Hk, D, R, S
+        self.codec = codec
         self.k = CodecStream(B, Hk, D, R, S, coeff_k, token_dtype, device,
-                             capacity)
+                             capacity, codec)
         self.v = CodecStream(B, Hk, D, R, S, coeff_v, token_dtype, device,
-                             capacity)
+                             capacity, codec)
         self.device = self.k.device
         self._ws: Optional[torch.Tensor] = None
         self._plans: dict = {}      # (Hq, n_blocks) -> split count

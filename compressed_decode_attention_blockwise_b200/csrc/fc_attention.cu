@@ -197,7 +197,7 @@ int prepare_decode(const void* q, int32_t q_dtype, const int64_t* q_strides, int
 int launch_prepared(const DecodeArgs& a, const fc_archive* ka, const fc_archive* va, int32_t flags,
                     cudaStream_t stream) {
   Basis basis;
-  make_basis(ka->R, ka->S, &basis);
+  make_basis(ka->codec, ka->R, ka->S, &basis);
   if (!(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, a.G))
     return launch_decode_tc(a, ka, va, basis, stream);
   const int kd = ka->coeff_dtype, vd = va->coeff_dtype;

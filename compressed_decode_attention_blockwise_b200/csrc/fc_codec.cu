@@ -388,7 +388,7 @@ extern "C" int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t*
   a.ts_h = tail ? tail->stride_h : 0;
   a.n_rem = n_rem;
   BasisF64 basis;
-  make_basis_f64(arc->R, arc->S, &basis);
+  make_basis_f64(arc->codec, arc->R, arc->S, &basis);
   const int64_t warps = arc->B * arc->H * n_full + (copy_tail ? arc->B * arc->H : 0);
   const int64_t grid = (warps + 7) / 8;
   if (grid > 0x7fffffffLL) return FC_ERR_UNSUPPORTED;
@@ -480,7 +480,7 @@ extern "C" int fc_append_step(const void* k_new, const void* v_new, int32_t dtyp
   a.complete = complete ? 1 : 0;
   a.slot = ka->n_blocks;
   BasisF64 basis;
-  make_basis_f64(ka->R, ka->S, &basis);
+  make_basis_f64(ka->codec, ka->R, ka->S, &basis);
   const int64_t warps = 2 * ka->B * ka->H;
   const int64_t grid = (warps + 7) / 8;
   st = dispatch_vec(a.D, [&](auto vec) {

@@ -1084,6 +1084,7 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
 // Whether the tensor-core kernel serves this problem.
 bool decode_tc_eligible(const fc_archive* ka, const fc_archive* va, int G) {
   if (ka->coeff_dtype != FC_DTYPE_I8 || va->coeff_dtype != FC_DTYPE_I8) return false;
+  if (ka->codec != FC_CODEC_DCT || va->codec != FC_CODEC_DCT) return false;
   if (ka->D != tc::kD || ka->n_blocks < 1) return false;
   const int S = ka->S, R = ka->R;
   if (R % S) return false;
@@ -1102,7 +1103,7 @@ int tc_tiles_per_head(int64_t nb, int S) { return int((nb + (tc::kRows / S) - 1)
 int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive* va, const Basis& basis,
                      cudaStream_t stream) {
   BasisF64 basis64;
-  make_basis_f64(d.R, d.S, &basis64);
+  make_basis_f64(FC_CODEC_DCT, d.R, d.S, &basis64);
   tc::TcArgs ta;
   ta.d = d;
   ta.tiles_per_head = tc_tiles_per_head(d.nb, d.S);

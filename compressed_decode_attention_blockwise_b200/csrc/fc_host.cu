@@ -7,30 +7,47 @@
 
 namespace fc {
 
-void make_basis(int R, int S, Basis* out) {
-  // Orthonormal DCT-II rows (flashcodec-kv README, "Math"):
-  // M[j][t] = c_j cos(pi / R (t + 1/2) j), c_0 = sqrt(1/R), c_j = sqrt(2/R).
+namespace {
+
+// Orthonormal DCT-II rows (flashcodec-kv README, "Math"):
+// M[j][t] = c_j cos(pi / R (t + 1/2) j), c_0 = sqrt(1/R), c_j = sqrt(2/R); the
+// same matrix encodes (C = M X) and, transposed, decodes (X = M^T C).
+double dct_entry(int R, int j, int t) {
   const double pi = 3.14159265358979323846;
+  const double c = (j == 0) ? std::sqrt(1.0 / R) : std::sqrt(2.0 / R);
+  return c * std::cos(pi / R * (t + 0.5) * j);
+}
+
+// PNG lossless tier (flashcodec-kv README, "Math", PNG bullet): the block is
+// stored as its first token (anchor) and the first differences
+// Delta_j = x_j - x_{j-1}, so encoding row j takes x_j - x_{j-1} (row 0: x_0)
+// and decoding is the cumulative sum x_t = sum_{j <= t} row_j.
+double png_encode_entry(int j, int t) {
+  if (j == 0) return t == 0 ? 1.0 : 0.0;
+  return t == j ? 1.0 : (t == j - 1 ? -1.0 : 0.0);
+}
+double png_decode_entry(int j, int t) { return j <= t ? 1.0 : 0.0; }
+
+}  // namespace
+
+// Decoding rows: X[t] = sum_j m[j][t] C[j] (fp32; the DCT rows, or the
+// cumulative-sum rows of the PNG tier).
+void make_basis(int codec, int R, int S, Basis* out) {
   for (int j = 0; j < kMaxS; ++j)
     for (int t = 0; t < kMaxR; ++t) {
       double v = 0.0;
-      if (j < S && t < R) {
-        const double c = (j == 0) ? std::sqrt(1.0 / R) : std::sqrt(2.0 / R);
-        v = c * std::cos(pi / R * (t + 0.5) * j);
-      }
+      if (j < S && t < R) v = codec == FC_CODEC_PNG ? png_decode_entry(j, t) : dct_entry(R, j, t);
       out->m[j][t] = static_cast<float>(v);
     }
 }
 
-void make_basis_f64(int R, int S, BasisF64* out) {
-  const double pi = 3.14159265358979323846;
+// Encoding rows: C[j] = sum_t m[j][t] X[t] (fp64; the DCT rows, or the
+// anchor / first-difference rows of the PNG tier).
+void make_basis_f64(int codec, int R, int S, BasisF64* out) {
   for (int j = 0; j < kMaxS; ++j)
     for (int t = 0; t < kMaxR; ++t) {
       double v = 0.0;
-      if (j < S && t < R) {
-        const double c = (j == 0) ? std::sqrt(1.0 / R) : std::sqrt(2.0 / R);
-        v = c * std::cos(pi / R * (t + 0.5) * j);
-      }
+      if (j < S && t < R) v = codec == FC_CODEC_PNG ? png_encode_entry(j, t) : dct_entry(R, j, t);
       out->m[j][t] = v;
     }
 }
@@ -60,6 +77,10 @@ int check_archive(const fc_archive* a) {
   const bool quant = a->coeff_dtype == FC_DTYPE_I8;
   if (quant != (a->scales != nullptr)) return FC_ERR_INVALID;
   if (a->B < 1 || a->H < 1 || a->R < 1 || a->S < 1 || a->S > a->R) return FC_ERR_INVALID;
+  if (a->codec != FC_CODEC_DCT && a->codec != FC_CODEC_PNG) return FC_ERR_INVALID;
+  // the PNG tier keeps every row (S = R) in fp32 (deltas are always fp32)
+  if (a->codec == FC_CODEC_PNG && (a->S != a->R || a->R < 2 || a->coeff_dtype != FC_DTYPE_F32))
+    return FC_ERR_INVALID;
   if (a->R > kMaxR || a->S > kMaxS || !supported_D(a->D)) return FC_ERR_UNSUPPORTED;
   if (a->capacity < 0 || a->n_blocks < 0 || a->n_blocks > a->capacity) return FC_ERR_INVALID;
   if (!aligned16(a->coeffs) || (quant && !aligned16(a->scales))) return FC_ERR_INVALID;

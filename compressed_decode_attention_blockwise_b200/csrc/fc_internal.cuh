@@ -19,15 +19,19 @@ struct Basis {
   float m[kMaxS][kMaxR];
 };
 
-// Host: fills M[j][t] = c_j cos(pi / R (t + 1/2) j) in double, rounded to fp32.
-void make_basis(int R, int S, Basis* out);
+// Host: the decoding rows of the codec in fp32: for the DCT,
+// M[j][t] = c_j cos(pi / R (t + 1/2) j) in double, rounded to fp32; for the
+// PNG tier, m[j][t] = 1 for j <= t (cumulative sum).
+void make_basis(int codec, int R, int S, Basis* out);
 
 // The same rows in double precision (used by the compression kernels, which
 // take the quantiser's rounding decision in fp64).
 struct BasisF64 {
   double m[kMaxS][kMaxR];
 };
-void make_basis_f64(int R, int S, BasisF64* out);
+// Host: the encoding rows of the codec in fp64 (the DCT rows; for the PNG
+// tier the anchor row and the first differences).
+void make_basis_f64(int codec, int R, int S, BasisF64* out);
 
 // Host: SM count of the current device (cached per device).
 int sm_count();

@@ -39,6 +39,7 @@ struct ViewArgs {
   int64_t out_row0;   // out row of token 0 of block `first`
   int64_t tail_row0;  // out row of tail token 0
   int32_t R, S;
+  int32_t codec;      // FC_CODEC_DCT or FC_CODEC_PNG (decoding rows)
   int32_t rows;       // tokens t < rows of each block are written (<= R)
   int64_t block_items;  // B * H * count
   int64_t tail_items;   // B * H when tail rows are copied, else 0
@@ -321,7 +322,7 @@ int launch_view(const ViewArgs& a, int coeff_dtype, int out_dtype, int64_t D, fc
   if (total == 0) return FC_OK;
   if (total >= (int64_t(1) << 31)) return FC_ERR_UNSUPPORTED;
   Basis basis;
-  make_basis(a.R, a.S, &basis);
+  make_basis(a.codec, a.R, a.S, &basis);
   return dispatch_coeff(coeff_dtype, [&](auto tc) {
     using TC = decltype(tc);
     return dispatch_view(out_dtype, [&](auto to) {
@@ -347,6 +348,7 @@ void fill_archive_side(ViewArgs& a, const fc_archive* arc) {
   a.H = arc->H;
   a.R = arc->R;
   a.S = arc->S;
+  a.codec = arc->codec;
 }
 
 // [lo, hi) byte span of every element a (B, H, extent) tensor can address.

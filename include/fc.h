@@ -66,6 +66,12 @@ enum {
   FC_DECODE_Q_FINAL = 8       /* with OVERLAP: q was final before that work began */
 };
 
+/* Codecs (fc_archive.codec). */
+enum {
+  FC_CODEC_DCT = 0, /* block DCT-II, S lowest frequencies (int8 / bf16 / fp32) */
+  FC_CODEC_PNG = 1  /* lossless PNG tier: anchor + fp32 first differences */
+};
+
 /* Element types. */
 enum {
   FC_DTYPE_F32 = 0,
@@ -84,6 +90,16 @@ enum {
  *   scales  device, (B, H, capacity, S) fp32, contiguous per (b, h); required
  *           when coeff_dtype == FC_DTYPE_I8, must be NULL otherwise.
  *   coeff_dtype  FC_DTYPE_I8 (quantised), FC_DTYPE_BF16 or FC_DTYPE_F32.
+ *   codec        FC_CODEC_DCT: rows C = M X_blk with the DCT-II rows M.
+ *                FC_CODEC_PNG (flashcodec-kv README, "Math", PNG bullet; the
+ *                lossless tier, keep_ratio 1.0): S == R rows per block in
+ *                fp32, row 0 the block's first token (the anchor, converted
+ *                exactly) and row j >= 1 the first difference
+ *                x_j - x_{j-1} rounded once to fp32; decoding is the
+ *                cumulative sum x_t = sum_{j <= t} row_j, and decode attention
+ *                takes the same per-block steps with A[t][j] = 1 for j <= t.
+ *                Every call of this header and of fc_view.h serves both
+ *                codecs; the tensor-core kernel serves the DCT only.
  *   n_blocks     archived blocks per (b, h), 0 <= n_blocks <= capacity; the
  *                library advances it when it archives blocks.
  *   *_stride_b / *_stride_h  element strides of the batch and head axes;
@@ -97,7 +113,7 @@ typedef struct fc_archive {
   int32_t coeff_dtype;
   int32_t R;
   int32_t S;
-  int32_t reserved;
+  int32_t codec;
   int64_t B, H, D;
   int64_t capacity;
   int64_t n_blocks;

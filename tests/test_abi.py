@@ -358,3 +358,23 @@ def test_state_save_restore_validate_on_the_host():
     st = lib.fc_state_save(ctypes.byref(arc), ctypes.byref(tail),
                            ctypes.c_void_p(buf.data_ptr()), n - 1, None)
     assert st == _lib.FC_ERR_INVALID
+
+
+def test_png_codec_descriptors_validate_on_the_host():
+    """FC_CODEC_PNG needs S == R and fp32 rows; an unknown codec is refused;
+    storage counts R fp32 rows per block."""
+    def arc(S, dtype, codec, R=8):
+        a = _arc(B=1, H=2, D=64, R=R, S=S, dtype=dtype, cap=16, nb=5)
+        a.codec = codec
+        return a
+    lib = _lib.load()
+    ok = arc(8, _lib.FC_DTYPE_F32, _lib.FC_CODEC_PNG)
+    assert _lib.fc_storage_bytes(ok) == 1 * 2 * 5 * 8 * 64 * 4
+    for bad in (arc(4, _lib.FC_DTYPE_F32, _lib.FC_CODEC_PNG),
+                arc(8, _lib.FC_DTYPE_BF16, _lib.FC_CODEC_PNG),
+                arc(2, _lib.FC_DTYPE_F32, 7)):
+        assert lib.fc_storage_bytes(ctypes.byref(bad), None) == -1
+    k = ctypes.c_int32(-1)
+    assert lib.fc_decode_kernel(ctypes.byref(ok), ctypes.byref(ok), 4, 0,
+                                ctypes.byref(k)) == _lib.FC_OK
+    assert k.value == _lib.FC_KERNEL_CUDA_CORE
