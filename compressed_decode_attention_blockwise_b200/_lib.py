@@ -53,7 +53,10 @@ EXPORTS = (
     "fc_storage_bytes", "fc_status_string", "fc_decode_step",
     "fc_read_view", "fc_crop", "fc_select_batch", "fc_noalloc_status",
     "fc_decode_kernel", "fc_state_bytes", "fc_state_save", "fc_state_restore",
+    "fc_decode_step_layers",
 )
+
+FC_MAX_LAYERS = 16
 
 
 class FcError(RuntimeError):
@@ -72,6 +75,19 @@ class FcArchive(ctypes.Structure):
         ("capacity", ctypes.c_int64), ("n_blocks", ctypes.c_int64),
         ("coeff_stride_b", ctypes.c_int64), ("coeff_stride_h", ctypes.c_int64),
         ("scale_stride_b", ctypes.c_int64), ("scale_stride_h", ctypes.c_int64),
+    ]
+
+
+class FcLayerStep(ctypes.Structure):
+    """fc_layer_step of include/fc.h (one layer of fc_decode_step_layers)."""
+    _fields_ = [
+        ("q", ctypes.c_void_p), ("q_strides", ctypes.c_int64 * 4),
+        ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p),
+        ("k_strides", ctypes.c_int64 * 4), ("v_strides", ctypes.c_int64 * 4),
+        ("ka", ctypes.c_void_p), ("va", ctypes.c_void_p),
+        ("kt", ctypes.c_void_p), ("vt", ctypes.c_void_p),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("out", ctypes.c_void_p), ("out_strides", ctypes.c_int64 * 4),
     ]
 
 
@@ -133,6 +149,10 @@ def load() -> ctypes.CDLL:
                                           PI64, PA, PA, PT, PT,
                                           ctypes.c_float, I32, I32, P,
                                           ctypes.c_size_t, P, I32, PI64, P]),
+        "fc_decode_step_layers": (ctypes.c_int, [I32,
+                                                 ctypes.POINTER(FcLayerStep),
+                                                 I32, I32, I32, I64,
+                                                 ctypes.c_float, I32, I32, P]),
         "fc_combine": (ctypes.c_int, [P, ctypes.c_size_t, I64, I64, I64, I32,
                                       P, I32, PI64, P]),
         "fc_decode_attention_noalloc": (ctypes.c_int, [P, I32, PI64, I64, PA,
@@ -306,6 +326,38 @@ def fc_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
         int(num_splits), flags, ws_ptr, ws_bytes, _ptr(out),
         dtype_code(out.dtype), _strides4(out), _stream(stream, q))
     _check(st, "fc_decode_step")
+
+
+def fc_decode_step_layers(qs, k_news, v_news, kas, vas, kts, vts, outs,
+                          workspaces, softmax_scale: float = 0.0,
+                          num_splits: int = 0, fuse_combine: bool = True,
+                          stream=None) -> None:
+    """One launch of the fused decode steps of len(qs) independent streams
+    (per-layer tensors and descriptors in matching lists)."""
+    n = len(qs)
+    arr = (FcLayerStep * max(1, n))()
+    for i in range(n):
+        L = arr[i]
+        L.q = qs[i].data_ptr()
+        L.q_strides[:] = list(qs[i].stride())
+        L.k_new, L.v_new = k_news[i].data_ptr(), v_news[i].data_ptr()
+        L.k_strides[:] = list(k_news[i].stride())
+        L.v_strides[:] = list(v_news[i].stride())
+        L.ka = ctypes.addressof(kas[i])
+        L.va = ctypes.addressof(vas[i])
+        L.kt = ctypes.addressof(kts[i])
+        L.vt = ctypes.addressof(vts[i])
+        ws = workspaces[i]
+        L.workspace = None if ws is None else ws.data_ptr()
+        L.workspace_bytes = 0 if ws is None else ws.numel() * ws.element_size()
+        L.out = outs[i].data_ptr()
+        L.out_strides[:] = list(outs[i].stride())
+    st = load().fc_decode_step_layers(
+        n, arr, dtype_code(qs[0].dtype), dtype_code(k_news[0].dtype),
+        dtype_code(outs[0].dtype), qs[0].shape[1], float(softmax_scale),
+        int(num_splits), FC_DECODE_FUSE_COMBINE if fuse_combine else 0,
+        _stream(stream, qs[0]))
+    _check(st, "fc_decode_step_layers")
 
 
 def fc_decode_attention_noalloc(q: torch.Tensor, ka: FcArchive, va: FcArchive,

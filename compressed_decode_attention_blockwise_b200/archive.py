@@ -502,5 +502,30 @@ class CodecKVCache:
         self.v.reset()
 
 
+def decode_step_layers(caches, qs, k_news, v_news, outs=None,
+                       softmax_scale: Optional[float] = None,
+                       out_dtype: torch.dtype = torch.float32):
+    """One decode step (append + attention) of every cache in ``caches`` in
+    one launch (fc_decode_step_layers): cache i appends (k_news[i],
+    v_news[i]) and attends qs[i]. The caches are independent streams of the
+    same shape (the layers of a step whose queries are all known, or the
+    sequences of a serving batch). Returns the outputs."""
+    n = len(caches)
+    for c in caches:
+        if c.k.tail_len + 1 == c.R:
+            c._grow_to(c.k.n_blocks + 1)
+    Hq = qs[0].shape[1]
+    if outs is None:
+        outs = [torch.empty((c.B, Hq, 1, c.D), dtype=out_dtype,
+                            device=qs[0].device) for c in caches]
+    wss = [c.workspace(Hq, c.num_splits(Hq)) for c in caches]
+    _lib.fc_decode_step_layers(
+        qs, k_news, v_news, [c.k.arc for c in caches],
+        [c.v.arc for c in caches], [c.k.tail_desc for c in caches],
+        [c.v.tail_desc for c in caches], outs, wss,
+        softmax_scale=0.0 if softmax_scale is None else float(softmax_scale))
+    return outs
+
+
 def default_scale(D: int) -> float:
     return 1.0 / math.sqrt(D)

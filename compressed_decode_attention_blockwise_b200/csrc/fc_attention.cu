@@ -238,37 +238,36 @@ extern "C" int fc_decode_attention(const void* q, int32_t q_dtype, const int64_t
   return launch_prepared(a, ka, va, flags, stream);
 }
 
-extern "C" int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int64_t Hq,
-                              const void* k_new, const void* v_new, int32_t new_dtype,
-                              const int64_t* k_strides, const int64_t* v_strides, fc_archive* ka,
-                              fc_archive* va, fc_tail* kt, fc_tail* vt, float softmax_scale,
-                              int32_t num_splits, int32_t flags, void* workspace,
-                              size_t workspace_bytes, void* out, int32_t out_dtype,
-                              const int64_t* out_strides, fc_stream stream) {
+namespace fc {
+namespace {
+
+// Argument set-up of one fused decode step (fc_decode_step): *fused tells
+// whether the tensor-core kernel serves it in one launch (then *ap holds the
+// step fields and *complete whether the token completes a block); otherwise
+// the caller issues fc_append_step + fc_decode_attention.
+int prepare_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int64_t Hq, const void* k_new,
+                 const void* v_new, int32_t new_dtype, const int64_t* k_strides, const int64_t* v_strides,
+                 const fc_archive* ka, const fc_archive* va, const fc_tail* kt, const fc_tail* vt,
+                 float softmax_scale, int32_t num_splits, int32_t flags, void* workspace,
+                 size_t workspace_bytes, void* out, int32_t out_dtype, const int64_t* out_strides,
+                 DecodeArgs* ap, bool* fused, bool* complete) {
   if (!k_new || !v_new || !k_strides || !v_strides || !kt || !vt || !kt->data || !vt->data)
     return FC_ERR_INVALID;
   DecodeArgs a;
   int st = prepare_decode(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
                           workspace, workspace_bytes, out, out_dtype, out_strides, true, &a);
   if (st != FC_OK) return st;
-  const bool fused = !(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, a.G) &&
-                     new_dtype == kt->dtype && k_strides[3] == 1 && v_strides[3] == 1 &&
-                     aligned16(k_new) && aligned16(v_new) && k_strides[0] >= 0 && k_strides[1] >= 0 &&
-                     v_strides[0] >= 0 && v_strides[1] >= 0;
-  if (!fused) {
-    // two launches: the append, then the attention over the updated stream
-    st = fc_append_step(k_new, v_new, new_dtype, k_strides, v_strides, ka, va, kt, vt, stream);
-    if (st != FC_OK) return st;
-    return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
-                               workspace, workspace_bytes, out, out_dtype, out_strides, stream);
-  }
+  *fused = !(flags & FC_DECODE_PORTABLE) && decode_tc_eligible(ka, va, a.G) && new_dtype == kt->dtype &&
+           k_strides[3] == 1 && v_strides[3] == 1 && aligned16(k_new) && aligned16(v_new) &&
+           k_strides[0] >= 0 && k_strides[1] >= 0 && v_strides[0] >= 0 && v_strides[1] >= 0;
+  if (!*fused) return FC_OK;
   const int esz = dtype_size(new_dtype);
   if ((k_strides[0] * esz) % 16 || (k_strides[1] * esz) % 16 || (v_strides[0] * esz) % 16 ||
       (v_strides[1] * esz) % 16)
     return FC_ERR_INVALID;
-  const bool complete = kt->len + 1 == ka->R;
-  if (complete && (ka->n_blocks >= ka->capacity || va->n_blocks >= va->capacity)) return FC_ERR_CAPACITY;
-  a.step = complete ? 2 : 1;
+  *complete = kt->len + 1 == ka->R;
+  if (*complete && (ka->n_blocks >= ka->capacity || va->n_blocks >= va->capacity)) return FC_ERR_CAPACITY;
+  a.step = *complete ? 2 : 1;
   a.kn = k_new;
   a.vn = v_new;
   a.kns_b = k_strides[0];
@@ -278,8 +277,12 @@ extern "C" int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_s
   a.kout = out_of(ka);
   a.vout = out_of(va);
   a.new_slot = ka->n_blocks;
-  st = launch_prepared(a, ka, va, flags, stream);
-  if (st != FC_OK) return st;
+  *ap = a;
+  return FC_OK;
+}
+
+// host descriptors after a step: the token joined the tail or completed a block
+void advance_step(fc_archive* ka, fc_archive* va, fc_tail* kt, fc_tail* vt, bool complete) {
   if (complete) {
     ka->n_blocks += 1;
     va->n_blocks += 1;
@@ -289,6 +292,71 @@ extern "C" int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_s
     kt->len += 1;
     vt->len += 1;
   }
+}
+
+}  // namespace
+}  // namespace fc
+
+extern "C" int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int64_t Hq,
+                              const void* k_new, const void* v_new, int32_t new_dtype,
+                              const int64_t* k_strides, const int64_t* v_strides, fc_archive* ka,
+                              fc_archive* va, fc_tail* kt, fc_tail* vt, float softmax_scale,
+                              int32_t num_splits, int32_t flags, void* workspace,
+                              size_t workspace_bytes, void* out, int32_t out_dtype,
+                              const int64_t* out_strides, fc_stream stream) {
+  DecodeArgs a;
+  bool fused = false, complete = false;
+  int st = prepare_step(q, q_dtype, q_strides, Hq, k_new, v_new, new_dtype, k_strides, v_strides, ka, va, kt, vt,
+                        softmax_scale, num_splits, flags, workspace, workspace_bytes, out, out_dtype,
+                        out_strides, &a, &fused, &complete);
+  if (st != FC_OK) return st;
+  if (!fused) {
+    // two launches: the append, then the attention over the updated stream
+    st = fc_append_step(k_new, v_new, new_dtype, k_strides, v_strides, ka, va, kt, vt, stream);
+    if (st != FC_OK) return st;
+    return fc_decode_attention(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
+                               workspace, workspace_bytes, out, out_dtype, out_strides, stream);
+  }
+  st = launch_prepared(a, ka, va, flags, stream);
+  if (st != FC_OK) return st;
+  advance_step(ka, va, kt, vt, complete);
+  return FC_OK;
+}
+
+extern "C" int fc_decode_step_layers(int32_t n_layers, fc_layer_step* layers, int32_t q_dtype,
+                                     int32_t new_dtype, int32_t out_dtype, int64_t Hq, float softmax_scale,
+                                     int32_t num_splits, int32_t flags, fc_stream stream) {
+  if (n_layers < 1 || n_layers > FC_MAX_LAYERS || !layers) return FC_ERR_INVALID;
+  if (flags & (FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL | FC_DECODE_PORTABLE)) return FC_ERR_INVALID;
+  DecodeArgs args[FC_MAX_LAYERS];
+  const fc_archive* kas[FC_MAX_LAYERS];
+  const fc_archive* vas[FC_MAX_LAYERS];
+  bool complete[FC_MAX_LAYERS];
+  for (int i = 0; i < n_layers; ++i) {
+    fc_layer_step& L = layers[i];
+    bool fused = false;
+    const int st = prepare_step(L.q, q_dtype, L.q_strides, Hq, L.k_new, L.v_new, new_dtype, L.k_strides,
+                                L.v_strides, L.ka, L.va, L.kt, L.vt, softmax_scale, num_splits, flags,
+                                L.workspace, L.workspace_bytes, L.out, out_dtype, L.out_strides, &args[i],
+                                &fused, &complete[i]);
+    if (st != FC_OK) return st;
+    if (!fused) return FC_ERR_UNSUPPORTED;
+    if (args[i].G != args[0].G || args[i].S != args[0].S || args[i].R != args[0].R ||
+        args[i].D != args[0].D)
+      return FC_ERR_UNSUPPORTED;
+    for (int j = 0; j < i; ++j)  // one launch writes every layer's streams
+      if (layers[j].ka == L.ka || layers[j].va == L.va || layers[j].kt == L.kt || layers[j].vt == L.vt ||
+          layers[j].workspace == L.workspace)
+        return FC_ERR_INVALID;
+    kas[i] = L.ka;
+    vas[i] = L.va;
+  }
+  Basis basis;
+  make_basis(FC_CODEC_DCT, args[0].R, args[0].S, &basis);
+  const int st = launch_decode_tc_layers(n_layers, args, kas, vas, basis, stream);
+  if (st != FC_OK) return st;
+  for (int i = 0; i < n_layers; ++i)
+    advance_step(layers[i].ka, layers[i].va, layers[i].kt, layers[i].vt, complete[i]);
   return FC_OK;
 }
 

@@ -509,6 +509,9 @@ bool decode_tc_eligible(const fc_archive* ka, const fc_archive* va, int G);
 int tc_tiles_per_head(int64_t nb, int S);
 int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive* va, const Basis& basis,
                      cudaStream_t stream);
+// The problems d[0..n) (same G, S, R; each tensor-core eligible) in one launch.
+int launch_decode_tc_layers(int n, const DecodeArgs* d, const fc_archive* const* ka, const fc_archive* const* va,
+                            const Basis& basis, cudaStream_t stream);
 
 // Combine kernel for fc_combine: one CTA per (b, q head).
 struct CombineArgs {

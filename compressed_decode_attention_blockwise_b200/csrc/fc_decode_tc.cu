@@ -116,6 +116,18 @@ struct TcArgs {
   int tiles_per_head;
 };
 
+// The problems of one launch (the layers of fc_decode_step_layers, or the
+// one problem of a single call): CTA x serves problem p for
+// cta_end[p - 1] <= x < cta_end[p]. Passed as a __grid_constant__ parameter,
+// so the tensor maps are addressed in parameter space.
+template <int NL>
+struct TcBatch {
+  CUtensorMap maps[NL][4];  // K codes, V codes, K scales, V scales
+  TcArgs prob[NL];
+  int cta_end[NL];
+  int n;
+};
+
 // The DCT basis rows the kernel needs, sized for its (S, R): fp32 for the
 // attention arithmetic, fp64 for encoding a block in the fused decode step
 // (the same values as the codec's). A small parameter block keeps launches
@@ -323,11 +335,20 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&r)[NP]) 
   }
 }
 
-template <int G, int S, int TPT>
+template <int G, int S, int TPT, int NL>
 __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
-    decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
-                     const TcArgs ta, const TcBasis<S, S * TPT> basis) {
+    decode_tc_kernel(const __grid_constant__ TcBatch<NL> batch, const TcBasis<S, S * TPT> basis) {
+  // this CTA's problem
+  int prob = 0;
+  if constexpr (NL > 1) {
+    while (prob + 1 < batch.n && int(blockIdx.x) >= batch.cta_end[prob]) ++prob;
+  }
+  const int bx_local = int(blockIdx.x) - (prob > 0 ? batch.cta_end[prob - 1] : 0);
+  const TcArgs& ta = batch.prob[prob];
+  const CUtensorMap& tm_k = batch.maps[prob][0];
+  const CUtensorMap& tm_v = batch.maps[prob][1];
+  const CUtensorMap& tm_ks = batch.maps[prob][2];
+  const CUtensorMap& tm_vs = batch.maps[prob][3];
   using C = Cfg<G, S, TPT>;
   constexpr int R = C::R, NP = C::NP, NI = C::NI, NKS = C::NKS, NVS = C::NVS, XP = C::XP;
   constexpr int NG = C::NG;
@@ -356,7 +377,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   // bal_q + 1 chunks, the others bal_q; a unit's tiles split evenly
   int unit, c, ns_u;
   {
-    const int bx = blockIdx.x, hi = a.bal_q + 1;
+    const int bx = bx_local, hi = a.bal_q + 1;
     if (bx < a.bal_rem * hi) {
       unit = bx / hi;
       c = bx - unit * hi;
@@ -1051,8 +1072,11 @@ bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G, int S, int TPT>
-int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CUtensorMap* maps,
+// CTAs of one problem: every kv head takes ns chunks
+int problem_ctas(const TcArgs& ta) { return ta.d.B * ta.d.Hk * ta.d.ns; }
+
+template <int G, int S, int TPT, int NL>
+int launch(const TcBatch<NL>& batch, const Basis& full, const BasisF64& full64, bool overlap,
            cudaStream_t stream) {
   TcBasis<S, S * TPT> basis;
   for (int j = 0; j < S; ++j)
@@ -1062,12 +1086,11 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
     }
   using C = Cfg<G, S, TPT>;
   const size_t smem = C::alloc;
-  auto kern = decode_tc_kernel<G, S, TPT>;
+  auto kern = decode_tc_kernel<G, S, TPT, NL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
     return FC_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  const unsigned units = unsigned(ta.d.B) * unsigned(ta.d.Hk);
-  cfg.gridDim = dim3(unsigned(ta.d.bal_rem) + units * unsigned(ta.d.bal_q));
+  cfg.gridDim = dim3(unsigned(batch.cta_end[batch.n - 1]));
   cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
@@ -1075,8 +1098,45 @@ int launch(const TcArgs& ta, const Basis& full, const BasisF64& full64, const CU
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = ta.d.overlap ? 1 : 0;
-  return cuda_status(cudaLaunchKernelEx(&cfg, kern, maps[0], maps[1], maps[2], maps[3], ta, basis));
+  cfg.numAttrs = overlap ? 1 : 0;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kern, batch, basis));
+}
+
+// Fills problem slot i of a batch: the tile geometry and the four tensor maps.
+template <int NL>
+bool fill_problem(TcBatch<NL>* batch, int i, const DecodeArgs& d, const fc_archive* ka,
+                  const fc_archive* va) {
+  TcArgs& ta = batch->prob[i];
+  ta.d = d;
+  ta.tiles_per_head = tc_tiles_per_head(d.nb, d.S);
+  ta.d.bal_q = d.ns;  // every kv head takes ns chunks
+  ta.d.bal_rem = 0;
+  const int64_t rows = d.nb * d.S;
+  if (!make_code_map(&batch->maps[i][0], ka, rows) || !make_code_map(&batch->maps[i][1], va, rows) ||
+      !make_scale_map(&batch->maps[i][2], ka, rows) || !make_scale_map(&batch->maps[i][3], va, rows))
+    return false;
+  batch->cta_end[i] = (i > 0 ? batch->cta_end[i - 1] : 0) + problem_ctas(ta);
+  batch->n = i + 1;
+  return true;
+}
+
+template <int NL>
+int dispatch(const TcBatch<NL>& batch, int G, int S, int R, const Basis& basis, const BasisF64& basis64,
+             bool overlap, cudaStream_t stream) {
+  const int key = G * 10000 + S * 100 + R / S;
+  switch (key) {
+#define FC_TC_CASE(G, S, T) \
+  case G * 10000 + S * 100 + T: return launch<G, S, T, NL>(batch, basis, basis64, overlap, stream);
+    FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
+    FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
+    FC_TC_CASE(1, 2, 4) FC_TC_CASE(2, 2, 4) FC_TC_CASE(4, 2, 4) FC_TC_CASE(8, 2, 4)
+    FC_TC_CASE(1, 2, 8) FC_TC_CASE(2, 2, 8) FC_TC_CASE(4, 2, 8)
+    FC_TC_CASE(1, 4, 2) FC_TC_CASE(2, 4, 2) FC_TC_CASE(4, 4, 2) FC_TC_CASE(8, 4, 2)
+    FC_TC_CASE(1, 4, 4) FC_TC_CASE(2, 4, 4) FC_TC_CASE(4, 4, 4) FC_TC_CASE(8, 4, 4)
+    FC_TC_CASE(1, 8, 2) FC_TC_CASE(2, 8, 2) FC_TC_CASE(4, 8, 2) FC_TC_CASE(8, 8, 2)
+#undef FC_TC_CASE
+    default: return FC_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace tc
@@ -1104,32 +1164,21 @@ int launch_decode_tc(const DecodeArgs& d, const fc_archive* ka, const fc_archive
                      cudaStream_t stream) {
   BasisF64 basis64;
   make_basis_f64(FC_CODEC_DCT, d.R, d.S, &basis64);
-  tc::TcArgs ta;
-  ta.d = d;
-  ta.tiles_per_head = tc_tiles_per_head(d.nb, d.S);
-  const int64_t units = int64_t(d.B) * d.Hk;
-  (void)units;
-  ta.d.bal_q = d.ns;  // every kv head takes ns chunks
-  ta.d.bal_rem = 0;
-  CUtensorMap maps[4];
-  const int64_t rows = d.nb * d.S;
-  if (!tc::make_code_map(&maps[0], ka, rows) || !tc::make_code_map(&maps[1], va, rows) ||
-      !tc::make_scale_map(&maps[2], ka, rows) || !tc::make_scale_map(&maps[3], va, rows))
-    return FC_ERR_CUDA;
-  const int key = d.G * 10000 + d.S * 100 + d.R / d.S;
-  switch (key) {
-#define FC_TC_CASE(G, S, T) \
-  case G * 10000 + S * 100 + T: return tc::launch<G, S, T>(ta, basis, basis64, maps, stream);
-    FC_TC_CASE(1, 1, 4) FC_TC_CASE(2, 1, 4) FC_TC_CASE(4, 1, 4) FC_TC_CASE(8, 1, 4)
-    FC_TC_CASE(1, 1, 8) FC_TC_CASE(2, 1, 8) FC_TC_CASE(4, 1, 8)
-    FC_TC_CASE(1, 2, 4) FC_TC_CASE(2, 2, 4) FC_TC_CASE(4, 2, 4) FC_TC_CASE(8, 2, 4)
-    FC_TC_CASE(1, 2, 8) FC_TC_CASE(2, 2, 8) FC_TC_CASE(4, 2, 8)
-    FC_TC_CASE(1, 4, 2) FC_TC_CASE(2, 4, 2) FC_TC_CASE(4, 4, 2) FC_TC_CASE(8, 4, 2)
-    FC_TC_CASE(1, 4, 4) FC_TC_CASE(2, 4, 4) FC_TC_CASE(4, 4, 4) FC_TC_CASE(8, 4, 4)
-    FC_TC_CASE(1, 8, 2) FC_TC_CASE(2, 8, 2) FC_TC_CASE(4, 8, 2) FC_TC_CASE(8, 8, 2)
-#undef FC_TC_CASE
-    default: return FC_ERR_UNSUPPORTED;
-  }
+  tc::TcBatch<1> batch;
+  if (!tc::fill_problem(&batch, 0, d, ka, va)) return FC_ERR_CUDA;
+  return tc::dispatch(batch, d.G, d.S, d.R, basis, basis64, d.overlap != 0, stream);
+}
+
+int launch_decode_tc_layers(int n, const DecodeArgs* d, const fc_archive* const* ka, const fc_archive* const* va,
+                            const Basis& basis, cudaStream_t stream) {
+  if (n < 1 || n > FC_MAX_LAYERS) return FC_ERR_INVALID;
+  BasisF64 basis64;
+  make_basis_f64(FC_CODEC_DCT, d[0].R, d[0].S, &basis64);
+  static_assert(FC_MAX_LAYERS == 16, "batch capacity");
+  tc::TcBatch<FC_MAX_LAYERS> batch;
+  for (int i = 0; i < n; ++i)
+    if (!tc::fill_problem(&batch, i, d[i], ka[i], va[i])) return FC_ERR_CUDA;
+  return tc::dispatch(batch, d[0].G, d[0].S, d[0].R, basis, basis64, false, stream);
 }
 
 }  // namespace fc

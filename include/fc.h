@@ -315,6 +315,57 @@ int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int
                    const int64_t* out_strides, fc_stream stream);
 
 /*
+ * fc_decode_step_layers -- the fused decode steps of n_layers independent
+ * streams in ONE kernel launch: layer i does fc_decode_step(layers[i].q,
+ * layers[i].k_new, layers[i].v_new, ...) with the results of that call
+ * (bitwise: every CTA runs the single call's code on its layer). The launch's
+ * CTAs are every layer's (kv head, chunk) pieces; the hardware starts the
+ * next layer's pieces as SMs free up, so one launch's start-up and one
+ * drain are paid instead of n_layers (flashcodec-kv README,
+ * "Materialization-free decode attention": the split/combine launches are
+ * the remaining end-to-end gap). Every query and new token must be final
+ * when the launch starts (the layers of a step whose queries are known, or
+ * the sequences of a serving batch with their own caches); a model whose
+ * layer l + 1 query depends on layer l's output calls fc_decode_step per
+ * layer.
+ *   n_layers   1 .. FC_MAX_LAYERS.
+ *   layers     per layer: q (B, Hq, 1, D) and its strides; k_new / v_new
+ *              (B, H, 1, D) and strides; the K and V archives and tails
+ *              (updated on success as fc_decode_step does); a workspace of
+ *              fc_decode_workspace_bytes for its split; out (B, Hq, 1, D) and
+ *              strides. No two layers share an archive, tail or workspace.
+ *   q_dtype, new_dtype, out_dtype, Hq, softmax_scale, num_splits: as in
+ *              fc_decode_step, shared by all layers.
+ *   flags      FC_DECODE_FUSE_COMBINE or 0 (the overlap flags and
+ *              FC_DECODE_PORTABLE are FC_ERR_INVALID).
+ * Every layer must be a tensor-core fused step (int8 K and V, D = 128, the
+ * sizes fc_decode_attention lists for that kernel) with the same G, S and
+ * R, else FC_ERR_UNSUPPORTED; FC_ERR_CAPACITY for any layer leaves every
+ * layer unchanged. One kernel launch.
+ */
+#define FC_MAX_LAYERS 16
+typedef struct fc_layer_step {
+  const void* q;
+  int64_t q_strides[4];
+  const void* k_new;
+  const void* v_new;
+  int64_t k_strides[4];
+  int64_t v_strides[4];
+  fc_archive* ka;
+  fc_archive* va;
+  fc_tail* kt;
+  fc_tail* vt;
+  void* workspace;
+  size_t workspace_bytes;
+  void* out;
+  int64_t out_strides[4];
+} fc_layer_step;
+int fc_decode_step_layers(int32_t n_layers, fc_layer_step* layers, int32_t q_dtype,
+                          int32_t new_dtype, int32_t out_dtype, int64_t Hq,
+                          float softmax_scale, int32_t num_splits, int32_t flags,
+                          fc_stream stream);
+
+/*
  * fc_combine -- merge split-K partials left in `workspace` by
  * fc_decode_attention without FC_DECODE_FUSE_COMBINE (flashcodec/triton_attention.py,
  * combine kernel): M = max_c m_c, L = sum_c l_c e^(m_c - M),

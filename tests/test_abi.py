@@ -378,3 +378,46 @@ def test_png_codec_descriptors_validate_on_the_host():
     assert lib.fc_decode_kernel(ctypes.byref(ok), ctypes.byref(ok), 4, 0,
                                 ctypes.byref(k)) == _lib.FC_OK
     assert k.value == _lib.FC_KERNEL_CUDA_CORE
+
+
+def test_decode_step_layers_validate_on_the_host():
+    """fc_decode_step_layers refuses, before any launch: a layer count out of
+    range, the overlap flags, layers of different (S, R), and two layers that
+    share a stream."""
+    lib = _lib.load()
+
+    def layer(S=2, R=8, arcs=None):
+        ka = arcs[0] if arcs else _arc(B=1, H=2, D=128, R=R, S=S, cap=32,
+                                       nb=10)
+        va = arcs[1] if arcs else _arc(B=1, H=2, D=128, R=R, S=S, cap=32,
+                                       nb=10)
+        kt, vt = _tail(ka, 3), _tail(va, 3)
+        L = _lib.FcLayerStep()
+        L.q = FAKE
+        L.q_strides[:] = [2 * 4 * 128, 4 * 128, 128, 1]
+        L.k_new = L.v_new = FAKE
+        L.k_strides[:] = [2 * 128, 128, 128, 1]
+        L.v_strides[:] = [2 * 128, 128, 128, 1]
+        L.ka, L.va = ctypes.addressof(ka), ctypes.addressof(va)
+        L.kt, L.vt = ctypes.addressof(kt), ctypes.addressof(vt)
+        L.workspace = 0x100000
+        L.workspace_bytes = 1 << 20
+        L.out = FAKE
+        L.out_strides[:] = [2 * 4 * 128, 4 * 128, 128, 1]
+        return L, (ka, va, kt, vt)
+
+    def call(layers, flags=_lib.FC_DECODE_FUSE_COMBINE, n=None):
+        arr = (_lib.FcLayerStep * max(1, len(layers)))(*[x[0] for x in layers])
+        return lib.fc_decode_step_layers(
+            len(layers) if n is None else n, arr, _lib.FC_DTYPE_BF16,
+            _lib.FC_DTYPE_BF16, _lib.FC_DTYPE_F32, 4, 0.0, 0, flags, None)
+
+    a, b = layer(), layer()
+    assert call([a, b], n=0) == _lib.FC_ERR_INVALID
+    assert call([a, b], n=_lib.FC_MAX_LAYERS + 1) == _lib.FC_ERR_INVALID
+    assert call([a, b], flags=_lib.FC_DECODE_FUSE_COMBINE |
+                _lib.FC_DECODE_OVERLAP) == _lib.FC_ERR_INVALID
+    c = layer(S=4, R=16)
+    assert call([a, c]) == _lib.FC_ERR_UNSUPPORTED
+    shared = layer(arcs=a[1][:2])
+    assert call([a, shared]) == _lib.FC_ERR_INVALID
