@@ -90,15 +90,16 @@ def test_layers_in_one_launch_match_per_layer_steps_and_oracle(name, tails,
 
 
 def test_layers_reject_a_capacity_shortfall_without_touching_any_layer():
-    w = synth.WORKLOADS["gqa"].replace(B=1, T=8 * 16 - 1, seed=77)
+    w = synth.WORKLOADS["gqa"].replace(B=1, T=8 * 16 + 7, seed=77, steps=1)
     data = synth.generate(w, q_steps=1)
     k, v = data["k"].to(DEV), data["v"].to(DEV)
     caches = []
-    for _ in range(2):
+    for T in (8 * 15 + 2, w.T):
         c = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV, capacity=16)
-        c.prefill(k[:, :, :w.T], v[:, :, :w.T])
+        c.prefill(k[:, :, :T], v[:, :, :T])
         caches.append(c)
-    # layer 1 completes block 16 in a 16-block archive
+    # layer 1 would complete a 17th block in its 16-block archive
+    assert caches[1].k.n_blocks == caches[1].k.capacity == 16
     state = [(c.k.n_blocks, c.k.tail_len) for c in caches]
     q = data["q"][0].to(DEV)
     tok = (k[:, :, w.T:w.T + 1], v[:, :, w.T:w.T + 1])
