@@ -288,6 +288,72 @@ def bench_workload(name, peak, W, world, dev, l2, budget_s=0.25):
     return entry
 
 
+def bench_layers(w, kd, vd, q_pool, dev, W, world, n_layers=8,
+                 n_steps=16):
+    """Decode steps of n_layers independent layer caches of the workload:
+    one fc_decode_step_layers launch per step against n_layers separate
+    fc_decode_step launches (plain, and with the overlap flags). CUDA graphs
+    of n_steps steps; microseconds per layer-step."""
+    from compressed_decode_attention_blockwise_b200 import (
+        CodecKVCache, decode_step_layers)
+    tok_dt = synth.torch_dtype(w.in_dtype)
+    esz = torch.tensor([], dtype=tok_dt).element_size()
+    need = (w.T + n_steps) // w.R + 1
+
+    def make():
+        cs = []
+        for _ in range(n_layers):
+            c = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, w.k_coeff, w.v_coeff,
+                             token_dtype=tok_dt, device=dev, capacity=need)
+            c.prefill(kd[:, :, :w.T], vd[:, :, :w.T])
+            cs.append(c)
+        return cs
+
+    outs = [torch.empty((w.B, w.Hq, 1, w.D), dtype=torch.float32,
+                        device=dev) for _ in range(n_layers)]
+    ev0, ev1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    res = {"layers": n_layers, "steps": n_steps}
+    modes = {"one_launch": None, "separate": (False, False),
+             "separate_overlap_q_final": (True, True)}
+    for name, flags in modes.items():
+        caches = make()
+        for c in caches:
+            c.workspace(w.Hq, c.num_splits(w.Hq))
+        torch.cuda.synchronize()
+        step_bytes = []
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for s in range(n_steps):
+                t = w.T + s
+                q = q_pool[s % len(q_pool)]
+                kn, vn = kd[:, :, t:t + 1], vd[:, :, t:t + 1]
+                if flags is None:
+                    decode_step_layers(caches, [q] * n_layers,
+                                       [kn] * n_layers, [vn] * n_layers,
+                                       outs=outs)
+                else:
+                    for l, c in enumerate(caches):
+                        c.step(q, kn, vn, out=outs[l], overlap=flags[0],
+                               q_final=flags[1])
+                step_bytes.append(sum(attention_bytes(c, w.Hq, esz, 4)
+                                      for c in caches))
+        for _ in range(max(W, 3)):
+            g.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        ev0.record()
+        g.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        t_rep = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, world)
+        per = t_rep / (n_steps * n_layers)
+        res[name] = {"us_per_layer": round(per * 1e6, 3),
+                     "GB_per_s": round(sum(step_bytes) / t_rep / 1e9, 2)}
+        del g, caches
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_fc(args, world, rank, local):
     from compressed_decode_attention_blockwise_b200 import CodecKVCache, _lib
 
@@ -546,6 +612,17 @@ def run_fc(args, world, rank, local):
         "gpu_launches": K,
         "clocks": clk.summary(),
     }
+    if args.layers > 0:
+        lay = bench_layers(w, kd, vd, q_pool, dev, W, world,
+                           n_layers=args.layers)
+        lay["peak"] = peak
+        for m in ("one_launch", "separate", "separate_overlap_q_final"):
+            lay[m]["frac"] = round(lay[m]["GB_per_s"] / peak, 4)
+        lay["note"] = ("decode steps (append + attention) of %d independent "
+                       "layer caches of this workload: one "
+                       "fc_decode_step_layers launch per step against one "
+                       "fc_decode_step launch per layer" % args.layers)
+        res["layers"] = lay
     if args.workloads:
         wl = {}
         for name in args.workloads.split(","):
@@ -703,6 +780,8 @@ def main(argv=None):
                     help="archive copies visited round-robin (0 = enough to "
                          "exceed twice the L2)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=8,
+                    help="layer caches of the multi-layer leg (0 = skip)")
     ap.add_argument("--workloads", default="tiny,gqa,large,stream",
                     help="comma-separated further workloads whose decode "
                          "attention is timed at full size ('' = none)")
