@@ -53,7 +53,8 @@ EXPORTS = (
     "fc_storage_bytes", "fc_status_string", "fc_decode_step",
     "fc_read_view", "fc_crop", "fc_select_batch", "fc_noalloc_status",
     "fc_decode_kernel", "fc_state_bytes", "fc_state_save", "fc_state_restore",
-    "fc_decode_step_layers",
+    "fc_decode_step_layers", "fc_decode_step_staging_bytes",
+    "fc_decode_step_host",
 )
 
 FC_MAX_LAYERS = 16
@@ -149,6 +150,12 @@ def load() -> ctypes.CDLL:
                                           PI64, PA, PA, PT, PT,
                                           ctypes.c_float, I32, I32, P,
                                           ctypes.c_size_t, P, I32, PI64, P]),
+        "fc_decode_step_staging_bytes": (ctypes.c_size_t, [I64, I64, I64, I64,
+                                                            I32, I32]),
+        "fc_decode_step_host": (ctypes.c_int, [P, P, P, ctypes.c_size_t, I32,
+                                               I32, I64, PA, PA, PT, PT,
+                                               ctypes.c_float, I32, I32, P,
+                                               ctypes.c_size_t, P]),
         "fc_decode_step_layers": (ctypes.c_int, [I32,
                                                  ctypes.POINTER(FcLayerStep),
                                                  I32, I32, I32, I64,
@@ -326,6 +333,51 @@ def fc_decode_step(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
         int(num_splits), flags, ws_ptr, ws_bytes, _ptr(out),
         dtype_code(out.dtype), _strides4(out), _stream(stream, q))
     _check(st, "fc_decode_step")
+
+
+class HostStep:
+    """fc_decode_step_host with its arguments marshalled once: calling it
+    runs one step from the host block ``in_host`` ([k_new | v_new | q]) to
+    ``out_host`` (both CPU tensors; pinned for asynchronous copies). The
+    archive and tail descriptors are passed by reference, so the library's
+    updates carry over from call to call."""
+
+    def __init__(self, cache, Hq: int, in_host: torch.Tensor,
+                 out_host: torch.Tensor, staging: torch.Tensor,
+                 workspace: torch.Tensor, softmax_scale: float = 0.0,
+                 num_splits: int = 0, fuse_combine: bool = True,
+                 overlap: bool = False, q_final: bool = False, stream=None):
+        flags = (FC_DECODE_FUSE_COMBINE if fuse_combine else 0) | \
+            (FC_DECODE_OVERLAP if overlap else 0) | \
+            (FC_DECODE_Q_FINAL if q_final else 0)
+        self._fn = load().fc_decode_step_host
+        self._args = (
+            ctypes.c_void_p(in_host.data_ptr()),
+            ctypes.c_void_p(out_host.data_ptr()),
+            ctypes.c_void_p(staging.data_ptr()),
+            ctypes.c_size_t(staging.numel() * staging.element_size()),
+            ctypes.c_int32(dtype_code(in_host.dtype)),
+            ctypes.c_int32(dtype_code(out_host.dtype)), ctypes.c_int64(Hq),
+            ctypes.byref(cache.k.arc), ctypes.byref(cache.v.arc),
+            ctypes.byref(cache.k.tail_desc), ctypes.byref(cache.v.tail_desc),
+            ctypes.c_float(softmax_scale), ctypes.c_int32(num_splits),
+            ctypes.c_int32(flags), ctypes.c_void_p(workspace.data_ptr()),
+            ctypes.c_size_t(workspace.numel() * workspace.element_size()),
+            _stream(stream, staging))
+        self._keep = (in_host, out_host, staging, workspace)
+
+    def __call__(self) -> None:
+        st = self._fn(*self._args)
+        if st != FC_OK:
+            raise FcError(st, "fc_decode_step_host")
+
+
+def fc_decode_step_staging_bytes(B: int, H: int, Hq: int, D: int,
+                                 io_dtype: torch.dtype,
+                                 out_dtype: torch.dtype) -> int:
+    return int(load().fc_decode_step_staging_bytes(
+        int(B), int(H), int(Hq), int(D), dtype_code(io_dtype),
+        dtype_code(out_dtype)))
 
 
 def fc_decode_step_layers(qs, k_news, v_news, kas, vas, kts, vts, outs,

@@ -323,6 +323,74 @@ extern "C" int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_s
   return FC_OK;
 }
 
+namespace fc {
+namespace {
+
+struct StagingLayout {
+  size_t k, v, q, out, total;
+};
+
+StagingLayout staging_layout(int64_t B, int64_t H, int64_t Hq, int64_t D, int io_dtype, int out_dtype) {
+  StagingLayout s;
+  const size_t tok = size_t(B) * size_t(H) * size_t(D) * size_t(dtype_size(io_dtype));
+  const size_t qb = size_t(B) * size_t(Hq) * size_t(D) * size_t(dtype_size(io_dtype));
+  s.k = 0;
+  s.v = pad256(tok);
+  s.q = s.v + pad256(tok);
+  s.out = s.q + pad256(qb);
+  s.total = s.out + pad256(size_t(B) * size_t(Hq) * size_t(D) * size_t(dtype_size(out_dtype)));
+  return s;
+}
+
+}  // namespace
+}  // namespace fc
+
+extern "C" size_t fc_decode_step_staging_bytes(int64_t B, int64_t H, int64_t Hq, int64_t D, int32_t io_dtype,
+                                               int32_t out_dtype) {
+  if (B < 1 || H < 1 || Hq < 1 || D < 1) return 0;
+  if ((io_dtype != FC_DTYPE_BF16 && io_dtype != FC_DTYPE_F32) ||
+      (out_dtype != FC_DTYPE_BF16 && out_dtype != FC_DTYPE_F32))
+    return 0;
+  return staging_layout(B, H, Hq, D, io_dtype, out_dtype).total;
+}
+
+extern "C" int fc_decode_step_host(const void* in_host, void* out_host, void* staging, size_t staging_bytes,
+                                   int32_t io_dtype, int32_t out_dtype, int64_t Hq, fc_archive* ka,
+                                   fc_archive* va, fc_tail* kt, fc_tail* vt, float softmax_scale,
+                                   int32_t num_splits, int32_t flags, void* workspace, size_t workspace_bytes,
+                                   fc_stream stream) {
+  if (!in_host || !out_host || !staging || (reinterpret_cast<uintptr_t>(staging) & 255u)) return FC_ERR_INVALID;
+  int st = check_archive(ka);
+  if (st != FC_OK) return st;
+  const size_t need = fc_decode_step_staging_bytes(ka->B, ka->H, Hq, ka->D, io_dtype, out_dtype);
+  if (need == 0 || staging_bytes < need) return FC_ERR_INVALID;
+  const StagingLayout L = staging_layout(ka->B, ka->H, Hq, ka->D, io_dtype, out_dtype);
+  uint8_t* sg = static_cast<uint8_t*>(staging);
+  const size_t esz = size_t(dtype_size(io_dtype));
+  const size_t tok = size_t(ka->B * ka->H * ka->D) * esz;
+  const size_t qb = size_t(ka->B * Hq * ka->D) * esz;
+  const int64_t tok_s[4] = {ka->H * ka->D, ka->D, ka->D, 1};
+  const int64_t q_s[4] = {Hq * ka->D, ka->D, ka->D, 1};
+  // the host block is [k_new | v_new | q], each contiguous (B, heads, 1, D);
+  // one copy when the staging offsets are contiguous too, else three
+  const uint8_t* in = static_cast<const uint8_t*>(in_host);
+  cudaError_t e = cudaSuccess;
+  if (L.v == tok && L.q == 2 * tok) {
+    e = cudaMemcpyAsync(sg, in, 2 * tok + qb, cudaMemcpyHostToDevice, stream);
+  } else {
+    e = cudaMemcpyAsync(sg + L.k, in, tok, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sg + L.v, in + tok, tok, cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(sg + L.q, in + 2 * tok, qb, cudaMemcpyHostToDevice, stream);
+  }
+  if (e != cudaSuccess) return FC_ERR_CUDA;
+  st = fc_decode_step(sg + L.q, io_dtype, q_s, Hq, sg + L.k, sg + L.v, io_dtype, tok_s, tok_s, ka, va, kt, vt,
+                      softmax_scale, num_splits, flags, workspace, workspace_bytes, sg + L.out, out_dtype, q_s,
+                      stream);
+  if (st != FC_OK) return st;
+  const size_t ob = size_t(ka->B * Hq * ka->D) * size_t(dtype_size(out_dtype));
+  return cuda_status(cudaMemcpyAsync(out_host, sg + L.out, ob, cudaMemcpyDeviceToHost, stream));
+}
+
 extern "C" int fc_decode_step_layers(int32_t n_layers, fc_layer_step* layers, int32_t q_dtype,
                                      int32_t new_dtype, int32_t out_dtype, int64_t Hq, float softmax_scale,
                                      int32_t num_splits, int32_t flags, fc_stream stream) {

@@ -315,6 +315,31 @@ int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int
                    const int64_t* out_strides, fc_stream stream);
 
 /*
+ * fc_decode_step_host -- fc_decode_step fed from and returning to HOST
+ * memory, for a serving loop whose tokens and queries arrive on the host:
+ * one host-to-device copy of the step's inputs into `staging`, the fused
+ * step, one device-to-host copy of the output, all on `stream` (pinned host
+ * memory makes the copies asynchronous; the output is complete once
+ * `stream` reaches the last copy).
+ *   in_host    host, the contiguous block [k_new | v_new | q]: k_new and
+ *              v_new (B, H, 1, D), q (B, Hq, 1, D), each contiguous, of
+ *              io_dtype (FC_DTYPE_BF16 or FC_DTYPE_F32, the tails' dtype).
+ *   out_host   host, (B, Hq, 1, D) contiguous of out_dtype.
+ *   staging    device, >= fc_decode_step_staging_bytes(...), 256-byte
+ *              aligned: the inputs' and the output's device copies.
+ *   other arguments as in fc_decode_step (the archives and tails are
+ *              updated in the same way).
+ */
+size_t fc_decode_step_staging_bytes(int64_t B, int64_t H, int64_t Hq, int64_t D,
+                                    int32_t io_dtype, int32_t out_dtype);
+int fc_decode_step_host(const void* in_host, void* out_host, void* staging,
+                        size_t staging_bytes, int32_t io_dtype, int32_t out_dtype,
+                        int64_t Hq, fc_archive* ka, fc_archive* va, fc_tail* kt,
+                        fc_tail* vt, float softmax_scale, int32_t num_splits,
+                        int32_t flags, void* workspace, size_t workspace_bytes,
+                        fc_stream stream);
+
+/*
  * fc_decode_step_layers -- the fused decode steps of n_layers independent
  * streams in ONE kernel launch: layer i does fc_decode_step(layers[i].q,
  * layers[i].k_new, layers[i].v_new, ...) with the results of that call

@@ -222,3 +222,34 @@ def _dequant(stream, b, h):
     c = stream.coeffs[b:b + 1, h:h + 1, :stream.n_blocks].cpu().numpy()
     sc = stream.scales[b:b + 1, h:h + 1, :stream.n_blocks].cpu().numpy()
     return oracle.dequantize(c, sc)
+
+
+def test_host_buffer_step_equals_device_step():
+    """fc_decode_step_host (inputs from one pinned host block, output to host
+    memory) gives the archive, tail and output of fc_decode_step on device
+    copies of the same inputs, across a block completion."""
+    w = synth.Workload("hstep", B=2, Hq=8, Hk=2, D=128, T=8 * 50 + 5, R=8,
+                       S=2, seed=17, steps=6)
+    data = synth.generate(w, q_steps=w.steps)
+    dev_cache, host_cache = _twin_caches(w, data)
+    for c in (dev_cache, host_cache):
+        c._grow_to((w.T + w.steps) // w.R + 1)
+    nk, nq = w.B * w.Hk * w.D, w.B * w.Hq * w.D
+    staging = torch.empty(_lib.fc_decode_step_staging_bytes(
+        w.B, w.Hk, w.Hq, w.D, torch.bfloat16, torch.float32),
+        dtype=torch.uint8, device=DEV)
+    ws = host_cache.workspace(w.Hq, host_cache.num_splits(w.Hq))
+    for s in range(w.steps):
+        t = w.T + s
+        blk = torch.empty(2 * nk + nq, dtype=torch.bfloat16, pin_memory=True)
+        blk[:nk] = data["k"][:, :, t].reshape(-1)
+        blk[nk:2 * nk] = data["v"][:, :, t].reshape(-1)
+        blk[2 * nk:] = data["q"][s].reshape(-1)
+        out_h = torch.empty((w.B, w.Hq, 1, w.D), pin_memory=True)
+        _lib.HostStep(host_cache, w.Hq, blk, out_h, staging, ws)()
+        ref = dev_cache.step(data["q"][s].to(DEV),
+                             data["k"][:, :, t:t + 1].to(DEV),
+                             data["v"][:, :, t:t + 1].to(DEV))
+        torch.cuda.synchronize()
+        _same_stream(dev_cache, host_cache)
+        assert torch.equal(out_h, ref.cpu())
