@@ -1043,7 +1043,46 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // int8 codes of one archive as a 4-d tensor {D, live rows, H, B}, 128 x 128
 // boxes with 128-byte swizzle
-bool make_code_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
+// Encoded tensor maps of recent archives, keyed by everything the encoding
+// reads, so that a decode loop encodes each map once per archived block
+// instead of once per launch (a small round-robin table, shared by host
+// threads under a mutex).
+struct MapKey {
+  const void* base;
+  int64_t rows, H, B, sh, sb, D;
+  int kind;  // 2 S (codes) or 2 S + 1 (scales)
+  bool operator==(const MapKey& o) const {
+    return base == o.base && rows == o.rows && H == o.H && B == o.B && sh == o.sh && sb == o.sb &&
+           D == o.D && kind == o.kind;
+  }
+};
+
+template <typename Encode>
+bool cached_map(CUtensorMap* m, const MapKey& key, Encode&& encode) {
+  constexpr int kSlots = 32;
+  static std::mutex mu;
+  static MapKey keys[kSlots];
+  static CUtensorMap maps[kSlots];
+  static bool used[kSlots] = {false};
+  static int next = 0;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < kSlots; ++i)
+      if (used[i] && keys[i] == key) {
+        *m = maps[i];
+        return true;
+      }
+  }
+  if (!encode(m)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  keys[next] = key;
+  maps[next] = *m;
+  used[next] = true;
+  next = (next + 1) % kSlots;
+  return true;
+}
+
+bool encode_code_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
   auto enc = encode_fn();
   if (!enc) return false;
   const int64_t sh = arc->H > 1 ? arc->coeff_stride_h : arc->capacity * arc->S * arc->D;
@@ -1058,7 +1097,7 @@ bool make_code_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
 }
 
 // fp32 scales as a 3-d tensor {live rows, H, B}, boxes of 128 rows
-bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
+bool encode_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
   auto enc = encode_fn();
   if (!enc) return false;
   const int64_t sh = arc->H > 1 ? arc->scale_stride_h : arc->capacity * arc->S;
@@ -1070,6 +1109,18 @@ bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, arc->scales, dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_code_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
+  const MapKey key{arc->coeffs, rows, arc->H, arc->B, arc->H > 1 ? arc->coeff_stride_h : arc->capacity,
+                   arc->B > 1 ? arc->coeff_stride_b : arc->capacity, arc->D, 2 * arc->S};
+  return cached_map(m, key, [&](CUtensorMap* out) { return encode_code_map(out, arc, rows); });
+}
+
+bool make_scale_map(CUtensorMap* m, const fc_archive* arc, int64_t rows) {
+  const MapKey key{arc->scales, rows, arc->H, arc->B, arc->H > 1 ? arc->scale_stride_h : arc->capacity,
+                   arc->B > 1 ? arc->scale_stride_b : arc->capacity, arc->D, 2 * arc->S + 1};
+  return cached_map(m, key, [&](CUtensorMap* out) { return encode_scale_map(out, arc, rows); });
 }
 
 // CTAs of one problem: every kv head takes ns chunks
@@ -1087,8 +1138,20 @@ int launch(const TcBatch<NL>& batch, const Basis& full, const BasisF64& full64, 
   using C = Cfg<G, S, TPT>;
   const size_t smem = C::alloc;
   auto kern = decode_tc_kernel<G, S, TPT, NL>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-    return FC_ERR_CUDA;
+  // the attribute is a per-device property of the function: set once per
+  // device (a launch on another device sets it there)
+  static std::mutex attr_mu;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FC_ERR_CUDA;
+  {
+    std::lock_guard<std::mutex> lock(attr_mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return FC_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(unsigned(batch.cta_end[batch.n - 1]));
   cfg.blockDim = dim3(C::kThreads);
