@@ -371,6 +371,19 @@ extern "C" int fc_decode_step_host(const void* in_host, void* out_host, void* st
   const size_t qb = size_t(ka->B * Hq * ka->D) * esz;
   const int64_t tok_s[4] = {ka->H * ka->D, ka->D, ka->D, 1};
   const int64_t q_s[4] = {Hq * ka->D, ka->D, ka->D, 1};
+  // pinned host memory that the device can address (mapped, as every pinned
+  // allocation is under unified addressing): the kernels read the inputs and
+  // write the output there directly, and the copies happen inside them
+  cudaPointerAttributes pin{}, pout{};
+  if (cudaPointerGetAttributes(&pin, in_host) == cudaSuccess &&
+      cudaPointerGetAttributes(&pout, out_host) == cudaSuccess && pin.type == cudaMemoryTypeHost &&
+      pout.type == cudaMemoryTypeHost && pin.devicePointer && pout.devicePointer) {
+    const uint8_t* din = static_cast<const uint8_t*>(pin.devicePointer);
+    return fc_decode_step(din + 2 * tok, io_dtype, q_s, Hq, din, din + tok, io_dtype, tok_s, tok_s, ka, va, kt, vt,
+                          softmax_scale, num_splits, flags, workspace, workspace_bytes, pout.devicePointer,
+                          out_dtype, q_s, stream);
+  }
+  (void)cudaGetLastError();  // pageable memory: an unregistered pointer is not an error here
   // the host block is [k_new | v_new | q], each contiguous (B, heads, 1, D);
   // one copy when the staging offsets are contiguous too, else three
   const uint8_t* in = static_cast<const uint8_t*>(in_host);

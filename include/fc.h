@@ -316,11 +316,13 @@ int fc_decode_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int
 
 /*
  * fc_decode_step_host -- fc_decode_step fed from and returning to HOST
- * memory, for a serving loop whose tokens and queries arrive on the host:
- * one host-to-device copy of the step's inputs into `staging`, the fused
- * step, one device-to-host copy of the output, all on `stream` (pinned host
- * memory makes the copies asynchronous; the output is complete once
- * `stream` reaches the last copy).
+ * memory, for a serving loop whose tokens and queries arrive on the host.
+ * When both host buffers are pinned memory the device can address (every
+ * pinned allocation under unified addressing), the kernels read the inputs
+ * and write the output there directly; otherwise one host-to-device copy of
+ * the inputs into `staging`, the fused step and one device-to-host copy of
+ * the output are queued. All work is on `stream`; the output is complete
+ * once `stream` has reached it.
  *   in_host    host, the contiguous block [k_new | v_new | q]: k_new and
  *              v_new (B, H, 1, D), q (B, Hq, 1, D), each contiguous, of
  *              io_dtype (FC_DTYPE_BF16 or FC_DTYPE_F32, the tails' dtype).

@@ -224,10 +224,13 @@ def _dequant(stream, b, h):
     return oracle.dequantize(c, sc)
 
 
-def test_host_buffer_step_equals_device_step():
-    """fc_decode_step_host (inputs from one pinned host block, output to host
-    memory) gives the archive, tail and output of fc_decode_step on device
-    copies of the same inputs, across a block completion."""
+@pytest.mark.parametrize("pinned", [True, False], ids=["pinned", "pageable"])
+def test_host_buffer_step_equals_device_step(pinned):
+    """fc_decode_step_host (inputs from one host block, output to host
+    memory; pinned buffers are read and written by the kernels in place,
+    pageable ones go through the staging copies) gives the archive, tail and
+    output of fc_decode_step on device copies of the same inputs, across a
+    block completion."""
     w = synth.Workload("hstep", B=2, Hq=8, Hk=2, D=128, T=8 * 50 + 5, R=8,
                        S=2, seed=17, steps=6)
     data = synth.generate(w, q_steps=w.steps)
@@ -241,12 +244,13 @@ def test_host_buffer_step_equals_device_step():
     ws = host_cache.workspace(w.Hq, host_cache.num_splits(w.Hq))
     for s in range(w.steps):
         t = w.T + s
-        blk = torch.empty(2 * nk + nq, dtype=torch.bfloat16, pin_memory=True)
+        blk = torch.empty(2 * nk + nq, dtype=torch.bfloat16, pin_memory=pinned)
         blk[:nk] = data["k"][:, :, t].reshape(-1)
         blk[nk:2 * nk] = data["v"][:, :, t].reshape(-1)
         blk[2 * nk:] = data["q"][s].reshape(-1)
-        out_h = torch.empty((w.B, w.Hq, 1, w.D), pin_memory=True)
+        out_h = torch.empty((w.B, w.Hq, 1, w.D), pin_memory=pinned)
         _lib.HostStep(host_cache, w.Hq, blk, out_h, staging, ws)()
+        torch.cuda.synchronize()
         ref = dev_cache.step(data["q"][s].to(DEV),
                              data["k"][:, :, t:t + 1].to(DEV),
                              data["v"][:, :, t:t + 1].to(DEV))
