@@ -631,7 +631,7 @@ def run_fc(args, world, rank, local):
                        "fc_decode_step_layers launch per step against one "
                        "fc_decode_step launch per layer" % args.layers)
         res["layers"] = lay
-    if args.workloads:
+    if args.workloads and args.workloads != "none":
         wl = {}
         for name in args.workloads.split(","):
             if name and name != w.name:
@@ -792,7 +792,7 @@ def main(argv=None):
                     help="layer caches of the multi-layer leg (0 = skip)")
     ap.add_argument("--workloads", default="tiny,gqa,large,stream",
                     help="comma-separated further workloads whose decode "
-                         "attention is timed at full size ('' = none)")
+                         "attention is timed at full size ('none' = none)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -31,8 +31,9 @@
  *     updated only when the call returns FC_OK.
  *   - There is no fallback path: an unsupported shape or dtype is an error.
  *
- * Supported sizes: D in {32, 64, 128, 256}; 1 <= S <= R <= 32 and S <= 16;
- * Hq a multiple of Hk with G = Hq / Hk in {1, 2, 4, 8, 16}.
+ * Supported sizes: D in {32, 64, 128, 256}; 1 <= S <= R <= 32 and S <= 16
+ * (the PNG tier: S = R <= 16); Hq a multiple of Hk with G = Hq / Hk in
+ * {1, 2, 4, 8, 16}.
  */
 #ifndef FC_H_
 #define FC_H_
@@ -243,8 +244,11 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *              spin-waits: an atomic ticket); without it only the partials
  *              are written and fc_combine produces `out`.
  *              FC_DECODE_PORTABLE: use the portable CUDA-core kernel even
- *              where the tensor-core kernel applies (int8 K and V, D = 128,
- *              S dividing 32, R / S in {2, 4, 8}, G <= 8).
+ *              where the tensor-core kernel applies (DCT codec, int8 K and
+ *              V, D = 128, (S, R / S) in {(1, 4), (1, 8), (2, 4), (2, 8),
+ *              (4, 2), (4, 4), (8, 2)}, G in {1, 2, 4, 8} with
+ *              max(1, G / S) R <= 32, at least one archived block;
+ *              fc_decode_kernel reports the choice).
  *              FC_DECODE_OVERLAP (tensor-core kernel; ignored otherwise):
  *              launch as a programmatic dependent of the preceding work on
  *              `stream`. The kernel then streams archive blocks
