@@ -29,6 +29,7 @@ FC_DECODE_FUSE_COMBINE = 1
 FC_DECODE_PORTABLE = 2
 FC_DECODE_OVERLAP = 4
 FC_DECODE_Q_FINAL = 8
+FC_DECODE_TEST_TIMEOUT = 16
 
 FC_KERNEL_CUDA_CORE = 0
 FC_KERNEL_TENSOR_CORE = 1
@@ -292,14 +293,15 @@ def fc_decode_attention(q: torch.Tensor, ka: FcArchive, va: FcArchive,
                         softmax_scale: float = 0.0, num_splits: int = 0,
                         fuse_combine: bool = True, portable: bool = False,
                         overlap: bool = False, q_final: bool = False,
-                        stream=None) -> None:
+                        test_timeout: bool = False, stream=None) -> None:
     ws_ptr = _ptr(workspace)
     ws_bytes = 0 if workspace is None else workspace.numel() * \
         workspace.element_size()
     flags = (FC_DECODE_FUSE_COMBINE if fuse_combine else 0) | \
         (FC_DECODE_PORTABLE if portable else 0) | \
         (FC_DECODE_OVERLAP if overlap else 0) | \
-        (FC_DECODE_Q_FINAL if q_final else 0)
+        (FC_DECODE_Q_FINAL if q_final else 0) | \
+        (FC_DECODE_TEST_TIMEOUT if test_timeout else 0)
     st = load().fc_decode_attention(
         _ptr(q), dtype_code(q.dtype), _strides4(q), q.shape[1],
         ctypes.byref(ka), ctypes.byref(va), _ref(kt), _ref(vt),

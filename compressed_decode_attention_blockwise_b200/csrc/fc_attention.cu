@@ -124,11 +124,16 @@ int prepare_decode(const void* q, int32_t q_dtype, const int64_t* q_strides, int
   int ns = num_splits;
   if (ns == 0) ns = plan_splits(ka->n_blocks, ka->B, ka->H, ka->S, int(ka->D));
   if (ns < 1 || ns > kMaxSplits) return FC_ERR_INVALID;
-  if (flags & ~(FC_DECODE_FUSE_COMBINE | FC_DECODE_PORTABLE | FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL))
+  if (flags & ~(FC_DECODE_FUSE_COMBINE | FC_DECODE_PORTABLE | FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL |
+                FC_DECODE_TEST_TIMEOUT))
     return FC_ERR_INVALID;
   const bool fuse_combine = (flags & FC_DECODE_FUSE_COMBINE) != 0;
   if (ka->B > 65535 || ka->H > 65535) return FC_ERR_UNSUPPORTED;
   const bool need_ws = !(fuse_combine && ns == 1);
+  if (flags & FC_DECODE_TEST_TIMEOUT) {
+    if (!need_ws) return FC_ERR_INVALID;  // no status word to record the error in
+    if ((flags & FC_DECODE_PORTABLE) || !decode_tc_eligible(ka, va, int(G))) return FC_ERR_UNSUPPORTED;
+  }
   const WorkspaceLayout wl = workspace_layout(ka->B, Hq, ka->D, ns);
   if (need_ws) {
     if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
@@ -185,6 +190,7 @@ int prepare_decode(const void* q, int32_t q_dtype, const int64_t* q_strides, int
   a.fuse = fuse_combine ? 1 : 0;
   a.overlap = (flags & FC_DECODE_OVERLAP) ? 1 : 0;
   a.q_final = (a.overlap && (flags & FC_DECODE_Q_FINAL)) ? 1 : 0;
+  a.test_stall = (flags & FC_DECODE_TEST_TIMEOUT) ? 1 : 0;
   a.out = out;
   a.out_dtype = out_dtype;
   a.os_b = out_strides[0];
@@ -253,6 +259,7 @@ int prepare_step(const void* q, int32_t q_dtype, const int64_t* q_strides, int64
                  DecodeArgs* ap, bool* fused, bool* complete) {
   if (!k_new || !v_new || !k_strides || !v_strides || !kt || !vt || !kt->data || !vt->data)
     return FC_ERR_INVALID;
+  if (flags & FC_DECODE_TEST_TIMEOUT) return FC_ERR_INVALID;  // fc_decode_attention only
   DecodeArgs a;
   int st = prepare_decode(q, q_dtype, q_strides, Hq, ka, va, kt, vt, softmax_scale, num_splits, flags,
                           workspace, workspace_bytes, out, out_dtype, out_strides, true, &a);

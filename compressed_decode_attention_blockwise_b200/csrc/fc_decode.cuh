@@ -56,6 +56,7 @@ struct DecodeArgs {
   // bal_q + 1 chunks, the others bal_q (one CTA per SM in all); 0 = ns each
   int bal_q, bal_rem;
   int auto_split;  // num_splits was 0: ns is the planner's slot count
+  int test_stall;  // test hook: one wait that nothing ends, with a short limit
   float qscale;  // sigma * log2(e)
   uint32_t* status;
   uint32_t* tickets;

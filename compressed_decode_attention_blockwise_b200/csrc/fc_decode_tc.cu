@@ -64,6 +64,7 @@ constexpr int kD = 128;     // head dim served by this kernel
 constexpr uint32_t kTileBytes = kRows * kD;
 constexpr uint32_t kScaleBytes = kRows * 4;
 constexpr unsigned long long kWaitCycles = 4000000000ull;  // ~2 s at 2 GHz
+constexpr unsigned long long kStallCycles = 1ull << 20;     // the test hook's wait
 constexpr int kFinBar = 8;   // named barrier over every compute warp
 constexpr float kMagic = 12582912.f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
@@ -241,13 +242,14 @@ __device__ __forceinline__ float pick(const float (&v)[N], int i) {
 struct Waiter {
   int* abort;
   uint32_t* status;
+  unsigned long long limit;  // clock cycles
   __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity) {
     if (*reinterpret_cast<volatile int*>(abort)) return false;
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = clock64();
     while (!ptx::mbar_try_wait(bar, parity)) {
       if (*reinterpret_cast<volatile int*>(abort)) return false;
-      if (clock64() - t0 > kWaitCycles) {
+      if (clock64() - t0 > limit) {
         *reinterpret_cast<volatile int*>(abort) = 1;
         if (status) atomicOr(status, 1u);
         return false;
@@ -391,7 +393,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   }
   const int h = unit % a.Hk, b = unit / a.Hk;
   const int Hq = a.Hk * G;
-  Waiter waiter{abort_flag, a.status};
+  Waiter waiter{abort_flag, a.status, kWaitCycles};
 
   // chunks of ceil(tiles / ns_u) tiles: the last chunk, which also folds
   // in the raw tail, gets what is left (at most as many tiles as the others)
@@ -560,17 +562,17 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       }
       __nanosleep(32);
     }
-    // after an abort, the newest load of every stage must land before the
-    // CTA exits (older ones completed before their stage was reissued)
-    if (*reinterpret_cast<volatile int*>(abort_flag)) {
-      for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
-      for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
-    }
   }
+  int mk = 0, mv = 0;  // tiles whose K-side / V-side MMAs were issued
   if (kmma_warp && lane == 0) {
     // ================= K-MMA thread: S_int of each tile into its group's
     // TMEM buffer as soon as it lands
     waiter.wait(qready, 0u);
+    if (a.test_stall) {
+      // test hook: the next phase of qready, which nothing completes
+      Waiter stall{abort_flag, a.status, kStallCycles};
+      stall.wait(qready, 1u);
+    }
     int i = 0;
     for (; i < ntiles; ++i) {
       const int s = i % NKS, g = i % NG, k = i / NG, x = k & 1;
@@ -588,8 +590,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       ptx::mma_commit(&kfree[s]);
       ptx::mma_commit(&gq[x]);
     }
-    // after an abort, the MMAs already issued finish before TMEM is freed
-    if (i < ntiles && i > 0) drain_wait(&kfree[(i - 1) % NKS], uint32_t((i - 1) / NKS) & 1u);
+    mk = i;
   }
   if (vmma_warp && lane == 0) {
     // ================= V-MMA thread: Acc_int of each tile as soon as its W is
@@ -612,7 +613,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       ptx::mma_commit(&vfree[s]);
       ptx::mma_commit(&gq[6 + x]);
     }
-    if (i < ntiles && i > 0) drain_wait(&vfree[(i - 1) % NVS], uint32_t((i - 1) / NVS) & 1u);
+    mv = i;
   }
 
   // ================= compute groups
@@ -1011,6 +1012,21 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
+  // every wait that can give up lies before the barrier above, so the abort
+  // flag is final here (and the same for every thread). After an abort the
+  // newest load of every stage lands and the last MMAs of each side complete
+  // (a commit tracks all earlier MMAs of its thread) before the CTA frees
+  // its TMEM and exits; older loads completed before their stage was reissued.
+  if (*reinterpret_cast<volatile int*>(abort_flag)) {
+    if (tma_warp && lane == 0) {
+      for (int i = max(0, nk - NKS); i < nk; ++i) drain_wait(&kfull[i % NKS], uint32_t(i / NKS) & 1u);
+      for (int i = max(0, nv - NVS); i < nv; ++i) drain_wait(&vfull[i % NVS], uint32_t(i / NVS) & 1u);
+    }
+    if (kmma_warp && lane == 0 && mk > 0) drain_wait(&kfree[(mk - 1) % NKS], uint32_t((mk - 1) / NKS) & 1u);
+    if (vmma_warp && lane == 0 && mv > 0) drain_wait(&vfree[(mv - 1) % NVS], uint32_t((mv - 1) / NVS) & 1u);
+    ptx::tc_fence_before();
+    __syncthreads();
+  }
   if (kmma_warp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);

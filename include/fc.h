@@ -64,7 +64,8 @@ enum {
   FC_DECODE_FUSE_COMBINE = 1, /* the last CTA of each kv head writes `out` */
   FC_DECODE_PORTABLE = 2,     /* force the portable CUDA-core kernel */
   FC_DECODE_OVERLAP = 4,      /* start before the preceding stream work ends */
-  FC_DECODE_Q_FINAL = 8       /* with OVERLAP: q was final before that work began */
+  FC_DECODE_Q_FINAL = 8,      /* with OVERLAP: q was final before that work began */
+  FC_DECODE_TEST_TIMEOUT = 16 /* test hook: make one device wait run out */
 };
 
 /* Codecs (fc_archive.codec). */
@@ -270,6 +271,20 @@ size_t fc_decode_workspace_bytes(int64_t B, int64_t Hq, int64_t D,
  *              work completes; it still waits before block n_blocks - 1,
  *              the tails, the workspace and `out`. Ignored without
  *              FC_DECODE_OVERLAP.
+ *              FC_DECODE_TEST_TIMEOUT (fc_decode_attention only; a test
+ *              hook for the error path): every CTA of the tensor-core
+ *              kernel makes one wait on a barrier phase that nothing
+ *              completes, with a limit of about 2^20 clock cycles instead
+ *              of the usual ~2 s. The wait runs out, the CTA records the
+ *              error in the workspace status word, stops issuing loads and
+ *              MMAs, drains the ones in flight, frees its TMEM and returns;
+ *              the tickets still return to zero, so the workspace serves
+ *              the next call. The call returns FC_OK (the launch worked);
+ *              fc_workspace_status then reports FC_ERR_DEVICE and `out` is
+ *              unspecified. FC_ERR_UNSUPPORTED where the tensor-core kernel
+ *              does not apply (or with FC_DECODE_PORTABLE); FC_ERR_INVALID
+ *              with FC_DECODE_FUSE_COMBINE and a single split (no
+ *              workspace, so no status word).
  *   workspace       device, >= fc_decode_workspace_bytes(B, Hq, D, splits)
  *                   bytes, 256-byte aligned. Its first 256 + 4*B*Hq bytes
  *                   (status word and tickets) must be zero before the first

@@ -172,6 +172,7 @@ def test_decode_step_validates_without_launching():
     assert step(k_new=None) == _lib.FC_ERR_INVALID
     assert step(kt_=None) == _lib.FC_ERR_INVALID
     assert step(flags=1 << 8) == _lib.FC_ERR_INVALID
+    assert step(flags=1 | _lib.FC_DECODE_TEST_TIMEOUT) == _lib.FC_ERR_INVALID
     assert step() == _lib.FC_ERR_CAPACITY        # the token completes block 3
     assert (ka.n_blocks, kt.len, vt.len) == (2, 7, 7)
 
@@ -421,3 +422,27 @@ def test_decode_step_layers_validate_on_the_host():
     assert call([a, c]) == _lib.FC_ERR_UNSUPPORTED
     shared = layer(arcs=a[1][:2])
     assert call([a, shared]) == _lib.FC_ERR_INVALID
+
+
+def test_timeout_hook_validates_on_the_host():
+    """FC_DECODE_TEST_TIMEOUT needs the tensor-core kernel and a status word:
+    unsupported on the portable kernel and for archives the tensor-core
+    kernel does not serve, invalid for a fused single-split call (no
+    workspace)."""
+    lib = _lib.load()
+    q_str = (ctypes.c_int64 * 4)(32 * 128, 128, 128, 1)
+    tc = _arc(H=8, D=128, R=16, S=4, cap=64, nb=40)
+    narrow = _arc(H=8, D=64, R=8, S=2, cap=64, nb=40)
+    T = _lib.FC_DECODE_TEST_TIMEOUT
+
+    def attn(ka, ns, flags):
+        return lib.fc_decode_attention(
+            FAKE, _lib.FC_DTYPE_BF16, q_str, 32, ctypes.byref(ka),
+            ctypes.byref(ka), None, None, 0.0, ns, flags, FAKE, 1 << 30,
+            FAKE, _lib.FC_DTYPE_F32, q_str, None)
+
+    assert attn(tc, 1, _lib.FC_DECODE_FUSE_COMBINE | T) == _lib.FC_ERR_INVALID
+    assert attn(tc, 2, _lib.FC_DECODE_FUSE_COMBINE | _lib.FC_DECODE_PORTABLE
+                | T) == _lib.FC_ERR_UNSUPPORTED
+    assert attn(narrow, 2, _lib.FC_DECODE_FUSE_COMBINE | T) == \
+        _lib.FC_ERR_UNSUPPORTED
