@@ -228,6 +228,106 @@ __global__ void __launch_bounds__(kViewThreads, view_ctas_per_sm<TC, VEC, MAXS>(
   }
 }
 
+// The view of an int8 archive in the common geometry (D = 128, R = 8 or 16,
+// whole blocks, output rows contiguous: row stride D) with S and R fixed at
+// compile time. The row loop is unrolled, so every basis entry M[j][t] is an
+// FMA operand at a fixed offset of the kernel's parameters and every store
+// an immediate offset from the item's output pointer. Warp w takes the
+// contiguous item range [w * per, (w + 1) * per) and walks (b, h, block) by
+// counters (no divisions inside the loop), loading the next block's codes
+// and scales before it writes the current block's R rows; the first B * H
+// warps also copy one (b, h) raw tail each.
+template <int S>
+constexpr int view_rows_ctas_per_sm() {
+  return S >= 4 ? 3 : 4;  // registers: S coefficient rows of 4 values besides the output rows
+}
+
+template <typename TO, int S, int R>
+__global__ void __launch_bounds__(kViewThreads, view_rows_ctas_per_sm<S>())
+    read_view_rows_kernel(ViewArgs a, Basis basis) {
+  constexpr int VEC = 4, D = 128;
+  const int lane = threadIdx.x & 31;
+  const uint32_t nw = gridDim.x * kViewWarps;
+  const uint32_t gw = blockIdx.x * kViewWarps + (threadIdx.x >> 5);
+  const uint32_t H = uint32_t(a.H), count = uint32_t(a.count);
+  if (gw < uint32_t(a.tail_items)) {
+    const uint32_t b = gw / H, h = gw - b * H;
+    TO* op = static_cast<TO*>(a.out) + b * a.os_b + h * a.os_h + a.tail_row0 * D + lane * VEC;
+    const int64_t tbase = b * a.ts_b + h * a.ts_h + lane * VEC;
+    for (int r = 0; r < a.tail_len; ++r) {
+      float x[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) x[v] = load_any(a.tail, tbase + int64_t(r) * D + v, a.tail_dtype);
+      store_out<TO, VEC>(op + r * D, x);
+    }
+  }
+  const uint32_t items = uint32_t(a.block_items);
+  const uint32_t per = (items + nw - 1) / nw;
+  uint32_t i = gw * per;
+  const uint32_t iend = min(i + per, items);
+  if (i >= iend) return;
+  uint32_t bh = i / count;
+  uint32_t n = i - bh * count;
+  uint32_t b = bh / H, h = bh - b * H;
+  const int8_t* cp;
+  const float* sp;
+  TO* op;
+  auto locate = [&]() {
+    const int64_t blk = a.first + n;
+    cp = static_cast<const int8_t*>(a.coeffs) + b * a.cs_b + h * a.cs_h + blk * (S * D) + lane * VEC;
+    sp = a.scales + b * a.ss_b + h * a.ss_h + blk * S;
+    op = static_cast<TO*>(a.out) + b * a.os_b + h * a.os_h + (a.out_row0 + int64_t(n) * R) * D + lane * VEC;
+  };
+  locate();
+  RawRow<int8_t, VEC> raw[S];
+  float sc[S];
+#pragma unroll
+  for (int j = 0; j < S; ++j) {
+    raw[j].load(cp + j * D);
+    sc[j] = __ldg(sp + j);
+  }
+  for (; i < iend; ++i) {
+    float c[S][VEC];
+#pragma unroll
+    for (int j = 0; j < S; ++j) {
+      raw[j].to_float(c[j]);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) c[j][v] *= sc[j];
+    }
+    TO* o = op;
+    if (i + 1 < iend) {
+      if (++n == count) {
+        n = 0;
+        if (++h == H) {
+          h = 0;
+          ++b;
+        }
+        locate();
+      } else {
+        cp += S * D;
+        sp += S;
+        op += R * D;
+      }
+#pragma unroll
+      for (int j = 0; j < S; ++j) {
+        raw[j].load(cp + j * D);
+        sc[j] = __ldg(sp + j);
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < R; ++t) {
+      float x[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) x[v] = basis.m[0][t] * c[0][v];
+#pragma unroll
+      for (int j = 1; j < S; ++j)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) x[v] = fmaf(basis.m[j][t], c[j][v], x[v]);
+      store_out<TO, VEC>(o + t * D, x);
+    }
+  }
+}
+
 // ------------------------------------------------------------- batch gather
 
 struct GatherIndex {
@@ -317,12 +417,52 @@ int launch_view_as(const ViewArgs& a, const Basis& basis, int64_t total, fc_stre
 // Launches the view kernel for `a` (items already counted). Grid: enough
 // warps for every item, at most one wave of resident CTAs (a grid-stride
 // loop covers the rest).
+template <typename TO, int S, int R>
+int launch_view_rows(const ViewArgs& a, const Basis& basis, int64_t total, fc_stream stream) {
+  int64_t grid = (total + kViewWarps - 1) / kViewWarps;
+  const int64_t cap = int64_t(sm_count()) * view_rows_ctas_per_sm<S>();
+  if (grid > cap) grid = cap;
+  read_view_rows_kernel<TO, S, R><<<unsigned(grid), kViewThreads, 0, stream>>>(a, basis);
+  return cuda_status(cudaGetLastError());
+}
+
+// the unrolled kernel for int8, D = 128, whole blocks of R = 8 or 16 and
+// contiguous output rows; FC_ERR_UNSUPPORTED (nothing launched) otherwise
+template <typename TO>
+int try_view_rows(const ViewArgs& a, const Basis& basis, int64_t total, fc_stream stream) {
+  if (a.rows != a.R || a.os_t != 128) return FC_ERR_UNSUPPORTED;
+  if (a.tail_items && a.tail_len > a.R) return FC_ERR_UNSUPPORTED;
+  if (a.R == 8) {
+    switch (a.S) {
+      case 1: return launch_view_rows<TO, 1, 8>(a, basis, total, stream);
+      case 2: return launch_view_rows<TO, 2, 8>(a, basis, total, stream);
+      case 3: return launch_view_rows<TO, 3, 8>(a, basis, total, stream);
+      case 4: return launch_view_rows<TO, 4, 8>(a, basis, total, stream);
+      default: break;
+    }
+  } else if (a.R == 16) {
+    switch (a.S) {
+      case 2: return launch_view_rows<TO, 2, 16>(a, basis, total, stream);
+      case 4: return launch_view_rows<TO, 4, 16>(a, basis, total, stream);
+      case 8: return launch_view_rows<TO, 8, 16>(a, basis, total, stream);
+      default: break;
+    }
+  }
+  return FC_ERR_UNSUPPORTED;
+}
+
 int launch_view(const ViewArgs& a, int coeff_dtype, int out_dtype, int64_t D, fc_stream stream) {
   const int64_t total = a.block_items + a.tail_items;
   if (total == 0) return FC_OK;
   if (total >= (int64_t(1) << 31)) return FC_ERR_UNSUPPORTED;
   Basis basis;
   make_basis(a.codec, a.R, a.S, &basis);
+  if (coeff_dtype == FC_DTYPE_I8 && D == 128) {
+    const int st = out_dtype == FC_DTYPE_BF16 ? try_view_rows<__nv_bfloat16>(a, basis, total, stream)
+                   : out_dtype == FC_DTYPE_F32 ? try_view_rows<float>(a, basis, total, stream)
+                                               : FC_ERR_UNSUPPORTED;
+    if (st != FC_ERR_UNSUPPORTED) return st;
+  }
   return dispatch_coeff(coeff_dtype, [&](auto tc) {
     using TC = decltype(tc);
     return dispatch_view(out_dtype, [&](auto to) {

@@ -101,6 +101,8 @@ VIEW_CASES = [
     (2, 2, 32, 16, 12, "i8", "f32", 16 * 9 + 15),   # S > 8
     (1, 2, 256, 32, 16, "f32", "bf16", 32 * 5 + 1),
     (1, 3, 64, 4, 4, "bf16", "f32", 4 * 50),        # S = R, empty tail
+    (1, 4, 128, 8, 3, "i8", "f32", 8 * 33 + 2),     # unrolled rows, S = 3
+    (1, 2, 256, 16, 8, "i8", "bf16", 16 * 11 + 9),  # unrolled rows, D = 256
 ]
 
 
