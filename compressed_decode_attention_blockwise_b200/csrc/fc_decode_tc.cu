@@ -239,6 +239,19 @@ __device__ __forceinline__ float pick(const float (&v)[N], int i) {
   return r;
 }
 
+// The aligned 32-bit word that holds element `idx` of a bf16 or fp32 tensor
+// whose base and row strides are multiples of 16 bytes (the raw tails and a
+// fused step's new tokens; bf16: the pair the element belongs to), and the
+// element's value from that word given its column `col` in the row (the
+// parity of col and idx agree there).
+__device__ __forceinline__ const uint32_t* elem_word(const void* p, int64_t idx, bool f32) {
+  const char* c = static_cast<const char*>(p);
+  return reinterpret_cast<const uint32_t*>(f32 ? c + idx * 4 : c + (idx & ~int64_t(1)) * 2);
+}
+__device__ __forceinline__ float word_elem(uint32_t w, int col, bool f32) {
+  return __uint_as_float(f32 ? w : ((col & 1) ? (w & 0xffff0000u) : (w << 16)));
+}
+
 struct Waiter {
   int* abort;
   uint32_t* status;
@@ -860,37 +873,42 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
     // raw tail tokens, then the step's new token or block (last chunk)
     if (active && last_chunk && (a.nr > 0 || a.step != 0)) {
       float* red2 = reinterpret_cast<float*>(sm + C::xs) + grp * 4 * C::XW;
-      float qh[HPG];
-#pragma unroll
-      for (int y = 0; y < HPG; ++y) {
-        const int g = min(grp + NG * y, G - 1);
-        qh[y] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
-      }
       // the raw tokens of the tail, and the step's new token, in one batch:
       // one reduction over the group for every logit, then one online-softmax
       // update (thread t = channel d)
       const int n_raw = a.step == 2 ? 0 : a.nr;  // a completed block is folded coded
       const int n_tok = n_raw + (a.step == 1 ? 1 : 0);
       constexpr int kTok = S * TPT;  // at most R tokens: R - 1 tail rows + the new one
-      if (n_tok > 0) {
-        float kv[kTok], vv[kTok];
+      // every token's 32-bit words are requested first, before the query and
+      // before any is used (a conversion right behind each load would wait
+      // for it: one DRAM round trip per token), and converted where used
+      const bool f32 = a.t_dtype == FC_DTYPE_F32;
+      uint32_t kw[kTok], vw[kTok];
 #pragma unroll
-        for (int tt = 0; tt < kTok; ++tt) {
-          kv[tt] = 0.f;
-          vv[tt] = 0.f;
-          if (tt < n_raw) {
-            kv[tt] = load_any(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, a.t_dtype);
-            vv[tt] = load_any(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, a.t_dtype);
-          } else if (tt == n_raw && a.step == 1) {
-            kv[tt] = load_any(a.kn, b * a.kns_b + h * a.kns_h + t, a.t_dtype);
-            vv[tt] = load_any(a.vn, b * a.vns_b + h * a.vns_h + t, a.t_dtype);
-          }
+      for (int tt = 0; tt < kTok; ++tt) {
+        kw[tt] = 0u;
+        vw[tt] = 0u;
+        if (tt < n_raw) {
+          kw[tt] = __ldg(elem_word(a.kt, b * a.kts_b + h * a.kts_h + int64_t(tt) * kD + t, f32));
+          vw[tt] = __ldg(elem_word(a.vt, b * a.vts_b + h * a.vts_h + int64_t(tt) * kD + t, f32));
+        } else if (tt == n_raw && a.step == 1) {
+          kw[tt] = __ldg(elem_word(a.kn, b * a.kns_b + h * a.kns_h + t, f32));
+          vw[tt] = __ldg(elem_word(a.vn, b * a.vns_b + h * a.vns_h + t, f32));
         }
+      }
+      float qh[HPG];
+#pragma unroll
+      for (int y = 0; y < HPG; ++y) {
+        const int g = min(grp + NG * y, G - 1);
+        qh[y] = load_any(a.q, b * a.qs_b + (h * G + g) * a.qs_h + t, a.q_dtype) * a.qscale;
+      }
+      if (n_tok > 0) {
+        // all R reductions at once (unused tokens hold zeros)
         float lgt[kTok][HPG];
 #pragma unroll
         for (int tt = 0; tt < kTok; ++tt)
 #pragma unroll
-          for (int y = 0; y < HPG; ++y) lgt[tt][y] = tt < n_tok ? warp_sum(qh[y] * kv[tt]) : 0.f;
+          for (int y = 0; y < HPG; ++y) lgt[tt][y] = warp_sum(qh[y] * word_elem(kw[tt], t, f32));
         if (lane == 0) {
 #pragma unroll
           for (int tt = 0; tt < kTok; ++tt)
@@ -918,7 +936,7 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
             if (tt < n_tok) {
               const float p = ptx::ex2(lgt[tt][y] - mn);
               ps += p;
-              add = fmaf(p, vv[tt], add);
+              add = fmaf(p, word_elem(vw[tt], t, f32), add);
             }
           }
           Ah[y] = fmaf(Ah[y], al, add);
@@ -948,17 +966,23 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
           ksc[j] = __ldcg(ksp + j);
           vsc[j] = __ldcg(vsp + j);
         }
+        int kcode[S], vraw[S];  // requested together, converted after
+#pragma unroll
+        for (int j = 0; j < S; ++j) {
+          kcode[j] = __ldcg(kc + j * kD + t);
+          vraw[j] = __ldcg(vc + j * kD + t);
+        }
         float sj[S * HPG];
 #pragma unroll
         for (int j = 0; j < S; ++j) {
-          const float kv = float(__ldcg(kc + j * kD + t));
+          const float kv = float(kcode[j]);
 #pragma unroll
           for (int y = 0; y < HPG; ++y) sj[j * HPG + y] = kv * qh[y];
         }
         group_sum<S * HPG>(sj, red2, w, lane, 1 + grp);
         float vcode[S];
 #pragma unroll
-        for (int j = 0; j < S; ++j) vcode[j] = float(__ldcg(vc + j * kD + t));
+        for (int j = 0; j < S; ++j) vcode[j] = float(vraw[j]);
 #pragma unroll
         for (int y = 0; y < HPG; ++y) {
           float lg[S * TPT];
