@@ -128,8 +128,10 @@ constexpr int kStreamWarps = 8;  // warps per CTA of the pipelined compressor
 // of every row, so its own cp.async completion orders its reads. The
 // arithmetic is encode_block, unchanged: codes are bitwise those of the
 // unpipelined path and of the append kernel. The first B * H warps also copy
-// their (b, h)'s T mod R remaining tokens into the raw tail.
-template <int VEC, typename TIn, typename TOut, int NST>
+// their (b, h)'s T mod R remaining tokens into the raw tail. SC, RC > 0:
+// S and R fixed at compile time (encode_block's compile-time form, the same
+// codes).
+template <int VEC, typename TIn, typename TOut, int NST, int SC = 0, int RC = 0>
 __global__ void __launch_bounds__(kStreamWarps * 32, 2) compress_stream_kernel(CompressArgs a, BasisF64 basis) {
   extern __shared__ __align__(16) uint8_t csm[];
   constexpr int kLaneBytes = VEC * int(sizeof(TIn));
@@ -195,8 +197,9 @@ __global__ void __launch_bounds__(kStreamWarps * 32, 2) compress_stream_kernel(C
                 (a.slot0 + n) * a.S * a.D;
     float* scl = a.out.scales ? a.out.scales + b * a.out.ss_b + h * a.out.ss_h + (a.slot0 + n) * a.S
                               : nullptr;
-    encode_block<TOut, VEC>([&](int t, float (&xf)[VEC]) { load_vec_plain<TIn, VEC>(rows + t * a.D, xf); },
-                            a.R, a.S, a.D, lane, basis, blk, scl);
+    encode_block<TOut, VEC, SC, RC>(
+        [&](int t, float (&xf)[VEC]) { load_vec_plain<TIn, VEC>(rows + t * a.D, xf); }, a.R, a.S, a.D,
+        lane, basis, blk, scl);
     advance(cc);
   }
   cp_async_wait<0>();
@@ -415,6 +418,16 @@ extern "C" int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t*
             const int64_t g_tail = (copy_tail ? (arc->B * arc->H + kStreamWarps - 1) / kStreamWarps : 0);
             const unsigned grid_p = unsigned(g > g_tail ? g : g_tail);
             auto kern = nst == 3 ? compress_stream_kernel<VEC, TIn, TOut, 3> : compress_stream_kernel<VEC, TIn, TOut, 2>;
+            // the decode workloads' geometries (D = 128, bf16 tokens, three
+            // stages) with S and R fixed at compile time
+            if constexpr (VEC == 4 && std::is_same<TIn, __nv_bfloat16>::value &&
+                          !std::is_same<TOut, float>::value) {
+              if (nst == 3 && arc->codec == FC_CODEC_DCT) {
+                if (arc->S == 2 && arc->R == 8) kern = compress_stream_kernel<VEC, TIn, TOut, 3, 2, 8>;
+                if (arc->S == 3 && arc->R == 8) kern = compress_stream_kernel<VEC, TIn, TOut, 3, 3, 8>;
+                if (arc->S == 4 && arc->R == 16) kern = compress_stream_kernel<VEC, TIn, TOut, 3, 4, 16>;
+              }
+            }
             if (smem > 48 * 1024 &&
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
               return int(FC_ERR_CUDA);

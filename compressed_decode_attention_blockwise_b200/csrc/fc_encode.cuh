@@ -137,17 +137,22 @@ __device__ __forceinline__ void store_coeff_row(const double (&c)[VEC], int lane
 // Encodes the S kept frequencies of one block whose R token rows come from
 // `row_at(t, xf)` (VEC floats of row t for this lane), kJC frequencies per
 // pass, and stores them at `blk` (S x D elements) / `scl` (S floats).
-template <typename TOut, int VEC, typename RowAt, typename BasisT>
-__device__ __forceinline__ void encode_block(RowAt&& row_at, int R, int S, int D, int lane,
+// SC, RC > 0 fix S and R at compile time (the loops unroll, basis entries
+// become constant operands and the frequency guards fold away); the
+// arithmetic and its order are the same, so the codes are bitwise those of
+// the runtime-sized form.
+template <typename TOut, int VEC, int SC = 0, int RC = 0, typename RowAt, typename BasisT>
+__device__ __forceinline__ void encode_block(RowAt&& row_at, int R_, int S_, int D, int lane,
                                              const BasisT& basis, TOut* blk, float* scl) {
-  for (int j0 = 0; j0 < S; j0 += kJC) {
+  const int R = RC > 0 ? RC : R_;
+  const int S = SC > 0 ? SC : S_;
+  auto pass = [&](int j0) {
     double c[kJC][VEC];
 #pragma unroll
     for (int jj = 0; jj < kJC; ++jj)
 #pragma unroll
       for (int v = 0; v < VEC; ++v) c[jj][v] = 0.0;
-#pragma unroll 4
-    for (int t = 0; t < R; ++t) {
+    auto row = [&](int t) {
       float xf[VEC];
       row_at(t, xf);
       // one conversion per element (the conversion unit, not the fp64 FMAs,
@@ -163,12 +168,25 @@ __device__ __forceinline__ void encode_block(RowAt&& row_at, int R, int S, int D
           for (int v = 0; v < VEC; ++v) c[jj][v] = fma(m, xd[v], c[jj][v]);
         }
       }
+    };
+    if constexpr (RC > 0) {
+#pragma unroll
+      for (int t = 0; t < RC; ++t) row(t);
+    } else {
+#pragma unroll 4
+      for (int t = 0; t < R; ++t) row(t);
     }
 #pragma unroll
     for (int jj = 0; jj < kJC; ++jj) {
       const int j = j0 + jj;
       if (j < S) store_coeff_row<TOut, VEC>(c[jj], lane, blk + int64_t(j) * D, scl ? scl + j : nullptr);
     }
+  };
+  if constexpr (SC > 0) {
+#pragma unroll
+    for (int j0 = 0; j0 < SC; j0 += kJC) pass(j0);
+  } else {
+    for (int j0 = 0; j0 < S; j0 += kJC) pass(j0);
   }
 }
 

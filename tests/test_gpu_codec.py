@@ -86,33 +86,43 @@ def test_zero_block_stores_zero_scale_and_codes():
     _compare_stream(cache.k, f64(x))
 
 
-def test_append_matches_prefill_bitwise_and_is_causal():
-    w = synth.WORKLOADS["stream"].replace(B=2, T=8 * 40 + 3, steps=0, seed=5)
+@pytest.mark.parametrize("R,S,kc,vc", [(8, 2, "i8", "i8"), (16, 4, "i8", "i8"),
+                                       (8, 3, "i8", "bf16")])
+def test_append_matches_prefill_bitwise_and_is_causal(R, S, kc, vc):
+    # the prefill of these geometries runs the encoder with S and R fixed at
+    # compile time, the append its runtime-sized form: the codes must agree
+    w = synth.WORKLOADS["stream"].replace(B=2, T=R * 40 + 3, R=R, S=S,
+                                          k_coeff=kc, v_coeff=vc, steps=0,
+                                          seed=5)
     data = synth.generate(w, q_steps=0)
     k, v = data["k"].to(DEV), data["v"].to(DEV)
-    one = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV)
+    one = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, kc, vc, device=DEV)
     one.prefill(k, v)
-    inc = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, device=DEV)
+    inc = CodecKVCache(w.B, w.Hk, w.D, w.R, w.S, kc, vc, device=DEV)
     snap = None
     for t in range(w.T):
         inc.append(k[:, :, t:t + 1], v[:, :, t:t + 1])
-        if t == 8 * 20 + 2:  # 20 archived blocks
+        if t == R * 20 + 2:  # 20 archived blocks
             torch.cuda.synchronize()
-            snap = (inc.k.live_coeffs().clone(), inc.k.live_scales().clone(),
-                    inc.v.live_coeffs().clone(), inc.v.live_scales().clone())
+            snap = [(st.live_coeffs().clone(), st.live_scales())
+                    for st in (inc.k, inc.v)]
+            snap = [(c, None if sc is None else sc.clone()) for c, sc in snap]
     torch.cuda.synchronize()
     assert inc.k.n_blocks == one.k.n_blocks == 40
     assert inc.k.tail_len == one.k.tail_len == 3
     for a, b in ((inc.k, one.k), (inc.v, one.v)):
         assert torch.equal(a.live_coeffs(), b.live_coeffs())
-        assert torch.equal(a.live_scales(), b.live_scales())
+        if a.live_scales() is None:       # unquantised stream
+            assert b.live_scales() is None
+        else:
+            assert torch.equal(a.live_scales(), b.live_scales())
         assert torch.equal(a.live_tail(), b.live_tail())
     # archived blocks are never rewritten by later appends
-    nb0 = snap[0].shape[2]
-    assert torch.equal(inc.k.coeffs[:, :, :nb0], snap[0])
-    assert torch.equal(inc.k.scales[:, :, :nb0], snap[1])
-    assert torch.equal(inc.v.coeffs[:, :, :nb0], snap[2])
-    assert torch.equal(inc.v.scales[:, :, :nb0], snap[3])
+    for st, (c0, s0) in zip((inc.k, inc.v), snap):
+        nb0 = c0.shape[2]
+        assert torch.equal(st.coeffs[:, :, :nb0], c0)
+        if s0 is not None:
+            assert torch.equal(st.scales[:, :, :nb0], s0)
     # capacity doubled 16 -> 32 -> 64 along the way
     assert inc.k.capacity == 64
 
