@@ -712,7 +712,10 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       float vsc[S];  // V scales of my block
       load_floats<S>(scs + kRows + bt * S, vsc);
 
-      // logits of my items (basis entries are compile-time constant operands)
+      // logits of my items (basis entries are compile-time constant operands).
+      // The DCT rows are symmetric, A[R-1-t][j] = (-1)^j A[t][j], so the even-
+      // and odd-frequency parts of rows t < R/2 give both halves:
+      // logit_t = E_t + O_t, logit_{R-1-t} = E_t - O_t
       const bool live = tile * C::TB + bt < a.nb;
       float lg[NI][R];
       float mx[NI];
@@ -720,12 +723,19 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
       for (int ii = 0; ii < NI; ++ii) {
         float m = -INFINITY;
 #pragma unroll
-        for (int tk = 0; tk < R; ++tk) {
-          float v = basis.m[0][tk] * sb[ii][0];
+        for (int tk = 0; tk < R / 2; ++tk) {
+          float ev = basis.m[0][tk] * sb[ii][0];
 #pragma unroll
-          for (int q = 1; q < S; ++q) v = fmaf(basis.m[q][tk], sb[ii][q], v);
-          lg[ii][tk] = v;
-          m = fmaxf(m, v);
+          for (int q = 2; q < S; q += 2) ev = fmaf(basis.m[q][tk], sb[ii][q], ev);
+          float od = 0.f;
+          if constexpr (S > 1) {
+            od = basis.m[1][tk] * sb[ii][1];
+#pragma unroll
+            for (int q = 3; q < S; q += 2) od = fmaf(basis.m[q][tk], sb[ii][q], od);
+          }
+          lg[ii][tk] = ev + od;
+          lg[ii][R - 1 - tk] = ev - od;
+          m = fmaxf(m, fmaxf(lg[ii][tk], lg[ii][R - 1 - tk]));
         }
         m = live && own ? m : -INFINITY;
 #pragma unroll
@@ -778,12 +788,20 @@ __global__ void __launch_bounds__(Cfg<G, S, TPT>::kThreads, 1)
         }
         lsum[ii] = fmaf(lsum[ii], pick(alpha, hh), ps);
         const float wi = pick(winv, hh);
+        // w_j = sum_t p_t A[t][j] over the symmetric halves: with
+        // u_t = p_t + p_{R-1-t} (even j) or p_t - p_{R-1-t} (odd j), t < R/2
+        float pa[R / 2], pd[R / 2];
+#pragma unroll
+        for (int tk = 0; tk < R / 2; ++tk) {
+          pa[tk] = p[tk] + p[R - 1 - tk];
+          pd[tk] = p[tk] - p[R - 1 - tk];
+        }
         uint32_t by[3][S];
 #pragma unroll
         for (int q = 0; q < S; ++q) {
-          float wq = p[0] * basis.m[q][0];
+          float wq = ((q & 1) ? pd[0] : pa[0]) * basis.m[q][0];
 #pragma unroll
-          for (int tk = 1; tk < R; ++tk) wq = fmaf(p[tk], basis.m[q][tk], wq);
+          for (int tk = 1; tk < R / 2; ++tk) wq = fmaf((q & 1) ? pd[tk] : pa[tk], basis.m[q][tk], wq);
           limb_bytes(wq * vsc[q] * wi, by[0][q], by[1][q], by[2][q]);
         }
 #pragma unroll
