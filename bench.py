@@ -292,8 +292,8 @@ def bench_layers(w, kd, vd, q_pool, dev, W, world, n_layers=8,
                  n_steps=16):
     """Decode steps of n_layers independent layer caches of the workload:
     one fc_decode_step_layers launch per step against n_layers separate
-    fc_decode_step launches (plain, and with the overlap flags). CUDA graphs
-    of n_steps steps; microseconds per layer-step."""
+    fc_decode_step launches, each plain and with the overlap flags. CUDA
+    graphs of n_steps steps; microseconds per layer-step."""
     from compressed_decode_attention_blockwise_b200 import (
         CodecKVCache, decode_step_layers)
     tok_dt = synth.torch_dtype(w.in_dtype)
@@ -313,7 +313,8 @@ def bench_layers(w, kd, vd, q_pool, dev, W, world, n_layers=8,
                         device=dev) for _ in range(n_layers)]
     ev0, ev1 = torch.cuda.Event(True), torch.cuda.Event(True)
     res = {"layers": n_layers, "steps": n_steps}
-    modes = {"one_launch": None, "separate": (False, False),
+    modes = {"one_launch": (False, False), "separate": (False, False),
+             "one_launch_overlap_q_final": (True, True),
              "separate_overlap_q_final": (True, True)}
     for name, flags in modes.items():
         caches = make()
@@ -327,10 +328,11 @@ def bench_layers(w, kd, vd, q_pool, dev, W, world, n_layers=8,
                 t = w.T + s
                 q = q_pool[s % len(q_pool)]
                 kn, vn = kd[:, :, t:t + 1], vd[:, :, t:t + 1]
-                if flags is None:
+                if name.startswith("one_launch"):
                     decode_step_layers(caches, [q] * n_layers,
                                        [kn] * n_layers, [vn] * n_layers,
-                                       outs=outs)
+                                       outs=outs, overlap=flags[0],
+                                       q_final=flags[1])
                 else:
                     for l, c in enumerate(caches):
                         c.step(q, kn, vn, out=outs[l], overlap=flags[0],
@@ -624,12 +626,14 @@ def run_fc(args, world, rank, local):
         lay = bench_layers(w, kd, vd, q_pool, dev, W, world,
                            n_layers=args.layers)
         lay["peak"] = peak
-        for m in ("one_launch", "separate", "separate_overlap_q_final"):
+        for m in ("one_launch", "separate", "one_launch_overlap_q_final",
+                  "separate_overlap_q_final"):
             lay[m]["frac"] = round(lay[m]["GB_per_s"] / peak, 4)
         lay["note"] = ("decode steps (append + attention) of %d independent "
                        "layer caches of this workload: one "
                        "fc_decode_step_layers launch per step against one "
-                       "fc_decode_step launch per layer" % args.layers)
+                       "fc_decode_step launch per layer, each plain and with "
+                       "FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL" % args.layers)
         res["layers"] = lay
     if args.workloads and args.workloads != "none":
         wl = {}

@@ -385,6 +385,7 @@ def fc_decode_step_staging_bytes(B: int, H: int, Hq: int, D: int,
 def fc_decode_step_layers(qs, k_news, v_news, kas, vas, kts, vts, outs,
                           workspaces, softmax_scale: float = 0.0,
                           num_splits: int = 0, fuse_combine: bool = True,
+                          overlap: bool = False, q_final: bool = False,
                           stream=None) -> None:
     """One launch of the fused decode steps of len(qs) independent streams
     (per-layer tensors and descriptors in matching lists)."""
@@ -409,8 +410,9 @@ def fc_decode_step_layers(qs, k_news, v_news, kas, vas, kts, vts, outs,
     st = load().fc_decode_step_layers(
         n, arr, dtype_code(qs[0].dtype), dtype_code(k_news[0].dtype),
         dtype_code(outs[0].dtype), qs[0].shape[1], float(softmax_scale),
-        int(num_splits), FC_DECODE_FUSE_COMBINE if fuse_combine else 0,
-        _stream(stream, qs[0]))
+        int(num_splits), (FC_DECODE_FUSE_COMBINE if fuse_combine else 0) |
+        (FC_DECODE_OVERLAP if overlap else 0) |
+        (FC_DECODE_Q_FINAL if q_final else 0), _stream(stream, qs[0]))
     _check(st, "fc_decode_step_layers")
 
 

@@ -102,10 +102,12 @@ class CodecStream:
             new.n_blocks = self.arc.n_blocks if self.coeffs is not None else 0
         self.coeffs, self.scales, self.arc = coeffs, scales, new
 
-    def ensure_capacity(self, need_blocks: int):
+    def ensure_capacity(self, need_blocks: int) -> bool:
         cap = grown_capacity(int(self.arc.capacity), int(need_blocks))
         if cap != self.arc.capacity:
             self._alloc(cap)
+            return True
+        return False
 
     # -- views ---------------------------------------------------------------
     @property
@@ -288,9 +290,10 @@ class CodecKVCache:
     def seq_len(self) -> int:
         return self.k.seq_len
 
-    def _grow_to(self, need_blocks: int):
-        self.k.ensure_capacity(need_blocks)
-        self.v.ensure_capacity(need_blocks)
+    def _grow_to(self, need_blocks: int) -> bool:
+        """Grow both streams to hold need_blocks; True when they moved."""
+        grew = self.k.ensure_capacity(need_blocks)
+        return self.v.ensure_capacity(need_blocks) or grew
 
     # -- writes ------------------------------------------------------------
     def prefill(self, k: torch.Tensor, v: torch.Tensor):
@@ -326,9 +329,11 @@ class CodecKVCache:
              q_final: bool = False) -> torch.Tensor:
         """One decode step: append the (B, Hk, 1, D) token to both streams,
         then attend q over the updated cache (fc_decode_step: one launch on
-        the tensor-core path). Flags as in ``attention``."""
-        if self.k.tail_len + 1 == self.R:
-            self._grow_to(self.k.n_blocks + 1)
+        the tensor-core path). Flags as in ``attention``; a step that first
+        grows the archive (a copy kernel writes every block) runs without
+        the overlap flags, whose precondition that copy would break."""
+        if self.k.tail_len + 1 == self.R and self._grow_to(self.k.n_blocks + 1):
+            overlap = q_final = False
         Hq = q.shape[1]
         if out is None:
             out = torch.empty((self.B, Hq, 1, self.D), dtype=out_dtype,
@@ -504,16 +509,19 @@ class CodecKVCache:
 
 def decode_step_layers(caches, qs, k_news, v_news, outs=None,
                        softmax_scale: Optional[float] = None,
-                       out_dtype: torch.dtype = torch.float32):
+                       out_dtype: torch.dtype = torch.float32,
+                       overlap: bool = False, q_final: bool = False):
     """One decode step (append + attention) of every cache in ``caches`` in
     one launch (fc_decode_step_layers): cache i appends (k_news[i],
     v_news[i]) and attends qs[i]. The caches are independent streams of the
     same shape (the layers of a step whose queries are all known, or the
-    sequences of a serving batch). Returns the outputs."""
+    sequences of a serving batch). ``overlap`` / ``q_final`` as in
+    ``CodecKVCache.attention``, for a loop of such steps. Returns the
+    outputs."""
     n = len(caches)
     for c in caches:
-        if c.k.tail_len + 1 == c.R:
-            c._grow_to(c.k.n_blocks + 1)
+        if c.k.tail_len + 1 == c.R and c._grow_to(c.k.n_blocks + 1):
+            overlap = q_final = False   # a growth copy precedes the launch
     Hq = qs[0].shape[1]
     if outs is None:
         outs = [torch.empty((c.B, Hq, 1, c.D), dtype=out_dtype,
@@ -523,7 +531,8 @@ def decode_step_layers(caches, qs, k_news, v_news, outs=None,
         qs, k_news, v_news, [c.k.arc for c in caches],
         [c.v.arc for c in caches], [c.k.tail_desc for c in caches],
         [c.v.tail_desc for c in caches], outs, wss,
-        softmax_scale=0.0 if softmax_scale is None else float(softmax_scale))
+        softmax_scale=0.0 if softmax_scale is None else float(softmax_scale),
+        overlap=overlap, q_final=q_final)
     return outs
 
 

@@ -415,7 +415,7 @@ extern "C" int fc_decode_step_layers(int32_t n_layers, fc_layer_step* layers, in
                                      int32_t new_dtype, int32_t out_dtype, int64_t Hq, float softmax_scale,
                                      int32_t num_splits, int32_t flags, fc_stream stream) {
   if (n_layers < 1 || n_layers > FC_MAX_LAYERS || !layers) return FC_ERR_INVALID;
-  if (flags & (FC_DECODE_OVERLAP | FC_DECODE_Q_FINAL | FC_DECODE_PORTABLE)) return FC_ERR_INVALID;
+  if (flags & FC_DECODE_PORTABLE) return FC_ERR_INVALID;
   DecodeArgs args[FC_MAX_LAYERS];
   const fc_archive* kas[FC_MAX_LAYERS];
   const fc_archive* vas[FC_MAX_LAYERS];

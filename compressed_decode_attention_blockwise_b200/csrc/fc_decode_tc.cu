@@ -1299,7 +1299,7 @@ int launch_decode_tc_layers(int n, const DecodeArgs* d, const fc_archive* const*
   tc::TcBatch<FC_MAX_LAYERS> batch;
   for (int i = 0; i < n; ++i)
     if (!tc::fill_problem(&batch, i, d[i], ka[i], va[i])) return FC_ERR_CUDA;
-  return tc::dispatch(batch, d[0].G, d[0].S, d[0].R, basis, basis64, false, stream);
+  return tc::dispatch(batch, d[0].G, d[0].S, d[0].R, basis, basis64, d[0].overlap != 0, stream);
 }
 
 }  // namespace fc

@@ -382,8 +382,12 @@ int fc_decode_step_host(const void* in_host, void* out_host, void* staging,
  *              strides. No two layers share an archive, tail or workspace.
  *   q_dtype, new_dtype, out_dtype, Hq, softmax_scale, num_splits: as in
  *              fc_decode_step, shared by all layers.
- *   flags      FC_DECODE_FUSE_COMBINE or 0 (the overlap flags and
- *              FC_DECODE_PORTABLE are FC_ERR_INVALID).
+ *   flags      FC_DECODE_FUSE_COMBINE, FC_DECODE_OVERLAP and
+ *              FC_DECODE_Q_FINAL as in fc_decode_attention, for every layer
+ *              (with the overlap flags the launch is a programmatic dependent
+ *              of the preceding stream work, e.g. the previous step's
+ *              launch, under the same precondition); FC_DECODE_PORTABLE is
+ *              FC_ERR_INVALID.
  * Every layer must be a tensor-core fused step (int8 K and V, D = 128, the
  * sizes fc_decode_attention lists for that kernel) with the same G, S and
  * R, else FC_ERR_UNSUPPORTED; FC_ERR_CAPACITY for any layer leaves every

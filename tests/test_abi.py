@@ -417,7 +417,9 @@ def test_decode_step_layers_validate_on_the_host():
     assert call([a, b], n=0) == _lib.FC_ERR_INVALID
     assert call([a, b], n=_lib.FC_MAX_LAYERS + 1) == _lib.FC_ERR_INVALID
     assert call([a, b], flags=_lib.FC_DECODE_FUSE_COMBINE |
-                _lib.FC_DECODE_OVERLAP) == _lib.FC_ERR_INVALID
+                _lib.FC_DECODE_PORTABLE) == _lib.FC_ERR_INVALID
+    assert call([a, b], flags=_lib.FC_DECODE_FUSE_COMBINE |
+                _lib.FC_DECODE_TEST_TIMEOUT) == _lib.FC_ERR_INVALID
     c = layer(S=4, R=16)
     assert call([a, c]) == _lib.FC_ERR_UNSUPPORTED
     shared = layer(arcs=a[1][:2])

@@ -40,12 +40,17 @@ def _layers(w, tails, data):
     return caches, lens, k, v
 
 
-@pytest.mark.parametrize("name,tails,steps", [
-    ("long", (3, 14, 15, 7), 3),
-    ("gqa", (5, 6, 7, 0, 1, 2), 3),
+@pytest.mark.parametrize("name,tails,steps,overlap", [
+    ("long", (3, 14, 15, 7), 3, False),
+    ("gqa", (5, 6, 7, 0, 1, 2), 3, False),
+    ("long", (3, 14, 15, 7), 3, True),
 ])
 def test_layers_in_one_launch_match_per_layer_steps_and_oracle(name, tails,
-                                                              steps):
+                                                              steps, overlap):
+    # overlap: the layer launches of consecutive steps run as programmatic
+    # dependents with every query final up front (FC_DECODE_OVERLAP |
+    # FC_DECODE_Q_FINAL); pure scheduling, so the results are bitwise those
+    # of the plain per-layer steps
     w = synth.WORKLOADS[name]
     w = w.replace(T=(w.T // w.R) * w.R + w.R, steps=steps + w.R)
     data = synth.generate(w, q_steps=steps * len(tails))
@@ -54,21 +59,31 @@ def test_layers_in_one_launch_match_per_layer_steps_and_oracle(name, tails,
     L = len(tails)
     q = data["q"].to(DEV)
     G = w.G
+    all_outs = []
     for s in range(steps):
         qs = [q[s * L + l] for l in range(L)]
         kn = [k[:, :, lens[l] + s:lens[l] + s + 1] for l in range(L)]
         vn = [v[:, :, lens[l] + s:lens[l] + s + 1] for l in range(L)]
-        outs = decode_step_layers(one, qs, kn, vn)
+        outs = decode_step_layers(one, qs, kn, vn, overlap=overlap,
+                                  q_final=overlap)
+        all_outs.append(outs)
+    torch.cuda.synchronize()
+    for s in range(steps):
+        qs = [q[s * L + l] for l in range(L)]
+        kn = [k[:, :, lens[l] + s:lens[l] + s + 1] for l in range(L)]
+        vn = [v[:, :, lens[l] + s:lens[l] + s + 1] for l in range(L)]
+        outs = all_outs[s]
         refs = [per[l].step(qs[l], kn[l], vn[l]) for l in range(L)]
         torch.cuda.synchronize()
         for l in range(L):
-            a, b = one[l], per[l]
-            assert (a.k.n_blocks, a.k.tail_len) == (b.k.n_blocks,
-                                                    b.k.tail_len)
-            assert torch.equal(a.k.live_coeffs(), b.k.live_coeffs())
-            assert torch.equal(a.v.live_scales(), b.v.live_scales())
-            assert torch.equal(a.k.live_tail(), b.k.live_tail())
             assert torch.equal(outs[l], refs[l]), (s, l)
+    # after the last step every layer's streams equal the per-layer ones
+    for l in range(L):
+        a, b = one[l], per[l]
+        assert (a.k.n_blocks, a.k.tail_len) == (b.k.n_blocks, b.k.tail_len)
+        assert torch.equal(a.k.live_coeffs(), b.k.live_coeffs())
+        assert torch.equal(a.v.live_scales(), b.v.live_scales())
+        assert torch.equal(a.k.live_tail(), b.k.live_tail())
     # the last step of every layer against the oracle on its own archive
     s = steps - 1
     for l in range(L):
