@@ -132,7 +132,8 @@ constexpr int kStreamWarps = 8;  // warps per CTA of the pipelined compressor
 // S and R fixed at compile time (encode_block's compile-time form, the same
 // codes).
 template <int VEC, typename TIn, typename TOut, int NST, int SC = 0, int RC = 0>
-__global__ void __launch_bounds__(kStreamWarps * 32, 2) compress_stream_kernel(CompressArgs a, BasisF64 basis) {
+__global__ void __launch_bounds__(kStreamWarps * 32, (SC > 0 && NST == 2) ? 3 : 2)
+    compress_stream_kernel(CompressArgs a, BasisF64 basis) {
   extern __shared__ __align__(16) uint8_t csm[];
   constexpr int kLaneBytes = VEC * int(sizeof(TIn));
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -411,23 +412,32 @@ extern "C" int fc_compress_blocks(const void* x, int32_t x_dtype, const int64_t*
         constexpr int VEC = decltype(vec)::value;
         if constexpr (VEC * sizeof(TIn) >= 4) {
           if (pipelined) {
-            const size_t smem = size_t(kStreamWarps) * nst * stage_bytes;
+            size_t smem = size_t(kStreamWarps) * nst * stage_bytes;
             const int64_t need = (arc->B * arc->H * n_full + kStreamWarps - 1) / kStreamWarps;
-            const int64_t cap = int64_t(sm_count()) * (nst == 3 ? 2 : 1);  // one resident wave
-            const int64_t g = need < cap ? need : cap;
             const int64_t g_tail = (copy_tail ? (arc->B * arc->H + kStreamWarps - 1) / kStreamWarps : 0);
-            const unsigned grid_p = unsigned(g > g_tail ? g : g_tail);
             auto kern = nst == 3 ? compress_stream_kernel<VEC, TIn, TOut, 3> : compress_stream_kernel<VEC, TIn, TOut, 2>;
             // the decode workloads' geometries (D = 128, bf16 tokens, three
             // stages) with S and R fixed at compile time
+            int per_sm = nst == 3 ? 2 : 1;
             if constexpr (VEC == 4 && std::is_same<TIn, __nv_bfloat16>::value &&
                           !std::is_same<TOut, float>::value) {
+              // two stages, three CTAs per SM (more warps in flight)
               if (nst == 3 && arc->codec == FC_CODEC_DCT) {
-                if (arc->S == 2 && arc->R == 8) kern = compress_stream_kernel<VEC, TIn, TOut, 3, 2, 8>;
-                if (arc->S == 3 && arc->R == 8) kern = compress_stream_kernel<VEC, TIn, TOut, 3, 3, 8>;
-                if (arc->S == 4 && arc->R == 16) kern = compress_stream_kernel<VEC, TIn, TOut, 3, 4, 16>;
+                const int nst2 = 2;
+                bool fixed = true;
+                if (arc->S == 2 && arc->R == 8) kern = compress_stream_kernel<VEC, TIn, TOut, 2, 2, 8>;
+                else if (arc->S == 3 && arc->R == 8) kern = compress_stream_kernel<VEC, TIn, TOut, 2, 3, 8>;
+                else if (arc->S == 4 && arc->R == 16) kern = compress_stream_kernel<VEC, TIn, TOut, 2, 4, 16>;
+                else fixed = false;
+                if (fixed) {
+                  smem = size_t(kStreamWarps) * nst2 * stage_bytes;
+                  per_sm = 3;
+                }
               }
             }
+            const int64_t cap = int64_t(sm_count()) * per_sm;  // one resident wave
+            const int64_t g = need < cap ? need : cap;
+            const unsigned grid_p = unsigned(g > g_tail ? g : g_tail);
             if (smem > 48 * 1024 &&
                 cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
               return int(FC_ERR_CUDA);
