@@ -234,3 +234,51 @@ def test_failed_crop_leaves_both_streams_as_they_were(fake, monkeypatch):
     assert torch.all(c.k.tail == 3.0)
     with pytest.raises(ValueError):
         c.crop(1)
+
+
+def test_a_step_that_grows_the_archive_runs_without_the_overlap_flags(
+        fake, monkeypatch):
+    """FC_DECODE_OVERLAP lets the kernel stream archive blocks before the
+    preceding stream work has finished; a growth copy (which writes every
+    block of the new storage) right before the step would break that, so
+    the binding drops the flags for that one step, for single steps and for
+    the multi-layer launch."""
+    from compressed_decode_attention_blockwise_b200.archive import \
+        decode_step_layers
+    calls = []
+
+    def fake_step(q, k_new, v_new, ka, va, kt, vt, out, ws, softmax_scale=0.0,
+                  num_splits=0, fuse_combine=True, portable=False,
+                  overlap=False, q_final=False, stream=None):
+        calls.append((int(ka.capacity), overlap, q_final))
+        fake.fc_append_step(k_new, v_new, ka, va, kt, vt)
+
+    def fake_layers(qs, k_news, v_news, kas, vas, kts, vts, outs, wss,
+                    softmax_scale=0.0, num_splits=0, fuse_combine=True,
+                    overlap=False, q_final=False, stream=None):
+        calls.append((tuple(int(a.capacity) for a in kas), overlap, q_final))
+        for i in range(len(kas)):
+            fake.fc_append_step(k_news[i], v_news[i], kas[i], vas[i], kts[i],
+                                vts[i])
+
+    monkeypatch.setattr(_lib, "fc_decode_step", fake_step)
+    monkeypatch.setattr(_lib, "fc_decode_step_layers", fake_layers)
+    monkeypatch.setattr(_lib, "fc_decode_plan", lambda ka, kt, Hq: 1)
+    monkeypatch.setattr(_lib, "fc_decode_workspace_bytes",
+                        lambda B, Hq, D, ns: 1024)
+    c = _cache()                                    # R = 8
+    c.prefill(*_tokens(c, 8 * 16 + 6))              # 16 blocks fill capacity 16
+    assert c.k.capacity == 16
+    q = torch.zeros((c.B, 4, 1, c.D))
+    tok = _tokens(c, 1)
+    for _ in range(3):                              # the second completes block 17
+        c.step(q, *tok, overlap=True, q_final=True)
+    assert calls == [(16, True, True), (32, False, False), (32, True, True)]
+    calls.clear()
+    a, b = _cache(), _cache()
+    for x in (a, b):
+        x.prefill(*_tokens(x, 8 * 16 + 7))
+    for _ in range(2):                              # the first completes a block
+        decode_step_layers([a, b], [q, q], [tok[0]] * 2, [tok[1]] * 2,
+                           overlap=True, q_final=True)
+    assert calls == [((32, 32), False, False), ((32, 32), True, True)]
