@@ -103,6 +103,21 @@ __device__ __forceinline__ void store_bf16_row(__nv_bfloat16* p, const __nv_bflo
   }
 }
 
+// 1 / s for the quantiser (0 for s = 0) without an fp64 division: a
+// single-precision seed refined by two Newton steps r <- r + r (1 - s r),
+// accurate to about one fp64 ulp; scales outside the single-precision range
+// divide. Every encoder runs this same sequence, so their codes agree
+// bitwise; against the exact reciprocal a code can differ only where
+// c / s lies within ~1e-13 of a half-integer.
+__device__ __forceinline__ double quant_reciprocal(double s) {
+  if (s == 0.0) return 0.0;
+  if (!(s > 0x1p-120 && s < 0x1p120)) return 1.0 / s;
+  double r = double(__frcp_rn(float(s)));
+#pragma unroll
+  for (int k = 0; k < 2; ++k) r = fma(r, fma(-s, r, 1.0), r);
+  return r;
+}
+
 // Quantises (int8) or rounds (bf16 / f32) one coefficient row held in fp64
 // and stores it at `row` (D elements; lane owns VEC) and, for int8, its scale.
 template <typename TOut, int VEC>
@@ -113,8 +128,8 @@ __device__ __forceinline__ void store_coeff_row(const double (&c)[VEC], int lane
 #pragma unroll
     for (int v = 0; v < VEC; ++v) amax = fmax(amax, fabs(c[v]));
     amax = warp_max_d(amax);
-    const double scale = amax / 127.0;
-    const double inv = amax > 0.0 ? 1.0 / scale : 0.0;
+    const double scale = amax * (1.0 / 127.0);  // within two ulps of amax / 127
+    const double inv = quant_reciprocal(scale);
     int code[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) code[v] = max(-127, min(127, __double2int_rn(c[v] * inv)));
