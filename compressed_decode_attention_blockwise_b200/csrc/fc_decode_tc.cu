@@ -142,6 +142,7 @@ struct TcBasis {
 template <int S, int R>
 struct Basis64View {  // encode_block indexes basis.m[j][t]
   const double (&m)[S][R];
+  static constexpr int32_t mirror = R % 2 == 0 ? 1 : 0;  // the DCT rows
 };
 
 __device__ __forceinline__ float pow2i(int e) {

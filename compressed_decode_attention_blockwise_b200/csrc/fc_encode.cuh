@@ -155,18 +155,42 @@ __device__ __forceinline__ void store_coeff_row(const double (&c)[VEC], int lane
 // SC, RC > 0 fix S and R at compile time (the loops unroll, basis entries
 // become constant operands and the frequency guards fold away); the
 // arithmetic and its order are the same, so the codes are bitwise those of
-// the runtime-sized form.
+// the runtime-sized form. For mirror-symmetric rows (the DCT with an even R:
+// m[j][R-1-t] = (-1)^j m[j][t]) the sum runs over t < R/2 on
+// u_t = x_t + x_{R-1-t} (even j) or w_t = x_t - x_{R-1-t} (odd j), formed in
+// fp64: half the multiply-adds, the same value up to fp64 rounding.
 template <typename TOut, int VEC, int SC = 0, int RC = 0, typename RowAt, typename BasisT>
 __device__ __forceinline__ void encode_block(RowAt&& row_at, int R_, int S_, int D, int lane,
                                              const BasisT& basis, TOut* blk, float* scl) {
   const int R = RC > 0 ? RC : R_;
   const int S = SC > 0 ? SC : S_;
+  const bool mirror = basis.mirror != 0;
   auto pass = [&](int j0) {
     double c[kJC][VEC];
 #pragma unroll
     for (int jj = 0; jj < kJC; ++jj)
 #pragma unroll
       for (int v = 0; v < VEC; ++v) c[jj][v] = 0.0;
+    auto pair = [&](int t) {  // rows t and R-1-t folded (mirror rows)
+      float xa[VEC], xb[VEC];
+      row_at(t, xa);
+      row_at(R - 1 - t, xb);
+      double u[VEC], w[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) {
+        const double da = double(xa[v]), db = double(xb[v]);
+        u[v] = da + db;
+        w[v] = da - db;
+      }
+#pragma unroll
+      for (int jj = 0; jj < kJC; ++jj) {
+        if (j0 + jj < S) {
+          const double m = basis.m[j0 + jj][t];
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) c[jj][v] = fma(m, ((j0 + jj) & 1) ? w[v] : u[v], c[jj][v]);
+        }
+      }
+    };
     auto row = [&](int t) {
       float xf[VEC];
       row_at(t, xf);
@@ -185,8 +209,16 @@ __device__ __forceinline__ void encode_block(RowAt&& row_at, int R_, int S_, int
       }
     };
     if constexpr (RC > 0) {
+      if (mirror) {
 #pragma unroll
-      for (int t = 0; t < RC; ++t) row(t);
+        for (int t = 0; t < RC / 2; ++t) pair(t);
+      } else {
+#pragma unroll
+        for (int t = 0; t < RC; ++t) row(t);
+      }
+    } else if (mirror) {
+#pragma unroll 2
+      for (int t = 0; t < R / 2; ++t) pair(t);
     } else {
 #pragma unroll 4
       for (int t = 0; t < R; ++t) row(t);

@@ -50,6 +50,7 @@ void make_basis_f64(int codec, int R, int S, BasisF64* out) {
       if (j < S && t < R) v = codec == FC_CODEC_PNG ? png_encode_entry(j, t) : dct_entry(R, j, t);
       out->m[j][t] = v;
     }
+  out->mirror = codec == FC_CODEC_DCT && R % 2 == 0 ? 1 : 0;
 }
 
 int sm_count() {

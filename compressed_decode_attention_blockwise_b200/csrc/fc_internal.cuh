@@ -28,6 +28,9 @@ void make_basis(int codec, int R, int S, Basis* out);
 // take the quantiser's rounding decision in fp64).
 struct BasisF64 {
   double m[kMaxS][kMaxR];
+  // 1 when row j is (-1)^j-symmetric, m[j][R-1-t] = (-1)^j m[j][t] (the DCT
+  // with an even R): the encoder then folds the mirror rows first
+  int32_t mirror;
 };
 // Host: the encoding rows of the codec in fp64 (the DCT rows; for the PNG
 // tier the anchor row and the first differences).
