@@ -378,6 +378,15 @@ extern "C" int fc_decode_step_host(const void* in_host, void* out_host, void* st
   const size_t qb = size_t(ka->B * Hq * ka->D) * esz;
   const int64_t tok_s[4] = {ka->H * ka->D, ka->D, ka->D, 1};
   const int64_t q_s[4] = {Hq * ka->D, ka->D, ka->D, 1};
+  {
+    // every argument is checked before any copy or kernel is queued
+    DecodeArgs chk;
+    bool fused = false, complete = false;
+    st = prepare_step(sg + L.q, io_dtype, q_s, Hq, sg + L.k, sg + L.v, io_dtype, tok_s, tok_s, ka, va, kt, vt,
+                      softmax_scale, num_splits, flags, workspace, workspace_bytes, sg + L.out, out_dtype, q_s,
+                      &chk, &fused, &complete);
+    if (st != FC_OK) return st;
+  }
   // pinned host memory that the device can address (mapped, as every pinned
   // allocation is under unified addressing): the kernels read the inputs and
   // write the output there directly, and the copies happen inside them

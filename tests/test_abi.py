@@ -448,3 +448,47 @@ def test_timeout_hook_validates_on_the_host():
                 | T) == _lib.FC_ERR_UNSUPPORTED
     assert attn(narrow, 2, _lib.FC_DECODE_FUSE_COMBINE | T) == \
         _lib.FC_ERR_UNSUPPORTED
+
+
+def test_host_step_sizes_and_validates_before_queuing_anything():
+    """fc_decode_step_staging_bytes is host arithmetic (three 256-byte
+    aligned input slots and the output slot); fc_decode_step_host rejects
+    bad arguments before it queues a copy or a kernel, so these calls return
+    on a machine without a GPU."""
+    lib = _lib.load()
+    B, H, Hq, D = 2, 8, 32, 128
+    tok, q, out = B * H * D * 2, B * Hq * D * 2, B * Hq * D * 4
+    pad = lambda n: (n + 255) // 256 * 256
+    need = lib.fc_decode_step_staging_bytes(B, H, Hq, D, _lib.FC_DTYPE_BF16,
+                                            _lib.FC_DTYPE_F32)
+    assert need == 2 * pad(tok) + pad(q) + pad(out)
+    assert lib.fc_decode_step_staging_bytes(B, H, Hq, D, _lib.FC_DTYPE_I8,
+                                            _lib.FC_DTYPE_F32) == 0
+    assert lib.fc_decode_step_staging_bytes(0, H, Hq, D, _lib.FC_DTYPE_BF16,
+                                            _lib.FC_DTYPE_F32) == 0
+    ka = _arc(B=B, H=H, D=D, R=16, S=4, cap=64, nb=40)
+    va = _arc(B=B, H=H, D=D, R=16, S=4, cap=64, nb=40)
+    kt, vt = _tail(ka, 3), _tail(va, 3)
+
+    def call(staging=FAKE * 16, nbytes=need, flags=_lib.FC_DECODE_FUSE_COMBINE,
+             in_host=FAKE, io=_lib.FC_DTYPE_BF16):
+        return lib.fc_decode_step_host(
+            in_host, FAKE, staging, nbytes, io, _lib.FC_DTYPE_F32, Hq,
+            ctypes.byref(ka), ctypes.byref(va), ctypes.byref(kt),
+            ctypes.byref(vt), 0.0, 0, flags, FAKE * 16, 1 << 30, None)
+
+    assert call(in_host=None) == _lib.FC_ERR_INVALID
+    assert call(staging=FAKE * 16 + 16) == _lib.FC_ERR_INVALID   # 256-byte aligned
+    assert call(nbytes=need - 1) == _lib.FC_ERR_INVALID
+    assert call(io=_lib.FC_DTYPE_I8) == _lib.FC_ERR_INVALID
+    assert call(flags=1 << 8) == _lib.FC_ERR_INVALID
+    assert call(flags=_lib.FC_DECODE_FUSE_COMBINE |
+                _lib.FC_DECODE_TEST_TIMEOUT) == _lib.FC_ERR_INVALID
+    ka.n_blocks = ka.capacity = 40                 # the token would complete
+    kt.len = vt.len = 15                           # a block with no room
+    ka.coeff_stride_h = 40 * 4 * D
+    ka.coeff_stride_b = H * ka.coeff_stride_h
+    ka.scale_stride_h = 40 * 4
+    ka.scale_stride_b = H * ka.scale_stride_h
+    assert call() == _lib.FC_ERR_CAPACITY
+    assert (ka.n_blocks, kt.len) == (40, 15)
