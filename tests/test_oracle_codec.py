@@ -44,6 +44,26 @@ def test_basis_rows_orthonormal(R, S):
     np.testing.assert_array_equal(codec.synthesis_basis(R, S), M.T)
 
 
+@pytest.mark.parametrize("R", [2, 4, 8, 16, 32])
+def test_basis_rows_are_mirror_symmetric(R):
+    """M[j, R-1-n] = (-1)^j M[j, n] (cos(pi j - x) = (-1)^j cos x): the
+    identity behind the device encoder's and attention kernel's folded sums
+    (rows t < R/2 on x_t + x_{R-1-t} for even j, x_t - x_{R-1-t} for odd j).
+    Checked against scipy's DCT-II matrix, and the folded coefficients
+    against the plain product on random blocks."""
+    M = scipy.fft.dct(np.eye(R), type=2, norm="ortho", axis=0)   # (R, R)
+    sign = (-1.0) ** np.arange(R)[:, None]
+    np.testing.assert_allclose(M[:, ::-1], sign * M, atol=1e-15)
+    ours = codec.dct_basis(R, R)
+    np.testing.assert_allclose(ours[:, ::-1], sign * ours, atol=1e-15)
+    x = np.random.default_rng(R).standard_normal((R, 7))
+    h = R // 2
+    u, w = x[:h] + x[::-1][:h], x[:h] - x[::-1][:h]
+    folded = np.where(np.arange(R)[:, None] % 2 == 0, ours[:, :h] @ u,
+                      ours[:, :h] @ w)
+    np.testing.assert_allclose(folded, ours @ x, atol=1e-13)
+
+
 def test_constant_block_has_only_dc():
     R, S, D = 8, 4, 3
     x = np.array([1.5, -2.0, 0.25])
