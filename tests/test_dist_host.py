@@ -72,3 +72,29 @@ def test_single_process_defaults(monkeypatch):
     assert bench.dist_env() == (1, 0, 0)
     assert bench.max_over_ranks(3.5, 1) == 3.5
     assert bench.whole_job_gbs(2e9, 1, 1.0) == pytest.approx(2.0)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """``bench.py --impl reference`` (the oracle timed on the host cores on a
+    bounded sample of the workload) prints one JSON line with the keys the
+    benchmark contract names, on a machine without a GPU."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"),
+                        "--impl", "reference", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup",
+                "ms_per_step", "higher_is_better", "scaling", "vs_baseline",
+                "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["n_gpus"] == 1
+    assert d["value"] > 0 and d["config"]["workload"] == "long"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"]
+    assert cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"],
+                        "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
